@@ -1,0 +1,361 @@
+#!/usr/bin/env python
+"""Throughput of the B200 Muon / Dimuon step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload large_batch|gpt2_small|square1024|lora_r2|lora_r8|lora_r32]
+
+One step = one optimizer step (momentum, normalisation, five Newton-Schulz
+iterations, scale, decay, apply) over every matrix of the workload.  The
+default workload is the large batch: 8 x 4096^2, 4 x 4096x14336 and
+4 x 14336x4096 bf16 matrices (tall ones orthogonalised on their short side),
+Muon mode, bf16 tensor-core products with fp32 accumulation.
+
+Each rank runs its own copy of the workload on its own GPU (independent
+problems, no collective on the data path): weak scaling; `value` counts the
+matrices of all ranks.  Rank 0 prints one JSON line.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "Muon/Dimuon step matrices/s and NS5 TFLOP/s on B200 (% of bf16 / HBM roofline)"
+
+
+def workload_spec(name):
+    if name == "large_batch":
+        return dict(shapes=workloads.large_batch_shapes(), cond=False, mdt="bf16", lr=0.02,
+                    wd=0.0, moonshot=False, seed=3,
+                    desc="8x4096^2 + 4x4096x14336 + 4x14336x4096 bf16, Muon, 5 NS5 iterations")
+    if name == "gpt2_small":
+        return dict(shapes=workloads.gpt2_small_shapes(), cond=False, mdt="bf16", lr=0.02,
+                    wd=0.1, moonshot=True, seed=2,
+                    desc="GPT-2-small hidden matrices (72) bf16, Muon, Moonshot scale, wd 0.1")
+    if name == "square1024":
+        return dict(shapes=workloads.single_square_shapes(), cond=False, mdt="bf16", lr=0.02,
+                    wd=0.0, moonshot=False, seed=1, desc="one 1024x1024 bf16 matrix, Muon")
+    if name.startswith("lora_r"):
+        r = int(name[6:])
+        return dict(shapes=workloads.lora_shapes(r), cond=True, mdt="fp32",
+                    lr={2: 0.018, 8: 0.010, 32: 0.010}.get(r, 0.01), wd=0.0, moonshot=False,
+                    seed=4, desc=f"224 LoRA projections r={r} (A r x 4096, B 4096 x r), "
+                                 "fp32 momentum, bf16 weights, Dimuon")
+    raise SystemExit(f"unknown workload {name}")
+
+
+def ns_flops(shapes):
+    """Algorithmic Newton-Schulz flops per iteration: 3 m^2 n + m^3 per matrix
+    (symmetric products counted once), m the short side."""
+    tot = 0.0
+    for r, c in shapes:
+        m, n = min(r, c), max(r, c)
+        tot += 3.0 * m * m * n + m ** 3
+    return tot
+
+
+def step_bytes(spec):
+    """Algorithmic HBM bytes of one step outside the products: read G, read
+    and write M, read and write W."""
+    mb = 4 if spec["mdt"] == "fp32" else 2
+    return sum(r * c for r, c in spec["shapes"]) * (2 + 2 * mb + 4)
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return json.load(fh), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+         "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for ln in out.strip().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), util=float(f[4]),
+                                 hw=f[6], hwt=f[7], swt=f[8], pcap=f[9]))
+            except ValueError:
+                continue
+        load = [r for r in rows if r["util"] >= 50] or rows
+        if not load:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        reasons = set()
+        for r in load:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                            ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([r["sm"] for r in load])),
+                "sm_max_mhz": max(r["smax"] for r in load), "reasons": sorted(reasons),
+                "samples": len(load)}
+
+
+def oracle_sample_time(spec):
+    """Times the fp64 CPU oracle on one matrix of the workload (the cheapest
+    representative: the first shape) and extrapolates by algorithmic flops."""
+    import oracle as orc
+    shp = spec["shapes"][0]
+    rng = np.random.default_rng(spec["seed"])
+    G = rng.standard_normal(shp)
+    W = 0.02 * rng.standard_normal(shp)
+    M = np.zeros(shp)
+    h = orc.HParams(lr=spec["lr"], weight_decay=spec["wd"],
+                    scale_mode=orc.SCALE_MOONSHOT if spec["moonshot"] else orc.SCALE_NONE)
+    t0 = time.perf_counter()
+    if spec["cond"]:
+        orc.dimuon_step(W, G, M, np.zeros(shp[0]), np.zeros(shp[1]), h,
+                        momentum_dtype=spec["mdt"], weight_dtype="bf16")
+    else:
+        orc.muon_step(W, G, M, h, momentum_dtype=spec["mdt"], weight_dtype="bf16")
+    dt = time.perf_counter() - t0
+    scale = ns_flops(spec["shapes"]) / ns_flops([shp])
+    return dt, dt * scale, f"one {shp[0]}x{shp[1]} matrix of the workload per step, " \
+                           f"extrapolated to all {len(spec['shapes'])} by algorithmic flops"
+
+
+def run_reference(args, spec, rank):
+    if rank != 0:
+        return
+    threads = os.cpu_count()
+    oracle_sample_time(spec)  # one untimed warm-up step
+    times = []
+    for _ in range(args.steps):
+        _, full, sample = oracle_sample_time(spec)
+        times.append(full)
+    t = float(np.median(times))
+    value = len(spec["shapes"]) / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "matrices/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": 1, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": spec["desc"]},
+            "cpu_baseline": {"value": value, "unit": "matrices/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "matrices/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="large_batch")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    spec = workload_spec(args.workload)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, spec, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import dimuon_optimizer_b200 as dm
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    shapes = spec["shapes"]
+    bf = torch.bfloat16
+    mdt = torch.float32 if spec["mdt"] == "fp32" else bf
+    rng = np.random.default_rng(spec["seed"] + 17 * rank)
+    torch.manual_seed(spec["seed"] + 1000 + rank)
+    G_host, G, W, M, ER, EC = [], [], [], [], [], []
+    for (r, c) in shapes:
+        g = torch.from_numpy(rng.standard_normal((r, c), dtype=np.float32)).to(bf)
+        G_host.append(g.pin_memory())
+        G.append(g.to(dev))
+        W.append((0.02 * torch.randn((r, c), device=dev, dtype=torch.float32)).to(bf))
+        M.append(torch.zeros((r, c), device=dev, dtype=mdt))
+        ER.append(torch.zeros(r, device=dev, dtype=torch.float32) if spec["cond"] else None)
+        EC.append(torch.zeros(c, device=dev, dtype=torch.float32) if spec["cond"] else None)
+    mats = [dm.dm_matrix(W[i], G[i], M[i], ER[i], EC[i]) for i in range(len(shapes))]
+    hp = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"],
+                               scale_mode=dm.DM_SCALE_MOONSHOT if spec["moonshot"]
+                               else dm.DM_SCALE_NONE)
+    step_fn = dm.dm_dimuon_step if spec["cond"] else dm.dm_muon_step
+    ws = torch.empty(dm.dm_workspace_size(mats, hp, int(spec["cond"])), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def capture(h):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            dm.check(step_fn(mats, h, ws, stream=stream))
+        return g
+
+    # warm-up eagerly once (plans, tensor maps), then capture the step
+    with torch.cuda.stream(stream):
+        dm.check(step_fn(mats, hp, ws, stream=stream))
+    torch.cuda.synchronize(dev)
+    graph = capture(hp)
+
+    def timed(g, reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return e0.elapsed_time(e1) / 1e3
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    t_dev = max_over_ranks(timed(graph, args.steps))
+    clocks = sampler.stop()
+    ms_step = t_dev / args.steps * 1e3
+    n_mat = len(shapes)
+    value = world * n_mat * args.steps / t_dev
+
+    # dominant kernel (tensor-core product): 4 extra iterations of a 5-step
+    # schedule over a 1-step schedule, on the launch stream
+    reps = max(2, min(args.steps, 5))
+    hp1 = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"], ns_steps=1,
+                                scale_mode=hp.scale_mode)
+    g1 = capture(hp1)
+    g1.replay()
+    t5 = timed(graph, reps) / reps
+    t1 = timed(g1, reps) / reps
+    del g1
+    per_iter_flops = ns_flops([s for s in shapes if min(s) > dm.DM_THIN_MAX])
+    peaks, peak_kind = load_peaks()
+    tc_launches = 3 * 4
+    if per_iter_flops > 0 and t5 > t1:
+        achieved = 4 * per_iter_flops / (t5 - t1) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", 1400.0)
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": "tc_ns_product", "avg_launch_ms": (t5 - t1) / tc_launches * 1e3,
+                    "peak_kind": f"{peak_kind} bf16 dense, sustained"}
+    else:
+        gbs = step_bytes(spec) / (ms_step / 1e3) / 1e9
+        peak = peaks.get("hbm_gbs", 6650.0)
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                    "frac": gbs / peak, "traffic": None, "kernel": "thin_step",
+                    "peak_kind": f"{peak_kind} HBM copy"}
+
+    # end to end through the public API: pinned host gradients in, status out
+    h2d = sum(g.numel() * g.element_size() for g in G_host)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            for gd, gh in zip(G, G_host):
+                gd.copy_(gh, non_blocking=True)
+            dm.check(step_fn(mats, hp, ws, stream=stream))
+            st = dm.dm_read_device_status(ws, stream=stream)
+            assert st == dm.DM_OK, dm.dm_status_string(st)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    e2e = {"value": world * n_mat * args.steps / t_e2e, "unit": "matrices/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+
+    if rank != 0:
+        return
+    thin = sum(1 for s in shapes if min(s) <= dm.DM_THIN_MAX)
+    big = n_mat - thin
+    launches = 0
+    if thin:
+        launches += sum(math.ceil(sum(1 for s in shapes if min(s) <= dm.DM_THIN_MAX and
+                                      lo < min(s) <= hi) / 256)
+                        for lo, hi in ((0, 8), (8, 16), (16, 32)))
+    if big:
+        launches += 2 + 3 * hp.ns_steps + (3 if spec["cond"] else 0)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        _, full, sample = oracle_sample_time(spec)
+        cpu = {"value": n_mat / full, "unit": "matrices/s", "cores": os.cpu_count(),
+               "kind": "oracle", "sample": sample}
+    line = {"metric": METRIC, "value": value, "unit": "matrices/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) gradients, N(0,0.02^2) weights)",
+            "config": {"workload": spec["desc"], "matrices": n_mat, "parallelism":
+                       f"replica per GPU x{world}", "l2": "inputs larger than L2 (no flush)",
+                       "cuda_graph": True, "ns_tflops_step": ns_flops(shapes) * hp.ns_steps
+                       / (ms_step / 1e3) / 1e12},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": launches * args.steps}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

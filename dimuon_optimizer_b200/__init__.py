@@ -1,0 +1,210 @@
+"""Python binding of libdimuon.so (the B200 Muon / Dimuon optimizer step).
+
+Argument marshalling only: every step of the method runs in the CUDA kernels
+of the shared library.  The names mirror the C ABI in include/dimuon.h.
+PyTorch supplies device memory and streams.
+
+    import torch, dimuon_optimizer_b200 as dm
+    mats = [dm.dm_matrix(W, G, M)]                      # torch CUDA tensors
+    hp = dm.dm_default_hparams()
+    ws = torch.empty(dm.dm_workspace_size(mats, hp, 0), dtype=torch.uint8,
+                     device="cuda")
+    dm.check(dm.dm_muon_step(mats, hp, ws))
+
+The shared library must have been built (python -m dimuon_optimizer_b200.build,
+or __graft_entry__.build()); importing fails loudly otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import c_float, c_int, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdimuon.so")
+
+DM_OK = 0
+DM_ERR_INVALID_ARG = 1
+DM_ERR_UNSUPPORTED = 2
+DM_ERR_WORKSPACE = 3
+DM_ERR_CUDA = 4
+DM_ERR_DEVICE_TIMEOUT = 5
+DM_ERR_NONFINITE = 6
+
+DM_BF16 = 0
+DM_FP32 = 1
+DM_PREC_FP32 = 0
+DM_PREC_BF16_TC = 1
+DM_SCALE_NONE = 0
+DM_SCALE_MOONSHOT = 1
+DM_THIN_MAX = 32
+DM_DBG_NO_THIN = 0x1
+
+EXPORTED = ("dm_default_hparams", "dm_workspace_size", "dm_muon_step", "dm_dimuon_step",
+            "dm_read_device_status", "dm_status_string", "dm_version")
+
+
+class dm_matrix_t(ctypes.Structure):
+    _fields_ = [("rows", c_int64), ("cols", c_int64), ("weight", c_void_p),
+                ("weight_dtype", c_int32), ("grad_dtype", c_int32), ("grad", c_void_p),
+                ("momentum", c_void_p), ("momentum_dtype", c_int32), ("reserved0", c_int32),
+                ("row_energy", c_void_p), ("col_energy", c_void_p), ("update_out", c_void_p)]
+
+
+class dm_hparams_t(ctypes.Structure):
+    _fields_ = [("mu", c_float), ("lr", c_float), ("weight_decay", c_float),
+                ("ns_steps", c_int32), ("a", c_float), ("b", c_float), ("c", c_float),
+                ("cond_eps", c_float), ("scale_mode", c_int32), ("scale_coef", c_float),
+                ("precision", c_int32), ("debug_flags", c_uint32)]
+
+
+class DimuonError(RuntimeError):
+    def __init__(self, code):
+        super().__init__(f"libdimuon status {code}: {dm_status_string(code)}")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m dimuon_optimizer_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    lib.dm_default_hparams.argtypes = [P(dm_hparams_t)]
+    lib.dm_default_hparams.restype = None
+    lib.dm_workspace_size.argtypes = [P(dm_matrix_t), c_int, P(dm_hparams_t), c_int,
+                                      P(c_size_t)]
+    lib.dm_workspace_size.restype = c_int
+    for name in ("dm_muon_step", "dm_dimuon_step"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P(dm_matrix_t), c_int, P(dm_hparams_t), c_void_p, c_size_t, c_void_p]
+        fn.restype = c_int
+    lib.dm_read_device_status.argtypes = [c_void_p, c_void_p, P(c_int32)]
+    lib.dm_read_device_status.restype = c_int
+    lib.dm_status_string.argtypes = [c_int32]
+    lib.dm_status_string.restype = ctypes.c_char_p
+    lib.dm_version.argtypes = []
+    lib.dm_version.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+# ----------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return DM_BF16
+    if t.dtype == torch.float32:
+        return DM_FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def dm_matrix(weight, grad, momentum, row_energy=None, col_energy=None, update_out=None):
+    """A dm_matrix_t over torch CUDA tensors (row-major, contiguous)."""
+    rows, cols = weight.shape
+    for t in (weight, grad, momentum):
+        if t.shape != (rows, cols) or not t.is_contiguous():
+            raise ValueError("weight, grad and momentum must be contiguous rows x cols")
+    for t, n in ((row_energy, rows), (col_energy, cols)):
+        if t is not None and (t.numel() != n or t.dtype.itemsize != 4 or not t.is_contiguous()):
+            raise ValueError("energies must be contiguous fp32 vectors of rows / cols")
+    if update_out is not None and (update_out.shape != (rows, cols)
+                                   or not update_out.is_contiguous()):
+        raise ValueError("update_out must be a contiguous fp32 rows x cols tensor")
+    m = dm_matrix_t()
+    m.rows, m.cols = rows, cols
+    m.weight, m.weight_dtype = weight.data_ptr(), _dtype_code(weight)
+    m.grad, m.grad_dtype = grad.data_ptr(), _dtype_code(grad)
+    m.momentum, m.momentum_dtype = momentum.data_ptr(), _dtype_code(momentum)
+    m.row_energy = None if row_energy is None else row_energy.data_ptr()
+    m.col_energy = None if col_energy is None else col_energy.data_ptr()
+    m.update_out = None if update_out is None else update_out.data_ptr()
+    return m
+
+
+def _array(mats):
+    if isinstance(mats, ctypes.Array):
+        return mats, len(mats)
+    mats = list(mats)
+    arr = (dm_matrix_t * max(1, len(mats)))(*mats)
+    return arr, len(mats)
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        return c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return c_void_p(stream)
+    return c_void_p(stream.cuda_stream)
+
+
+def _ws(workspace):
+    if hasattr(workspace, "data_ptr"):
+        return c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+    ptr, nbytes = workspace
+    return c_void_p(ptr), nbytes
+
+
+# ----------------------------------------------------------------------------
+# the C ABI, by name
+# ----------------------------------------------------------------------------
+def dm_default_hparams(**overrides):
+    hp = dm_hparams_t()
+    _lib.dm_default_hparams(ctypes.byref(hp))
+    for k, v in overrides.items():
+        setattr(hp, k, v)
+    return hp
+
+
+def dm_workspace_size(mats, hp, conditioned):
+    arr, n = _array(mats)
+    out = c_size_t(0)
+    st = _lib.dm_workspace_size(arr, n, ctypes.byref(hp), int(conditioned), ctypes.byref(out))
+    if st != DM_OK:
+        raise DimuonError(st)
+    return out.value
+
+
+def dm_muon_step(mats, hp, workspace, stream=None):
+    arr, n = _array(mats)
+    ptr, nbytes = _ws(workspace)
+    return _lib.dm_muon_step(arr, n, ctypes.byref(hp), ptr, nbytes, _stream_handle(stream))
+
+
+def dm_dimuon_step(mats, hp, workspace, stream=None):
+    arr, n = _array(mats)
+    ptr, nbytes = _ws(workspace)
+    return _lib.dm_dimuon_step(arr, n, ctypes.byref(hp), ptr, nbytes, _stream_handle(stream))
+
+
+def dm_read_device_status(workspace, stream=None):
+    ptr, _ = _ws(workspace)
+    out = c_int32(0)
+    st = _lib.dm_read_device_status(ptr, _stream_handle(stream), ctypes.byref(out))
+    if st != DM_OK:
+        raise DimuonError(st)
+    return out.value
+
+
+def dm_status_string(code):
+    return _lib.dm_status_string(int(code)).decode()
+
+
+def dm_version():
+    return _lib.dm_version().decode()
+
+
+def check(status):
+    """Raises DimuonError for a non-zero status."""
+    if status != DM_OK:
+        raise DimuonError(status)
+    return status

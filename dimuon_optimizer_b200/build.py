@@ -1,0 +1,52 @@
+"""Builds libdimuon.so in-tree with nvcc for sm_100a.
+
+    python -m dimuon_optimizer_b200.build [--debug]
+
+The library is compiled for B200 only (-gencode arch=compute_100a,code=sm_100a)
+and links the CUDA runtime statically; the driver's tensor-map encoder is
+looked up at run time, so no -lcuda is needed.
+"""
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libdimuon.so")
+SOURCES = ["api.cu", "k_elementwise.cu", "k_ns_simt.cu", "k_ns_tc.cu", "k_thin.cu"]
+HEADERS = ["dm_common.cuh", "dm_internal.h", "dm_sm100.cuh", "dm_tiles.cuh"]
+
+
+def nvcc_path():
+    cand = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    return cand if os.path.exists(cand) else "nvcc"
+
+
+def _stale():
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [
+        os.path.join(INCLUDE, "dimuon.h"), os.path.abspath(__file__)]
+    return any(os.path.getmtime(d) > t for d in deps)
+
+
+def build(force=False, verbose=False, extra=()):
+    if not force and not _stale():
+        return LIB
+    cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
+           "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
+           "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp"]
+    cmd += list(extra)
+    cmd += [os.path.join(CSRC, f) for f in SOURCES]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force=True, verbose=True, extra=["-Xptxas", "-v"] if "-v" in sys.argv else [])

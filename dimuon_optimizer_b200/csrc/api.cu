@@ -1,0 +1,657 @@
+// Host side of libdimuon.so: argument validation, workspace layout, launch
+// planning and the C ABI declared in include/dimuon.h.
+//
+// Step order (one stream, no host synchronisation):
+//   status word cleared
+//   thin factors (short side <= DM_THIN_MAX): one CTA per factor, whole step
+//   other matrices:
+//     K0   (Dimuon) R, C from the previous momentum's energies
+//     K1   momentum, X_0 = R M_t C, partial norms / energies
+//     K1b  energies of M_t, ||X_0||_F scalars
+//     ns_steps x { A = X X^T ; B = bA + cA^2 ; X <- aX + BX }  (tensor cores
+//          in DM_PREC_BF16_TC, fp32 SIMT in DM_PREC_FP32); the last product
+//          applies the Muon update or emits X_5
+//     K3a, K3 (Dimuon) renormalise Y = R X_5 C, scale, decay, apply
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "dimuon.h"
+#include "dm_internal.h"
+#include "dm_tiles.cuh"
+
+namespace dm {
+namespace {
+
+constexpr size_t HEADER_BYTES = 1024;
+constexpr int64_t MAX_DIM = int64_t(1) << 24;
+constexpr int64_t MAX_ELEMS = (int64_t(1) << 31) - 1;
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+struct MatPlan {
+  int idx;
+  bool thin;
+  int64_t rows, cols;
+  int m, n;
+  bool tall;
+  int64_t ldx, ldm;
+  int k1_rt, k1_ct;
+  int n_part;
+  size_t off_scal, off_R, off_C, off_psum, off_perow, off_pecol, off_pfin;
+  size_t off_X[2], off_A, off_B;
+};
+
+struct Layout {
+  std::vector<MatPlan> mats;
+  size_t bytes = 0;
+  bool tc = false;
+  bool cond = false;
+};
+
+dm_status_t validate(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int cond) {
+  if (n < 0 || (n > 0 && !mats) || !hp) return DM_ERR_INVALID_ARG;
+  if (hp->ns_steps < 1 || hp->ns_steps > 64) return DM_ERR_INVALID_ARG;
+  if (hp->precision != DM_PREC_FP32 && hp->precision != DM_PREC_BF16_TC) return DM_ERR_INVALID_ARG;
+  if (hp->scale_mode != DM_SCALE_NONE && hp->scale_mode != DM_SCALE_MOONSHOT) return DM_ERR_INVALID_ARG;
+  const float scalars[] = {hp->mu, hp->lr, hp->weight_decay, hp->a, hp->b, hp->c, hp->cond_eps,
+                           hp->scale_coef};
+  for (float v : scalars)
+    if (!(v == v) || v > 3.0e38f || v < -3.0e38f) return DM_ERR_INVALID_ARG;
+  if (cond && !(hp->cond_eps >= 0.f)) return DM_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const dm_matrix_t& m = mats[i];
+    if (m.rows < 1 || m.cols < 1 || m.rows > MAX_DIM || m.cols > MAX_DIM ||
+        m.rows * m.cols > MAX_ELEMS)
+      return DM_ERR_INVALID_ARG;
+    if (!m.weight || !m.grad || !m.momentum) return DM_ERR_INVALID_ARG;
+    const int32_t dts[] = {m.weight_dtype, m.grad_dtype, m.momentum_dtype};
+    for (int32_t d : dts)
+      if (d != DM_BF16 && d != DM_FP32) return DM_ERR_UNSUPPORTED;
+    if (cond && (!m.row_energy || !m.col_energy)) return DM_ERR_INVALID_ARG;
+  }
+  return DM_OK;
+}
+
+Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int cond) {
+  Layout L;
+  L.tc = hp->precision == DM_PREC_BF16_TC;
+  L.cond = cond != 0;
+  const size_t esz = L.tc ? 2 : 4;
+  size_t cur = HEADER_BYTES;
+  auto take = [&](size_t bytes, size_t align) {
+    cur = round_up(cur, align);
+    const size_t o = cur;
+    cur += round_up(bytes, 16);
+    return o;
+  };
+  for (int i = 0; i < n; ++i) {
+    MatPlan p{};
+    p.idx = i;
+    p.rows = mats[i].rows;
+    p.cols = mats[i].cols;
+    p.tall = p.rows > p.cols;
+    p.m = (int)std::min(p.rows, p.cols);
+    p.n = (int)std::max(p.rows, p.cols);
+    p.thin = p.m <= DM_THIN_MAX && !(hp->debug_flags & DM_DBG_NO_THIN);
+    if (!p.thin) {
+      p.ldx = (int64_t)round_up((size_t)p.cols, 8);
+      p.ldm = (int64_t)round_up((size_t)p.m, 8);
+      p.k1_rt = (int)ceil_div(p.rows, K1_ROWS);
+      p.k1_ct = (int)ceil_div(p.cols, K1_COLS);
+      if (L.tc)
+        p.n_part = (int)(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN)) * 4;
+      else
+        p.n_part = (int)(ceil_div(p.rows, 128) * ceil_div(p.cols, 128));
+      p.off_scal = take(SC_COUNT * sizeof(float), 256);
+      p.off_psum = take((size_t)p.k1_rt * p.k1_ct * sizeof(float), 256);
+      if (L.cond) {
+        p.off_R = take((size_t)p.rows * sizeof(float), 256);
+        p.off_C = take((size_t)p.cols * sizeof(float), 256);
+        p.off_perow = take((size_t)p.k1_ct * p.rows * sizeof(float), 256);
+        p.off_pecol = take((size_t)p.k1_rt * p.cols * sizeof(float), 256);
+        p.off_pfin = take((size_t)p.n_part * 2 * sizeof(float), 256);
+      }
+      for (int b = 0; b < 2; ++b) p.off_X[b] = take((size_t)p.rows * p.ldx * esz, 1024);
+      p.off_A = take((size_t)p.m * p.ldm * esz, 1024);
+      p.off_B = take((size_t)p.m * p.ldm * esz, 1024);
+    }
+    L.mats.push_back(p);
+  }
+  L.bytes = round_up(cur, 1024);
+  return L;
+}
+
+// ------------------------------ tensor maps -------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 matrix [outer][inner] with leading dimension ld (elements); 64 x 64
+// boxes with the 128-byte swizzle the UMMA descriptors expect.
+bool make_map(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct MatMaps {
+  CUtensorMap X[2], A, B;
+};
+
+std::mutex g_cache_mu;
+std::unordered_map<std::string, std::vector<MatMaps>> g_map_cache;
+
+std::string cache_key(const Layout& L, const void* ws, int dev) {
+  std::string k;
+  auto put = [&](const void* p, size_t n) { k.append(reinterpret_cast<const char*>(p), n); };
+  put(&ws, sizeof(ws));
+  put(&dev, sizeof(dev));
+  for (const MatPlan& p : L.mats) {
+    if (p.thin) continue;
+    put(&p.rows, sizeof(p.rows));
+    put(&p.cols, sizeof(p.cols));
+    put(&p.off_X[0], sizeof(size_t));
+  }
+  return k;
+}
+
+bool get_maps(const Layout& L, uint8_t* ws, int dev, std::vector<MatMaps>& out) {
+  const std::string key = cache_key(L, ws, dev);
+  {
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    auto it = g_map_cache.find(key);
+    if (it != g_map_cache.end()) {
+      out = it->second;
+      return true;
+    }
+  }
+  out.assign(L.mats.size(), MatMaps{});
+  for (size_t i = 0; i < L.mats.size(); ++i) {
+    const MatPlan& p = L.mats[i];
+    if (p.thin) continue;
+    for (int b = 0; b < 2; ++b)
+      if (!make_map(&out[i].X[b], ws + p.off_X[b], p.cols, p.rows, p.ldx)) return false;
+    if (!make_map(&out[i].A, ws + p.off_A, p.m, p.m, p.ldm)) return false;
+    if (!make_map(&out[i].B, ws + p.off_B, p.m, p.m, p.ldm)) return false;
+  }
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  if (g_map_cache.size() > 64) g_map_cache.clear();
+  g_map_cache[key] = out;
+  return true;
+}
+
+int sm_count(int dev) {
+  static std::mutex mu;
+  static std::unordered_map<int, int> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  cache[dev] = v;
+  return v;
+}
+
+// ---------------------------- product plans -------------------------------
+enum Phase { PH_SYRK = 0, PH_POLY = 1, PH_GEMM = 2 };
+
+// Fills the epilogue / shape part of one product; operand sources are set by
+// the caller (tensor maps or pointers).  Returns operand-source descriptors.
+struct OperandSrc {
+  int a_buf, b_buf;   // 0/1 = X buffer, 2 = A, 3 = B
+};
+
+OperandSrc fill_gemm(GemmMat& g, const MatPlan& p, const dm_matrix_t& um, const dm_hparams_t* hp,
+                     uint8_t* ws, int phase, int k, bool cond, float kappa, int bm, int bn) {
+  std::memset(&g, 0, sizeof(g));
+  const int ns = hp->ns_steps;
+  const int xin = (k - 1) & 1, xout = k & 1;
+  float* scal = reinterpret_cast<float*>(ws + p.off_scal);
+  g.scal = scal;
+  g.scal_idx = -1;
+  OperandSrc src{};
+  if (phase == PH_SYRK) {
+    g.M = g.N = p.m;
+    g.K = p.n;
+    g.flags = GF_SYM | (p.tall ? (GF_A_MN | GF_B_MN) : 0);
+    g.out = ws + p.off_A;
+    g.ldo = (int)p.ldm;
+    g.epi = EPI_SYRK;
+    if (k == 1) g.scal_idx = SC_INV_S2;
+    src = {xin, xin};
+  } else if (phase == PH_POLY) {
+    g.M = g.N = p.m;
+    g.K = p.m;
+    g.flags = GF_SYM;
+    g.out = ws + p.off_B;
+    g.ldo = (int)p.ldm;
+    g.aux = ws + p.off_A;
+    g.ldaux = (int)p.ldm;
+    g.epi = EPI_POLY;
+    g.coef_acc = hp->c;
+    g.coef_aux = hp->b;
+    src = {2, 2};
+  } else {
+    g.M = (int)p.rows;
+    g.N = (int)p.cols;
+    g.K = p.m;
+    if (p.tall) {
+      g.flags = GF_N_FAST;
+      src = {xin, 3};
+    } else {
+      g.flags = GF_B_MN;
+      src = {3, xin};
+    }
+    g.aux = ws + p.off_X[xin];
+    g.ldaux = (int)p.ldx;
+    g.coef_aux = hp->a;
+    if (k == 1) g.scal_idx = SC_INV_S;
+    if (k < ns) {
+      g.epi = EPI_GEMM;
+      g.out = ws + p.off_X[xout];
+      g.ldo = (int)p.ldx;
+    } else if (!cond) {
+      g.epi = EPI_FINAL_MUON;
+      g.W = um.weight;
+      g.wdt = um.weight_dtype;
+      g.ldw = (int)p.cols;
+      g.upd = um.update_out;
+      g.kappa = kappa;
+    } else {
+      g.epi = EPI_FINAL_DIMUON;
+      g.out = ws + p.off_X[xout];
+      g.ldo = (int)p.ldx;
+      g.R = reinterpret_cast<const float*>(ws + p.off_R);
+      g.C = reinterpret_cast<const float*>(ws + p.off_C);
+      g.part = reinterpret_cast<float*>(ws + p.off_pfin);
+    }
+  }
+  g.tiles_m = (int)ceil_div(g.M, bm);
+  g.tiles_n = (int)ceil_div(g.N, bn);
+  return src;
+}
+
+float kappa_of(const dm_hparams_t* hp, int64_t rows, int64_t cols) {
+  if (hp->scale_mode == DM_SCALE_MOONSHOT)
+    return (float)((double)hp->scale_coef * std::sqrt((double)std::max(rows, cols)));
+  return 1.f;
+}
+
+#define DM_CUDA(x)                          \
+  do {                                      \
+    if ((x) != cudaSuccess) return DM_ERR_CUDA; \
+  } while (0)
+
+dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, void* workspace,
+                     size_t ws_bytes, void* stream_v, int cond) {
+  dm_status_t st = validate(mats, n, hp, cond);
+  if (st != DM_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DM_ERR_WORKSPACE;
+  const Layout L = make_layout(mats, n, hp, cond);
+  if (ws_bytes < L.bytes) return DM_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_v);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  int dev = 0;
+  DM_CUDA(cudaGetDevice(&dev));
+  const float decay = 1.f - hp->lr * hp->weight_decay;
+
+  DM_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  if (n == 0) return DM_OK;
+
+  // ---------------------------- thin factors -------------------------------
+  {
+    std::vector<int> groups[3];  // pad 8 / 16 / 32
+    for (const MatPlan& p : L.mats)
+      if (p.thin) groups[p.m <= 8 ? 0 : (p.m <= 16 ? 1 : 2)].push_back(p.idx);
+    const int pads[3] = {8, 16, 32};
+    for (int gi = 0; gi < 3; ++gi) {
+      const std::vector<int>& idx = groups[gi];
+      const int nchunks = (int)ceil_div((int64_t)idx.size(), THIN_MAX);
+      for (int ch = 0; ch < nchunks; ++ch) {
+        // split evenly so launches are balanced
+        const size_t b = idx.size() * ch / nchunks, e = idx.size() * (ch + 1) / nchunks;
+        static thread_local ThinParams tp;
+        std::memset(&tp, 0, sizeof(tp));
+        tp.count = (int)(e - b);
+        tp.pad = pads[gi];
+        tp.conditioned = cond;
+        tp.ns_steps = hp->ns_steps;
+        tp.mu = hp->mu;
+        tp.lr = hp->lr;
+        tp.decay = decay;
+        tp.a = hp->a;
+        tp.b = hp->b;
+        tp.c = hp->c;
+        tp.eps = hp->cond_eps;
+        tp.status = status;
+        for (size_t q = b; q < e; ++q) {
+          const dm_matrix_t& um = mats[idx[q]];
+          ThinMat& t = tp.mats[q - b];
+          t.G = um.grad;
+          t.M = um.momentum;
+          t.W = um.weight;
+          t.upd = um.update_out;
+          t.e_row = cond ? um.row_energy : nullptr;
+          t.e_col = cond ? um.col_energy : nullptr;
+          t.rows = um.rows;
+          t.cols = um.cols;
+          t.gdt = um.grad_dtype;
+          t.mdt = um.momentum_dtype;
+          t.wdt = um.weight_dtype;
+          t.kappa = kappa_of(hp, um.rows, um.cols);
+        }
+        DM_CUDA(launch_thin(tp, s));
+      }
+    }
+  }
+
+  // -------------------------- Newton-Schulz path ---------------------------
+  std::vector<const MatPlan*> big;
+  for (const MatPlan& p : L.mats)
+    if (!p.thin) big.push_back(&p);
+  if (big.empty()) return DM_OK;
+  // heaviest products first, so the persistent grid ends with small tiles
+  std::stable_sort(big.begin(), big.end(), [](const MatPlan* a, const MatPlan* b) {
+    return (double)a->m * a->m * a->n > (double)b->m * b->m * b->n;
+  });
+  const int xdt = L.tc ? DT_BF16 : DT_FP32;
+
+  // K0
+  if (cond) {
+    static thread_local K0Params p0;
+    for (size_t b = 0; b < big.size(); b += K0_MAX) {
+      std::memset(&p0, 0, sizeof(p0));
+      p0.eps = hp->cond_eps;
+      for (size_t q = b; q < std::min(big.size(), b + K0_MAX); ++q) {
+        const MatPlan& p = *big[q];
+        const dm_matrix_t& um = mats[p.idx];
+        K0Mat& k = p0.mats[p0.count++];
+        k.e_row = um.row_energy;
+        k.e_col = um.col_energy;
+        k.R = reinterpret_cast<float*>(ws + p.off_R);
+        k.C = reinterpret_cast<float*>(ws + p.off_C);
+        k.rows = p.rows;
+        k.cols = p.cols;
+      }
+      DM_CUDA(launch_k0(p0, s));
+    }
+  }
+  // K1
+  {
+    static thread_local K1Params p1;
+    for (size_t b = 0; b < big.size(); b += K1_MAX) {
+      std::memset(&p1, 0, sizeof(p1));
+      p1.mu = hp->mu;
+      int tiles = 0;
+      for (size_t q = b; q < std::min(big.size(), b + K1_MAX); ++q) {
+        const MatPlan& p = *big[q];
+        const dm_matrix_t& um = mats[p.idx];
+        p1.starts[p1.count] = tiles;
+        K1Mat& k = p1.mats[p1.count++];
+        k.G = um.grad;
+        k.M = um.momentum;
+        k.X0 = ws + p.off_X[0];
+        k.R = cond ? reinterpret_cast<const float*>(ws + p.off_R) : nullptr;
+        k.C = cond ? reinterpret_cast<const float*>(ws + p.off_C) : nullptr;
+        k.part_sumsq = reinterpret_cast<float*>(ws + p.off_psum);
+        k.part_erow = cond ? reinterpret_cast<float*>(ws + p.off_perow) : nullptr;
+        k.part_ecol = cond ? reinterpret_cast<float*>(ws + p.off_pecol) : nullptr;
+        k.rows = p.rows;
+        k.cols = p.cols;
+        k.ldx = p.ldx;
+        k.gdt = um.grad_dtype;
+        k.mdt = um.momentum_dtype;
+        k.xdt = xdt;
+        k.vec = (p.cols % 8 == 0) && !(reinterpret_cast<uintptr_t>(um.grad) & 15u) &&
+                !(reinterpret_cast<uintptr_t>(um.momentum) & 15u);
+        k.n_rt = p.k1_rt;
+        k.n_ct = p.k1_ct;
+        tiles += p.k1_rt * p.k1_ct;
+      }
+      p1.starts[p1.count] = tiles;
+      DM_CUDA(launch_k1(p1, tiles, s));
+    }
+  }
+  // K1b
+  {
+    static thread_local K1bParams pb;
+    for (size_t b = 0; b < big.size(); b += K1B_MAX) {
+      std::memset(&pb, 0, sizeof(pb));
+      pb.status = status;
+      int blocks = 0;
+      for (size_t q = b; q < std::min(big.size(), b + K1B_MAX); ++q) {
+        const MatPlan& p = *big[q];
+        const dm_matrix_t& um = mats[p.idx];
+        pb.starts[pb.count] = blocks;
+        K1bMat& k = pb.mats[pb.count++];
+        k.part_sumsq = reinterpret_cast<const float*>(ws + p.off_psum);
+        k.part_erow = cond ? reinterpret_cast<const float*>(ws + p.off_perow) : nullptr;
+        k.part_ecol = cond ? reinterpret_cast<const float*>(ws + p.off_pecol) : nullptr;
+        k.e_row = cond ? um.row_energy : nullptr;
+        k.e_col = cond ? um.col_energy : nullptr;
+        k.scal = reinterpret_cast<float*>(ws + p.off_scal);
+        k.rows = p.rows;
+        k.cols = p.cols;
+        k.n_rt = p.k1_rt;
+        k.n_ct = p.k1_ct;
+        blocks += 1 + (cond ? (int)ceil_div(p.rows + p.cols, K1B_THREADS) : 0);
+      }
+      pb.starts[pb.count] = blocks;
+      DM_CUDA(launch_k1b(pb, blocks, s));
+    }
+  }
+  // Newton-Schulz products
+  if (L.tc) {
+    std::vector<MatMaps> maps;
+    if (!get_maps(L, ws, dev, maps)) return DM_ERR_CUDA;
+    const int nsm = sm_count(dev);
+    static thread_local TcParams pt;
+    for (int k = 1; k <= hp->ns_steps; ++k)
+      for (int ph = 0; ph < 3; ++ph)
+        for (size_t b = 0; b < big.size(); b += TC_MAX) {
+          std::memset(&pt, 0, sizeof(pt));
+          pt.status = status;
+          pt.lr = hp->lr;
+          pt.decay = decay;
+          pt.debug = hp->debug_flags;
+          int tiles = 0;
+          for (size_t q = b; q < std::min(big.size(), b + TC_MAX); ++q) {
+            const MatPlan& p = *big[q];
+            TcMat& tm = pt.mats[pt.count];
+            const OperandSrc src =
+                fill_gemm(tm.g, p, mats[p.idx], hp, ws, ph, k, cond != 0,
+                          kappa_of(hp, p.rows, p.cols), TC_BM, TC_BN);
+            const MatMaps& mm = maps[p.idx];
+            auto pick = [&](int buf) -> const CUtensorMap& {
+              return buf < 2 ? mm.X[buf] : (buf == 2 ? mm.A : mm.B);
+            };
+            tm.ta = pick(src.a_buf);
+            tm.tb = pick(src.b_buf);
+            pt.starts[pt.count++] = tiles;
+            tiles += gemm_tile_count(tm.g, TC_BM, TC_BN);
+          }
+          pt.starts[pt.count] = tiles;
+          pt.total_tiles = tiles;
+          DM_CUDA(launch_tc(pt, std::min(tiles, nsm), s));
+        }
+  } else {
+    static thread_local SimtParams ps;
+    for (int k = 1; k <= hp->ns_steps; ++k)
+      for (int ph = 0; ph < 3; ++ph)
+        for (size_t b = 0; b < big.size(); b += SIMT_MAX) {
+          std::memset(&ps, 0, sizeof(ps));
+          ps.lr = hp->lr;
+          ps.decay = decay;
+          int tiles = 0;
+          for (size_t q = b; q < std::min(big.size(), b + SIMT_MAX); ++q) {
+            const MatPlan& p = *big[q];
+            SimtMat& sm = ps.mats[ps.count];
+            const OperandSrc src = fill_gemm(sm.g, p, mats[p.idx], hp, ws, ph, k, cond != 0,
+                                             kappa_of(hp, p.rows, p.cols), 128, 128);
+            auto ptr = [&](int buf) -> const float* {
+              return reinterpret_cast<const float*>(
+                  ws + (buf < 2 ? p.off_X[buf] : (buf == 2 ? p.off_A : p.off_B)));
+            };
+            auto ld = [&](int buf) -> int { return (int)(buf < 2 ? p.ldx : p.ldm); };
+            sm.a = ptr(src.a_buf);
+            sm.b = ptr(src.b_buf);
+            sm.lda = ld(src.a_buf);
+            sm.ldb = ld(src.b_buf);
+            ps.starts[ps.count++] = tiles;
+            tiles += gemm_tile_count(sm.g, 128, 128);
+          }
+          ps.starts[ps.count] = tiles;
+          DM_CUDA(launch_simt(ps, tiles, s));
+        }
+  }
+  // K3a / K3
+  if (cond) {
+    static thread_local K3Params p3;
+    for (size_t b = 0; b < big.size(); b += K3_MAX) {
+      std::memset(&p3, 0, sizeof(p3));
+      p3.lr = hp->lr;
+      p3.decay = decay;
+      int tiles = 0;
+      for (size_t q = b; q < std::min(big.size(), b + K3_MAX); ++q) {
+        const MatPlan& p = *big[q];
+        const dm_matrix_t& um = mats[p.idx];
+        p3.starts[p3.count] = tiles;
+        K3Mat& k = p3.mats[p3.count++];
+        k.X5 = ws + p.off_X[hp->ns_steps & 1];
+        k.W = um.weight;
+        k.upd = um.update_out;
+        k.R = reinterpret_cast<const float*>(ws + p.off_R);
+        k.C = reinterpret_cast<const float*>(ws + p.off_C);
+        k.part = reinterpret_cast<const float*>(ws + p.off_pfin);
+        k.scal = reinterpret_cast<float*>(ws + p.off_scal);
+        k.rows = p.rows;
+        k.cols = p.cols;
+        k.ldx = p.ldx;
+        k.xdt = xdt;
+        k.wdt = um.weight_dtype;
+        k.vec = (p.cols % 8 == 0) && !(reinterpret_cast<uintptr_t>(um.weight) & 15u) &&
+                !(reinterpret_cast<uintptr_t>(um.update_out) & 15u);
+        k.n_part = p.n_part;
+        k.n_rt = p.k1_rt;
+        k.n_ct = p.k1_ct;
+        k.kappa = kappa_of(hp, p.rows, p.cols);
+        tiles += p.k1_rt * p.k1_ct;
+      }
+      p3.starts[p3.count] = tiles;
+      DM_CUDA(launch_k3a(p3, s));
+      DM_CUDA(launch_k3(p3, tiles, s));
+    }
+  }
+  return DM_OK;
+}
+
+}  // namespace
+}  // namespace dm
+
+extern "C" {
+
+void dm_default_hparams(dm_hparams_t* hp) {
+  if (!hp) return;
+  hp->mu = 0.95f;
+  hp->lr = 0.02f;
+  hp->weight_decay = 0.f;
+  hp->ns_steps = 5;
+  hp->a = 3.4445f;
+  hp->b = -4.7750f;
+  hp->c = 2.0315f;
+  hp->cond_eps = 1e-4f;
+  hp->scale_mode = DM_SCALE_NONE;
+  hp->scale_coef = 0.2f;
+  hp->precision = DM_PREC_BF16_TC;
+  hp->debug_flags = 0;
+}
+
+dm_status_t dm_workspace_size(const dm_matrix_t* mats, int n, const dm_hparams_t* hp,
+                              int conditioned, size_t* bytes) {
+  if (!bytes) return DM_ERR_INVALID_ARG;
+  try {
+    const dm_status_t st = dm::validate(mats, n, hp, conditioned);
+    if (st != DM_OK) return st;
+    *bytes = dm::make_layout(mats, n, hp, conditioned).bytes;
+    return DM_OK;
+  } catch (...) {
+    return DM_ERR_INVALID_ARG;
+  }
+}
+
+dm_status_t dm_muon_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  try {
+    return dm::run_step(mats, n, hp, workspace, workspace_bytes, stream, 0);
+  } catch (...) {
+    return DM_ERR_CUDA;
+  }
+}
+
+dm_status_t dm_dimuon_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  try {
+    return dm::run_step(mats, n, hp, workspace, workspace_bytes, stream, 1);
+  } catch (...) {
+    return DM_ERR_CUDA;
+  }
+}
+
+dm_status_t dm_read_device_status(const void* workspace, void* stream, int32_t* out) {
+  if (!workspace || !out) return DM_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DM_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DM_ERR_CUDA;
+  *out = v;
+  return DM_OK;
+}
+
+const char* dm_status_string(int32_t status) {
+  switch (status) {
+    case DM_OK: return "ok";
+    case DM_ERR_INVALID_ARG: return "invalid argument";
+    case DM_ERR_UNSUPPORTED: return "unsupported dtype or mode";
+    case DM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case DM_ERR_CUDA: return "CUDA call failed";
+    case DM_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case DM_ERR_NONFINITE: return "non-finite Frobenius norm (update set to zero)";
+    default: return "unknown status";
+  }
+}
+
+const char* dm_version(void) { return "0.1.0"; }
+
+}  // extern "C"

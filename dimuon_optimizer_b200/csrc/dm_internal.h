@@ -1,0 +1,212 @@
+// Internal (non-ABI) definitions of libdimuon: kernel parameter blocks,
+// workspace scalar slots and the launch entry points of each kernel file.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dm {
+
+enum { DT_BF16 = 0, DT_FP32 = 1 };
+
+// Per-matrix scalar slots (float[SC_COUNT] in the workspace).
+enum {
+  SC_SUMSQ = 0,   // ||X_0||_F^2 of the stored X_0
+  SC_INV_S = 1,   // 1 / max(||X_0||_F, 1e-30)
+  SC_INV_S2 = 2,  // its square
+  SC_VALID = 3,   // 1 when ||X_0||_F is finite, else 0 (update forced to 0)
+  SC_FINAL = 4,   // Dimuon: kappa * ||X_5||_F / ||R X_5 C||_F (0 if invalid)
+  SC_COUNT = 16
+};
+
+// Device status codes (mirror dm_status_t).
+enum { ST_OK = 0, ST_TIMEOUT = 5, ST_NONFINITE = 6 };
+
+// ------------------------------- K0 ---------------------------------------
+// Dimuon conditioning vectors R, C from the previous momentum's energies.
+struct K0Mat {
+  const float* e_row;
+  const float* e_col;
+  float* R;
+  float* C;
+  int64_t rows, cols;
+};
+constexpr int K0_MAX = 256;
+struct K0Params {
+  int count;
+  float eps;
+  K0Mat mats[K0_MAX];
+};
+
+// ------------------------------- K1 ---------------------------------------
+// Momentum update, X_0 = R M_t C (or M_t), partial sums of squares, partial
+// row / column energies.  Tiles of K1_ROWS x K1_COLS.
+constexpr int K1_ROWS = 64;
+constexpr int K1_COLS = 256;
+struct K1Mat {
+  const void* G;
+  void* M;
+  void* X0;
+  const float* R;          // null: no conditioning
+  const float* C;
+  float* part_sumsq;       // [n_rt * n_ct]
+  float* part_erow;        // [n_ct][rows], null: energies not needed
+  float* part_ecol;        // [n_rt][cols]
+  int64_t rows, cols, ldx;
+  int gdt, mdt, xdt, vec;
+  int n_rt, n_ct;
+};
+constexpr int K1_MAX = 200;
+struct K1Params {
+  int count;
+  float mu;
+  int starts[K1_MAX + 1];
+  K1Mat mats[K1_MAX];
+};
+
+// ------------------------------- K1b --------------------------------------
+// Reduction of the K1 partials: energies of M_t and the norm scalars.
+constexpr int K1B_THREADS = 256;
+struct K1bMat {
+  const float* part_sumsq;
+  const float* part_erow;
+  const float* part_ecol;
+  float* e_row;            // user output, null in Muon mode
+  float* e_col;
+  float* scal;
+  int64_t rows, cols;
+  int n_rt, n_ct;
+};
+constexpr int K1B_MAX = 200;
+struct K1bParams {
+  int count;
+  int* status;
+  int starts[K1B_MAX + 1];  // blocks per matrix: 1 + energy blocks
+  K1bMat mats[K1B_MAX];
+};
+
+// --------------------------- NS products ----------------------------------
+enum {
+  EPI_SYRK = 0,          // out = S * acc                       (symmetric)
+  EPI_POLY = 1,          // out = c * acc + b * aux             (symmetric)
+  EPI_GEMM = 2,          // out = S * (acc + a * aux)
+  EPI_FINAL_MUON = 3,    // W <- decay W - lr kappa S (acc + a aux), upd = O
+  EPI_FINAL_DIMUON = 4   // out = S (acc + a aux) = X_5, plus norm partials
+};
+
+// One product of one matrix.  Output tile grid tiles_m x tiles_n; `sym`
+// enumerates only tiles that meet the upper triangle and mirrors them.
+struct GemmMat {
+  void* out;
+  const void* aux;
+  const float* scal;      // per-matrix scalar slots
+  void* W;                // final epilogues
+  float* upd;
+  const float* R;         // Dimuon final: user-orientation R and C
+  const float* C;
+  float* part;            // Dimuon final: per-tile (sum x^2, sum y^2)
+  int ldo, ldaux, ldw;
+  int M, N, K;
+  int tiles_m, tiles_n;
+  int flags;              // bit0 a_mn, bit1 b_mn, bit2 sym, bit3 n-fast raster
+  int epi;                // EPI_*
+  int scal_idx;           // slot multiplying the result, -1 for none
+  int wdt;                // weight dtype
+  float coef_acc, coef_aux, kappa;
+};
+enum { GF_A_MN = 1, GF_B_MN = 2, GF_SYM = 4, GF_N_FAST = 8 };
+
+// fp32 SIMT products
+constexpr int SIMT_MAX = 120;
+// A operand element (i, k) at a_mn ? a[k*lda + i] : a[i*lda + k];
+// B operand element (j, k) at b_mn ? b[k*ldb + j] : b[j*ldb + k].
+struct SimtMat {
+  GemmMat g;
+  const float* a;
+  const float* b;
+  int lda, ldb;
+};
+struct SimtParams {
+  int count;
+  float lr, decay;
+  int starts[SIMT_MAX + 1];
+  SimtMat mats[SIMT_MAX];
+};
+
+// tcgen05 products (bf16 operands, fp32 accumulation in TMEM)
+constexpr int TC_BM = 128, TC_BN = 256, TC_BK = 64;
+struct TcMat {
+  CUtensorMap ta;   // A-operand map, box 64 x 64 bf16, 128-byte swizzle
+  CUtensorMap tb;   // B-operand map
+  GemmMat g;
+};
+constexpr int TC_MAX = 76;
+struct TcParams {
+  int count;
+  int total_tiles;
+  float lr, decay;
+  int* status;
+  unsigned debug;
+  int starts[TC_MAX + 1];
+  TcMat mats[TC_MAX];
+};
+
+// ------------------------------- K3 ---------------------------------------
+struct K3Mat {
+  const void* X5;
+  void* W;
+  float* upd;
+  const float* R;
+  const float* C;
+  const float* part;
+  float* scal;
+  int64_t rows, cols, ldx;
+  int xdt, wdt, vec, n_part;
+  int n_rt, n_ct;
+  float kappa;
+};
+constexpr int K3_MAX = 200;
+struct K3Params {
+  int count;
+  float lr, decay;
+  int starts[K3_MAX + 1];
+  K3Mat mats[K3_MAX];
+};
+
+// ------------------------------ thin --------------------------------------
+// Whole step of one short-side <= 32 factor in one CTA (Gram route).
+struct ThinMat {
+  const void* G;
+  void* M;
+  void* W;
+  float* upd;
+  float* e_row;           // user orientation, null in Muon mode
+  float* e_col;
+  int64_t rows, cols;
+  int gdt, mdt, wdt;
+  float kappa;
+};
+constexpr int THIN_MAX = 256;
+struct ThinParams {
+  int count;
+  int pad;                // padded short side of every factor in the launch
+  int conditioned;
+  int ns_steps;
+  float mu, lr, decay, a, b, c, eps;
+  int* status;
+  ThinMat mats[THIN_MAX];
+};
+
+// ------------------------------ launches ----------------------------------
+cudaError_t launch_k0(const K0Params& p, cudaStream_t s);
+cudaError_t launch_k1(const K1Params& p, int total_tiles, cudaStream_t s);
+cudaError_t launch_k1b(const K1bParams& p, int total_blocks, cudaStream_t s);
+cudaError_t launch_k3a(const K3Params& p, cudaStream_t s);
+cudaError_t launch_k3(const K3Params& p, int total_tiles, cudaStream_t s);
+cudaError_t launch_simt(const SimtParams& p, int total_tiles, cudaStream_t s);
+cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s);
+int tc_smem_bytes();
+cudaError_t launch_thin(const ThinParams& p, cudaStream_t s);
+
+}  // namespace dm

@@ -1,0 +1,396 @@
+// Tensor-core (tcgen05) products of the quintic Newton-Schulz iteration,
+// precision mode DM_PREC_BF16_TC:
+//   A  = X X^T             (symmetric: only tiles meeting the upper triangle)
+//   B  = b A + c A A       (symmetric; A A = A A^T since A is symmetric)
+//   X' = a X + B X         (last iteration: fused update / X_5 + norm partials)
+// sitech.ge Muon post, "Instead of SVD - Newton-Schulz": X_next = aX +
+// b(XX^T)X + c(XX^T)^2X, "efficient in bfloat16"; coefficients from
+// "Muon Optimizer 정리", "Why orthogonalise".
+//
+// Structure (one CTA per SM, persistent over a static round-robin tile list):
+//   warp 0      TMA producer: 64 x 64 bf16 boxes, 128-byte swizzle, 4 stages
+//               of (128 x 64 A-operand, 256 x 64 B-operand) in shared memory
+//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16) into one of
+//               two 256-column fp32 accumulators in tensor memory
+//   warps 2..5  epilogue: tcgen05.ld -> registers -> fused epilogue -> global
+// Operands may be K-major or MN-major per matrix (runtime descriptor bits),
+// so wide matrices and tall matrices (handled transposed) need no copies.
+// Every wait is bounded (see mbar_wait_bounded); no multicast loads are used.
+#include "dm_common.cuh"
+#include "dm_sm100.cuh"
+#include "dm_tiles.cuh"
+
+namespace dm {
+namespace {
+
+using namespace sm100;
+
+constexpr int STAGES = 4;
+constexpr int BOX_BYTES = 64 * 64 * 2;
+constexpr int A_BYTES = TC_BM * TC_BK * 2;      // 16 KB
+constexpr int B_BYTES = TC_BN * TC_BK * 2;      // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;             // two 128 x 256 fp32 accumulators
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // any single wait > 2 s is a hang
+constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
+
+struct Tile {
+  int g, lt, tm, tn;
+};
+
+__device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
+  Tile tl;
+  tl.g = find_group(p.starts, p.count, t);
+  tl.lt = t - p.starts[tl.g];
+  gemm_tile_coord(p.mats[tl.g].g, tl.lt, TC_BM, TC_BN, tl.tm, tl.tn);
+  return tl;
+}
+
+__device__ __forceinline__ void ld_bf16x8(const void* p, float v[8]) {
+  ld8(p, 0, DT_BF16, v);
+}
+__device__ __forceinline__ void st_bf16x8(void* p, const float v[8]) { st8(p, 0, DT_BF16, v); }
+
+__device__ __forceinline__ bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// Loads 32 consecutive elements of row r of a bf16 matrix (scalar tail).
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* base, int ld, int r, int c0,
+                                           int ncols, float v[32]) {
+  const __nv_bfloat16* p = base + (int64_t)r * ld + c0;
+  if (c0 + 32 <= ncols) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ld_bf16x8(p + 8 * q, v + 8 * q);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) v[q] = (c0 + q < ncols) ? __bfloat162float(p[q]) : 0.f;
+  }
+}
+
+__device__ __forceinline__ void store_row32(__nv_bfloat16* base, int ld, int r, int c0, int ncols,
+                                            const float v[32]) {
+  __nv_bfloat16* p = base + (int64_t)r * ld + c0;
+  if (c0 + 32 <= ncols) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) st_bf16x8(p + 8 * q, v + 8 * q);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 32; ++q)
+      if (c0 + q < ncols) p[q] = __float2bfloat16_rn(v[q]);
+  }
+}
+
+// Symmetric store of 32 values of row r: element (r, c) for c >= r, and its
+// mirror (c, r) for c > r.
+__device__ __forceinline__ void store_sym32(const GemmMat& g, int r, int c0, const float v[32]) {
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(g.out);
+  const int n = g.M;  // square output
+  if (c0 >= r && c0 + 32 <= n) {
+    store_row32(o, g.ldo, r, c0, n, v);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int c = c0 + q;
+      if (c < n && c >= r) o[(int64_t)r * g.ldo + c] = __float2bfloat16_rn(v[q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const int c = c0 + q;
+    if (c < n && c > r) o[(int64_t)c * g.ldo + r] = __float2bfloat16_rn(v[q]);
+  }
+}
+
+// Fused epilogue for 32 accumulator columns of one output row.
+__device__ __forceinline__ void epilogue32(const GemmMat& g, const TcParams& p, int r, int c0,
+                                           float v[32], float S, float valid, float& sx,
+                                           float& sy) {
+  switch (g.epi) {
+    case EPI_SYRK: {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] *= S;
+      store_sym32(g, r, c0, v);
+      break;
+    }
+    case EPI_POLY: {
+      float ax[32];
+      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = fmaf(g.coef_acc, v[q], g.coef_aux * ax[q]);
+      store_sym32(g, r, c0, v);
+      break;
+    }
+    case EPI_GEMM: {
+      float ax[32];
+      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = fmaf(g.coef_aux, ax[q], v[q]) * S;
+      store_row32(reinterpret_cast<__nv_bfloat16*>(g.out), g.ldo, r, c0, g.N, v);
+      break;
+    }
+    case EPI_FINAL_MUON: {
+      float ax[32];
+      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
+      const float ks = valid != 0.f ? g.kappa * S : 0.f;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = (valid != 0.f) ? fmaf(g.coef_aux, ax[q], v[q]) * ks : 0.f;
+      const int64_t wi = (int64_t)r * g.ldw + c0;
+      const bool full = c0 + 32 <= g.N;
+      const int es = g.wdt == DT_BF16 ? 2 : 4;
+      const void* wp = reinterpret_cast<const char*>(g.W) + wi * es;
+      if (full && aligned16(wp)) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float w8[8];
+          ld8(g.W, wi + 8 * q, g.wdt, w8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w8[e] = p.decay * w8[e] - p.lr * v[8 * q + e];
+          st8(g.W, wi + 8 * q, g.wdt, w8);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (c0 + q < g.N)
+            st_elem(g.W, wi + q, g.wdt, p.decay * ld_elem(g.W, wi + q, g.wdt) - p.lr * v[q]);
+      }
+      if (g.upd) {
+        if (full && aligned16(g.upd + wi)) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) st8(g.upd, wi + 8 * q, DT_FP32, v + 8 * q);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (c0 + q < g.N) g.upd[wi + q] = v[q];
+        }
+      }
+      break;
+    }
+    case EPI_FINAL_DIMUON: {
+      float ax[32];
+      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
+      const float rr = g.R[r];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        v[q] = round_to(fmaf(g.coef_aux, ax[q], v[q]) * S, DT_BF16);
+        if (c0 + q < g.N) {
+          const float y = rr * v[q] * g.C[c0 + q];
+          sx += v[q] * v[q];
+          sy += y * y;
+        }
+      }
+      store_row32(reinterpret_cast<__nv_bfloat16*>(g.out), g.ldo, r, c0, g.N, v);
+      break;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ----------------------------- TMA producer -----------------------------
+    if (lane == 0) {
+      for (int g = 0; g < p.count; ++g) {
+        tma_prefetch_map(&p.mats[g].ta);
+        tma_prefetch_map(&p.mats[g].tb);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // per-stage bits of the last armed phase
+      for (int t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x) {
+        const Tile tl = decode_tile(p, t);
+        const TcMat& mt = p.mats[tl.g];
+        const int a_mn = mt.g.flags & GF_A_MN, b_mn = mt.g.flags & GF_B_MN;
+        const int m0 = tl.tm * TC_BM, n0 = tl.tn * TC_BN;
+        const int nkb = (mt.g.K + TC_BK - 1) / TC_BK;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort, p.status, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          const int k0 = kb * TC_BK;
+#pragma unroll
+          for (int q = 0; q < TC_BM / 64; ++q) {
+            if (a_mn)
+              tma_load_2d(sa + q * BOX_BYTES, &mt.ta, &full[stage], m0 + 64 * q, k0);
+            else
+              tma_load_2d(sa + q * BOX_BYTES, &mt.ta, &full[stage], k0, m0 + 64 * q);
+          }
+#pragma unroll
+          for (int q = 0; q < TC_BN / 64; ++q) {
+            if (b_mn)
+              tma_load_2d(sb + q * BOX_BYTES, &mt.tb, &full[stage], n0 + 64 * q, k0);
+            else
+              tma_load_2d(sb + q * BOX_BYTES, &mt.tb, &full[stage], k0, n0 + 64 * q);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort) {
+        // Let the copies already in flight land before the CTA exits.
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s))
+            mbar_wait_bounded(&full[s], (armed_par >> s) & 1u, abort, nullptr, DRAIN_LIMIT_NS);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++local) {
+        const Tile tl = decode_tile(p, t);
+        const GemmMat& g = p.mats[tl.g].g;
+        const int a_mn = (g.flags & GF_A_MN) ? 1 : 0, b_mn = (g.flags & GF_B_MN) ? 1 : 0;
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort, p.status, WAIT_LIMIT_NS)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * TC_BN);
+        const uint32_t idesc = idesc_bf16(TC_BM, TC_BN, a_mn, b_mn);
+        const int nkb = (g.K + TC_BK - 1) / TC_BK;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort, p.status, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+            const uint64_t ad = a_mn ? smem_desc(sa + kk * 2048, BOX_BYTES, 1024)
+                                     : smem_desc(sa + kk * 32, 16, 1024);
+            const uint64_t bd = b_mn ? smem_desc(sb + kk * 2048, BOX_BYTES, 1024)
+                                     : smem_desc(sb + kk * 32, 16, 1024);
+            mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+      }
+      // Every MMA this thread issued has completed once `drain` flips.
+      mma_commit(drain);
+      mbar_wait_bounded(drain, 0, abort, nullptr, DRAIN_LIMIT_NS);
+    }
+  } else {
+    // ------------------------------- epilogue -------------------------------
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    int local = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
+      const Tile tl = decode_tile(p, t);
+      const GemmMat& g = p.mats[tl.g].g;
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort, p.status, WAIT_LIMIT_NS)) break;
+      tc_fence_after();
+      const int r = tl.tm * TC_BM + row_in_tile;
+      const bool row_ok = r < g.M;
+      const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
+      const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
+      float sx = 0.f, sy = 0.f;
+      const int nch = min(TC_BN, g.N - tl.tn * TC_BN + 31) / 32;  // chunks holding columns < N
+#pragma unroll 1
+      for (int ch = 0; ch < TC_BN / 32; ++ch) {
+        float v[32];
+        tmem_ld32(tmem_base + (uint32_t)(acc * TC_BN + ch * 32) + ((uint32_t)(quarter * 32) << 16),
+                  v);
+        if (row_ok && ch < nch) epilogue32(g, p, r, tl.tn * TC_BN + ch * 32, v, S, valid, sx, sy);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (g.epi == EPI_FINAL_DIMUON) {
+        // One (sum x^2, sum y^2) pair per epilogue warp; no barrier needed.
+        sx = warp_sum(sx);
+        sy = warp_sum(sy);
+        if (lane == 0) {
+          const int slot = (tl.tm * g.tiles_n + tl.tn) * 4 + quarter;
+          g.part[2 * slot] = sx;
+          g.part[2 * slot + 1] = sy;
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+int tc_smem_bytes() { return SMEM_BYTES; }
+
+cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s) {
+  if (p.total_tiles <= 0 || grid <= 0) return cudaSuccess;
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(tc_ns_product, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  tc_ns_product<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace dm

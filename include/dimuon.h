@@ -1,0 +1,166 @@
+/*
+ * dimuon.h - C ABI of libdimuon.so: the Muon optimizer step for 2-D hidden
+ * weight matrices, with Dimuon's diagonal conditioning as an optional mode,
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The step, per matrix (sources: web pages, cited by title and section):
+ *   1. M_t = mu M_{t-1} + G
+ *        "Muon Optimizer 정리" (dongju923.github.io), "Update rule", eq. (1).
+ *   2. Dimuon only: R = diag((e_row/mean(e_row) + eps)^(-1/4)),
+ *      C = diag((e_col/mean(e_col) + eps)^(-1/4)) from the row / column sums
+ *      of squares of the PREVIOUS momentum M_{t-1}; X_0 = R M_t C.
+ *      Muon: X_0 = M_t.
+ *        "Dimuon: LoRA 에 맞춰 다시 짠 Muon" (lameproof.com optim-book),
+ *        "-1/4 power from both sides", "Why the *last* momentum", Problem 4.
+ *   3. X <- X_0 / ||X_0||_F, then ns_steps times
+ *      X <- a X + b (X X^T) X + c (X X^T)^2 X, (a,b,c) = (3.4445,-4.7750,2.0315),
+ *      on the short side of the matrix (tall matrices are handled transposed).
+ *        sitech.ge Muon post, "Instead of SVD - Newton-Schulz";
+ *        "Muon Optimizer 정리", "Why orthogonalise".
+ *   4. Dimuon only: Y = R X C rescaled to ||X||_F ("the norm is fixed
+ *      afterwards", Dimuon page, Problem 4 (c)).  Muon: Y = X.
+ *   5. O = kappa Y, kappa = 1 (DM_SCALE_NONE) or
+ *      scale_coef * sqrt(max(rows, cols)) (DM_SCALE_MOONSHOT, RMS matched to
+ *      AdamW: sitech.ge, "From speedrun to real training").
+ *   6. W_t = (1 - lr * weight_decay) W_{t-1} - lr O   (decoupled decay:
+ *      "Muon Optimizer 정리", "Scaling up"; eq. (3)).
+ *
+ * Conventions
+ *   - Every matrix is row-major and contiguous (leading dimension == cols).
+ *   - All pointers in dm_matrix_t and the workspace are DEVICE pointers on the
+ *     current CUDA device; hyper-parameters are host values.
+ *   - The caller owns every buffer.  The library allocates no device memory
+ *     and keeps no state between calls apart from a host-side cache of
+ *     launch plans keyed by the workspace pointer and the matrix shapes.
+ *   - dm_muon_step / dm_dimuon_step validate their arguments synchronously and
+ *     return an error before launching anything; otherwise they enqueue all
+ *     work on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     return without synchronising.  No C++ exception crosses this ABI.
+ *   - Conditions found on the device (a non-finite Frobenius norm, a bounded
+ *     wait that ran out) are written to a status word inside the workspace;
+ *     dm_read_device_status synchronises the stream and reads it.  Each step
+ *     clears the word at its start.
+ *   - Calls are re-entrant for distinct workspaces.  Two steps that share a
+ *     workspace must be ordered on the device (same stream, or events).
+ *   - The enqueued work contains no host synchronisation and no allocation,
+ *     so a step can be captured into a CUDA graph by the caller.
+ */
+#ifndef DIMUON_H_
+#define DIMUON_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DM_OK = 0,
+  DM_ERR_INVALID_ARG = 1,     /* null pointer, non-positive shape, bad enum  */
+  DM_ERR_UNSUPPORTED = 2,     /* dtype / mode combination not provided       */
+  DM_ERR_WORKSPACE = 3,       /* workspace null, misaligned or too small      */
+  DM_ERR_CUDA = 4,            /* a CUDA runtime / driver call failed          */
+  DM_ERR_DEVICE_TIMEOUT = 5,  /* device status: a bounded wait gave up        */
+  DM_ERR_NONFINITE = 6        /* device status: non-finite ||X_0||_F; that
+                                 matrix got O = 0 (its W was only decayed)    */
+} dm_status_t;
+
+typedef enum { DM_BF16 = 0, DM_FP32 = 1 } dm_dtype_t;
+
+/* Arithmetic of the Newton-Schulz products for matrices whose short side is
+ * larger than DM_THIN_MAX.  Matrices with a short side <= DM_THIN_MAX take the
+ * thin-factor path (fp64 Gram iteration) in both modes. */
+typedef enum {
+  DM_PREC_FP32 = 0,     /* fp32 SIMT products, fp32 intermediates           */
+  DM_PREC_BF16_TC = 1   /* bf16 operands on tcgen05 tensor cores, fp32
+                           accumulation in tensor memory                      */
+} dm_precision_t;
+
+typedef enum { DM_SCALE_NONE = 0, DM_SCALE_MOONSHOT = 1 } dm_scale_t;
+
+#define DM_THIN_MAX 32
+
+/* One matrix of the group.  Orientation: rows x cols as stored by the caller.
+ *   weight      in/out  rows x cols, weight_dtype
+ *   grad        in      rows x cols, grad_dtype
+ *   momentum    in/out  rows x cols, momentum_dtype; all zero before step 1
+ *   row_energy  in/out  fp32[rows]; Dimuon only (ignored by dm_muon_step):
+ *                       in = row sums of squares of M_{t-1} (zeros before
+ *                       step 1), out = those of the stored M_t
+ *   col_energy  in/out  fp32[cols]; as row_energy, for columns
+ *   update_out  out     optional fp32 rows x cols (NULL to skip): O_t       */
+typedef struct {
+  int64_t rows;
+  int64_t cols;
+  void* weight;
+  int32_t weight_dtype;
+  int32_t grad_dtype;
+  const void* grad;
+  void* momentum;
+  int32_t momentum_dtype;
+  int32_t reserved0;
+  float* row_energy;
+  float* col_energy;
+  float* update_out;
+} dm_matrix_t;
+
+typedef struct {
+  float mu;             /* momentum coefficient                         */
+  float lr;             /* eta                                          */
+  float weight_decay;   /* lambda (decoupled)                           */
+  int32_t ns_steps;     /* Newton-Schulz iterations, >= 1               */
+  float a, b, c;        /* quintic coefficients                         */
+  float cond_eps;       /* Dimuon damping, default 1e-4                 */
+  int32_t scale_mode;   /* dm_scale_t                                   */
+  float scale_coef;     /* DM_SCALE_MOONSHOT coefficient, default 0.2   */
+  int32_t precision;    /* dm_precision_t                               */
+  uint32_t debug_flags; /* 0 in production; bits below are test hooks   */
+} dm_hparams_t;
+
+/* debug_flags bits (test hooks; none of them changes the arithmetic) */
+#define DM_DBG_NO_THIN 0x1u       /* send short-side <= DM_THIN_MAX matrices
+                                     down the Newton-Schulz path as well   */
+
+/* Fills *hp with the defaults: mu 0.95, lr 0.02, wd 0, ns_steps 5,
+ * (a,b,c) = (3.4445, -4.7750, 2.0315), cond_eps 1e-4, DM_SCALE_NONE,
+ * scale_coef 0.2, DM_PREC_BF16_TC, debug_flags 0. */
+void dm_default_hparams(dm_hparams_t* hp);
+
+/* Bytes of device workspace a step over `mats[0..n)` needs with these
+ * hyper-parameters; `conditioned` = 0 for dm_muon_step, 1 for
+ * dm_dimuon_step.  Host-only; touches no device memory.  The workspace must
+ * be 256-byte aligned; its contents need no initialisation. */
+dm_status_t dm_workspace_size(const dm_matrix_t* mats, int n,
+                              const dm_hparams_t* hp, int conditioned,
+                              size_t* bytes);
+
+/* One Muon step over the group (steps 1, 3, 5, 6 above; row_energy and
+ * col_energy are ignored).  Asynchronous on `stream`. */
+dm_status_t dm_muon_step(const dm_matrix_t* mats, int n,
+                         const dm_hparams_t* hp, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* One Dimuon step over the group (steps 1-6).  row_energy / col_energy must
+ * be non-null for every matrix.  Asynchronous on `stream`. */
+dm_status_t dm_dimuon_step(const dm_matrix_t* mats, int n,
+                           const dm_hparams_t* hp, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the device status word of the last step
+ * that used `workspace` into *out (DM_OK, DM_ERR_NONFINITE or
+ * DM_ERR_DEVICE_TIMEOUT).  Returns DM_ERR_CUDA if the synchronisation or the
+ * copy fails. */
+dm_status_t dm_read_device_status(const void* workspace, void* stream,
+                                  int32_t* out);
+
+/* Static, NUL-terminated description of a status code. */
+const char* dm_status_string(int32_t status);
+
+/* Library version, "major.minor.patch". */
+const char* dm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DIMUON_H_ */

@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+the header declares, struct layouts agree, and argument errors come back
+synchronously before anything is launched (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dimuon_optimizer_b200 as dm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dimuon.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\S.*?\b(dm_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) >= 7
+    lib = ctypes.CDLL(dm.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(dm.EXPORTED)
+
+
+def test_struct_layouts():
+    assert ctypes.sizeof(dm.dm_matrix_t) == 80
+    assert ctypes.sizeof(dm.dm_hparams_t) == 48
+    assert dm.dm_matrix_t.update_out.offset == 72
+    assert dm.dm_hparams_t.debug_flags.offset == 44
+
+
+def test_defaults_and_strings():
+    hp = dm.dm_default_hparams()
+    assert (round(hp.a, 4), round(hp.b, 4), round(hp.c, 4)) == (3.4445, -4.775, 2.0315)
+    assert hp.ns_steps == 5 and abs(hp.mu - 0.95) < 1e-7 and abs(hp.cond_eps - 1e-4) < 1e-10
+    assert hp.precision == dm.DM_PREC_BF16_TC
+    assert dm.dm_status_string(dm.DM_OK) == "ok"
+    assert "workspace" in dm.dm_status_string(dm.DM_ERR_WORKSPACE)
+    assert dm.dm_status_string(1234) == "unknown status"
+    assert re.match(r"\d+\.\d+\.\d+", dm.dm_version())
+
+
+def fake_matrix(rows, cols, wdt=dm.DM_BF16, energies=True):
+    m = dm.dm_matrix_t()
+    m.rows, m.cols = rows, cols
+    m.weight, m.grad, m.momentum = 0x1000, 0x2000, 0x3000
+    m.weight_dtype = m.grad_dtype = m.momentum_dtype = wdt
+    if energies:
+        m.row_energy, m.col_energy = 0x4000, 0x5000
+    return m
+
+
+def test_workspace_size_host_only():
+    hp = dm.dm_default_hparams()
+    thin = dm.dm_workspace_size([fake_matrix(8, 4096)], hp, 1)
+    big = dm.dm_workspace_size([fake_matrix(1024, 1024)], hp, 0)
+    big_cond = dm.dm_workspace_size([fake_matrix(1024, 1024)], hp, 1)
+    assert thin == 1024                       # thin factors need no scratch
+    assert big >= 2 * 1024 * 1024 * 2 + 2 * 1024 * 1024 * 2   # X ping-pong + A + B
+    assert big_cond > big
+    hp32 = dm.dm_default_hparams(precision=dm.DM_PREC_FP32)
+    assert dm.dm_workspace_size([fake_matrix(1024, 1024)], hp32, 0) > big
+    # the thin threshold can be lifted for testing
+    hp_nt = dm.dm_default_hparams(debug_flags=dm.DM_DBG_NO_THIN)
+    assert dm.dm_workspace_size([fake_matrix(8, 4096)], hp_nt, 0) > thin
+
+
+@pytest.mark.parametrize("mutate,code", [
+    (lambda m, h: setattr(m, "rows", 0), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(m, "cols", -3), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(m, "grad", None), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(m, "weight_dtype", 7), dm.DM_ERR_UNSUPPORTED),
+    (lambda m, h: setattr(h, "ns_steps", 0), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(h, "precision", 5), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(h, "scale_mode", 9), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(h, "lr", float("nan")), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(m, "row_energy", None), dm.DM_ERR_INVALID_ARG),
+])
+def test_argument_errors_are_synchronous(mutate, code):
+    m = fake_matrix(64, 96)
+    hp = dm.dm_default_hparams()
+    mutate(m, hp)
+    # validated before any device call: these return without touching a GPU
+    assert dm.dm_dimuon_step([m], hp, (0x100000, 1 << 30), stream=0) == code
+
+
+def test_workspace_errors():
+    m = fake_matrix(64, 96)
+    hp = dm.dm_default_hparams()
+    need = dm.dm_workspace_size([m], hp, 0)
+    assert dm.dm_muon_step([m], hp, (0, need), stream=0) == dm.DM_ERR_WORKSPACE
+    assert dm.dm_muon_step([m], hp, (0x100010, need), stream=0) == dm.DM_ERR_WORKSPACE   # misaligned
+    assert dm.dm_muon_step([m], hp, (0x100000, need - 1), stream=0) == dm.DM_ERR_WORKSPACE
+
+
+def test_muon_ignores_missing_energies():
+    m = fake_matrix(64, 96, energies=False)
+    hp = dm.dm_default_hparams()
+    assert dm.dm_workspace_size([m], hp, 0) > 0
+    with pytest.raises(dm.DimuonError):
+        dm.dm_workspace_size([m], hp, 1)

@@ -1,0 +1,282 @@
+"""GPU parity: the CUDA library against the fp64 oracle, element by element,
+on the same seeded inputs (teacher-forced every step), through the C ABI.
+
+Tolerances (written here, derived from the method's arithmetic):
+  O_t          relative Frobenius <= 1e-5 (fp32 mode, thin path),
+               <= 3e-2 (bf16 tensor-core mode)
+  sing. values of O_t / kappa within 0.05
+  M_t          <= 1 storage ulp per element
+  W_t          <= 1 storage ulp of (1 - lr wd) W_{t-1} - lr O_t (GPU's own O_t)
+  energies     relative 2e-5 of the sums of squares of the stored M_t
+"""
+import numpy as np
+import pytest
+import torch
+
+import dimuon_optimizer_b200 as dm
+import oracle as orc
+import workloads
+from gpu_harness import (TOL_BF16, TOL_FP32, Group, rel_fro, run_gpu_step, step_and_compare,
+                         to_dev, to_host)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+BF, F32 = dm.DM_BF16, dm.DM_FP32
+
+
+def gaussian(shapes, seed, scale_cols=False):
+    rng = np.random.default_rng(seed)
+    out = []
+    for (r, c) in shapes:
+        g = rng.standard_normal((r, c))
+        if scale_cols:
+            g *= rng.lognormal(0.0, 1.0, c)[None, :]
+        out.append(g)
+    return out
+
+
+def hparams(precision, **kw):
+    return dm.dm_default_hparams(precision=precision, **kw)
+
+
+# --------------------------------------------------------------------------
+# Newton-Schulz path, fp32 SIMT products
+# --------------------------------------------------------------------------
+NS_SHAPES = [(64, 96), (130, 200), (300, 140), (257, 513), (40, 33)]
+
+
+@pytest.mark.parametrize("cond", [False, True])
+@pytest.mark.parametrize("dts", [(BF, BF, BF), (F32, F32, F32), (BF, BF, F32)])
+def test_fp32_mode_ns_path(cond, dts):
+    wdt, gdt, mdt = dts
+    grp = Group(NS_SHAPES, wdt, gdt, mdt, cond=cond, seed=11)
+    hp = hparams(dm.DM_PREC_FP32, weight_decay=0.05, scale_mode=dm.DM_SCALE_MOONSHOT)
+    ws = None
+    for t in range(3):
+        _, ws = step_and_compare(grp, gaussian(NS_SHAPES, 100 + t, scale_cols=True), hp,
+                                 TOL_FP32, ws=ws)
+
+
+# --------------------------------------------------------------------------
+# Newton-Schulz path, bf16 tcgen05 products
+# --------------------------------------------------------------------------
+TC_SHAPES = [(384, 640), (700, 260), (257, 513), (40, 100), (128, 256), (520, 136)]
+
+
+@pytest.mark.parametrize("cond", [False, True])
+def test_tc_mode_ns_path(cond):
+    grp = Group(TC_SHAPES, BF, BF, BF, cond=cond, seed=12)
+    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.1, scale_mode=dm.DM_SCALE_MOONSHOT)
+    ws = None
+    for t in range(3):
+        rep, ws = step_and_compare(grp, gaussian(TC_SHAPES, 200 + t, scale_cols=True), hp,
+                                   TOL_BF16, ws=ws)
+    assert max(rep.o_err) < 2e-2
+
+
+def test_tc_mode_fp32_storage():
+    shapes = [(300, 520), (520, 300)]
+    grp = Group(shapes, F32, F32, F32, cond=True, seed=13)
+    hp = hparams(dm.DM_PREC_BF16_TC)
+    ws = None
+    for t in range(2):
+        _, ws = step_and_compare(grp, gaussian(shapes, 300 + t), hp, TOL_BF16, ws=ws)
+
+
+@pytest.mark.parametrize("ns_steps", [1, 2, 6])
+def test_ns_step_counts(ns_steps):
+    shapes = [(200, 330), (330, 200)]
+    for prec, tol in ((dm.DM_PREC_FP32, TOL_FP32), (dm.DM_PREC_BF16_TC, TOL_BF16)):
+        grp = Group(shapes, BF, BF, F32, cond=True, seed=14)
+        hp = hparams(prec, ns_steps=ns_steps)
+        ws = None
+        for t in range(2):
+            _, ws = step_and_compare(grp, gaussian(shapes, 400 + t), hp, tol, ws=ws)
+
+
+# --------------------------------------------------------------------------
+# thin factors (Gram route, one CTA per factor)
+# --------------------------------------------------------------------------
+THIN_SHAPES = [(4, 16), (2, 100), (8, 4096), (4096, 8), (17, 333), (32, 4096), (4096, 32),
+               (1, 50), (50, 1), (31, 31)]
+
+
+@pytest.mark.parametrize("cond", [False, True])
+@pytest.mark.parametrize("mdt", [F32, BF])
+def test_thin_path(cond, mdt):
+    grp = Group(THIN_SHAPES, BF, BF, mdt, cond=cond, seed=15)
+    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.01)
+    ws = None
+    for t in range(3):
+        _, ws = step_and_compare(grp, gaussian(THIN_SHAPES, 500 + t, scale_cols=True), hp,
+                                 TOL_FP32, ws=ws)
+
+
+def test_thin_threshold_hook_matches_ns_path():
+    """The same thin factors through the Newton-Schulz kernels (test hook)
+    agree with the oracle too."""
+    shapes = [(8, 300), (300, 8), (32, 257)]
+    grp = Group(shapes, F32, F32, F32, cond=True, seed=16)
+    hp = hparams(dm.DM_PREC_FP32, debug_flags=dm.DM_DBG_NO_THIN)
+    ws = None
+    for t in range(2):
+        _, ws = step_and_compare(grp, gaussian(shapes, 600 + t, scale_cols=True), hp, TOL_FP32,
+                                 ws=ws)
+
+
+# --------------------------------------------------------------------------
+# invariants and edge cases
+# --------------------------------------------------------------------------
+def test_first_dimuon_step_equals_muon():
+    """'Why the *last* momentum': with M_0 = 0 the conditioning is off."""
+    shapes = [(96, 160), (16, 300)]
+    g = gaussian(shapes, 700)
+    outs = []
+    for cond in (False, True):
+        grp = Group(shapes, F32, F32, F32, cond=cond, seed=17)
+        run_gpu_step(grp, g, hparams(dm.DM_PREC_FP32))
+        outs.append([to_host(u) for u in grp.upd])
+    for a, b in zip(*outs):
+        assert rel_fro(b, a) < 1e-6
+
+
+def test_nonfinite_gradient_reports_and_only_decays():
+    shapes = [(64, 128), (8, 256)]
+    g = gaussian(shapes, 800)
+    g[0][3, 5] = np.inf
+    g[1][2, 7] = np.nan
+    grp = Group(shapes, F32, F32, F32, cond=False, seed=18)
+    W0 = [to_host(w) for w in grp.W]
+    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.5, lr=0.1)
+    ws, _ = run_gpu_step(grp, g, hp)
+    assert dm.dm_read_device_status(ws) == dm.DM_ERR_NONFINITE
+    decay = np.float32(1) - np.float32(0.1) * np.float32(0.5)
+    for w0, w in zip(W0, grp.W):
+        np.testing.assert_allclose(to_host(w), np.float32(decay) * w0.astype(np.float32),
+                                   rtol=1e-7)
+    # a clean step on the same workspace clears the status word
+    grp2 = Group(shapes, F32, F32, F32, cond=False, seed=18)
+    run_gpu_step(grp2, gaussian(shapes, 801), hp, ws)
+    assert dm.dm_read_device_status(ws) == dm.DM_OK
+
+
+def test_zero_gradient_gives_zero_update():
+    shapes = [(64, 128), (4, 64)]
+    for prec in (dm.DM_PREC_FP32, dm.DM_PREC_BF16_TC):
+        for cond in (False, True):
+            grp = Group(shapes, F32, F32, F32, cond=cond, seed=19)
+            W0 = [to_host(w) for w in grp.W]
+            ws, _ = run_gpu_step(grp, [np.zeros(s) for s in shapes], hparams(prec))
+            assert dm.dm_read_device_status(ws) == dm.DM_OK
+            for w0, w, u in zip(W0, grp.W, grp.upd):
+                assert np.all(to_host(u) == 0.0)
+                np.testing.assert_array_equal(to_host(w), w0)
+
+
+def test_empty_group():
+    hp = hparams(dm.DM_PREC_BF16_TC)
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    assert dm.dm_muon_step([], hp, ws) == dm.DM_OK
+    assert dm.dm_read_device_status(ws) == dm.DM_OK
+
+
+def test_cuda_graph_capture_matches_eager():
+    shapes = [(256, 384), (384, 256), (8, 512)]
+    g = gaussian(shapes, 900)
+    hp = hparams(dm.DM_PREC_BF16_TC)
+    eager = Group(shapes, BF, BF, BF, cond=True, seed=20)
+    graphed = Group(shapes, BF, BF, BF, cond=True, seed=20)
+    ws_e, _ = run_gpu_step(eager, g, hp)
+    G = [to_dev(x, BF) for x in g]
+    mats = graphed.matrices(G)
+    ws = torch.empty(dm.dm_workspace_size(mats, hp, 1), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        dm.check(dm.dm_dimuon_step(mats, hp, ws, stream=s))
+    graph.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(eager.W, graphed.W):
+        assert torch.equal(a, b)
+    for a, b in zip(eager.er, graphed.er):
+        assert torch.equal(a, b)
+
+
+# --------------------------------------------------------------------------
+# the workloads
+# --------------------------------------------------------------------------
+def test_toy_lora_factor_two_steps():
+    """4x16 fp32 toy: step 1 unconditioned (71 % top-4 share printed on the
+    Dimuon page), step 2 conditioned by step 1's momentum."""
+    G, _ = workloads.toy_lora_factor()
+    grp = Group([(4, 16)], F32, F32, F32, cond=True, seed=0)
+    hp = dm.dm_default_hparams(precision=dm.DM_PREC_FP32)
+    shares = []
+    for t in range(2):
+        step_and_compare(grp, [G], hp, TOL_FP32)
+        shares.append(orc.top_column_share(to_host(grp.upd[0]), [12, 13, 14, 15]))
+    assert round(shares[0], 2) == 0.71
+    assert shares[1] < 0.25
+
+
+@pytest.mark.parametrize("prec,tol", [(dm.DM_PREC_FP32, TOL_FP32), (dm.DM_PREC_BF16_TC, TOL_BF16)])
+def test_square_1024(prec, tol):
+    shapes = workloads.single_square_shapes()
+    grp = Group(shapes, BF, BF, BF, cond=False, seed=1)
+    step_and_compare(grp, workloads.gaussian_grads(shapes, 1), hparams(prec), tol)
+
+
+def test_gpt2_small_group():
+    shapes = workloads.gpt2_small_shapes()
+    grads = workloads.gpt2_small_grads()
+    grp = Group(shapes, BF, BF, BF, cond=False, seed=2)
+    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.1, scale_mode=dm.DM_SCALE_MOONSHOT)
+    rep, _ = step_and_compare(grp, grads, hp, TOL_BF16, sample=list(range(12)))
+    assert len(rep.o_err) == 12
+
+
+@pytest.mark.slow
+def test_large_batch_sampled():
+    """The full large batch in one grouped call; the oracle checks one square
+    and one tall matrix (each takes the oracle tens of seconds)."""
+    shapes = workloads.large_batch_shapes()
+    rng = np.random.default_rng(3)
+    grads = [rng.standard_normal(s, dtype=np.float32) for s in shapes]
+    grp = Group(shapes, BF, BF, BF, cond=False, seed=3)
+    hp = hparams(dm.DM_PREC_BF16_TC)
+    rep, _ = step_and_compare(grp, grads, hp, TOL_BF16, sample=[0, 15], check_sv=False)
+    assert max(rep.o_err) < 2e-2
+
+
+@pytest.mark.parametrize("r", [2, 8, 32])
+def test_lora_batch_twenty_steps(r):
+    """224 projections (A r x 4096, B 4096 x r), fp32 momentum, bf16 weights,
+    Dimuon, 20 steps: teacher-forced parity on a sample each step, dead rows
+    of B capped at a 10x per-side gain, and a free-running oracle rerun of
+    one projection at the end."""
+    shapes = workloads.lora_shapes(r)
+    stream = workloads.LoraGradStream(r)
+    grp = Group(shapes, BF, BF, F32, cond=True, seed=4)
+    lr = {2: 0.018, 8: 0.010, 32: 0.010}[r]
+    hp = hparams(dm.DM_PREC_BF16_TC, lr=lr)
+    ws = None
+    h = orc.HParams(lr=lr)
+    free = None
+    for t in range(1, 21):
+        grads = stream.step(t)
+        if free is None:
+            free = dict(W=to_host(grp.W[1]), M=to_host(grp.M[1]), er=np.zeros(shapes[1][0]),
+                        ec=np.zeros(shapes[1][1]))
+        g1 = to_host(to_dev(grads[1], BF))
+        fr = orc.dimuon_step(free["W"], g1, free["M"], free["er"], free["ec"], h,
+                             momentum_dtype="fp32", weight_dtype="bf16")
+        free = dict(W=fr.W, M=fr.M, er=fr.e_row, ec=fr.e_col)
+        sample = [0, 1, 2 * 111, 2 * 111 + 1, len(shapes) - 1]
+        _, ws = step_and_compare(grp, grads, hp, TOL_FP32, ws=ws, sample=sample)
+        if 2 <= t <= 6:
+            # rows of B whose previous gradient was zero get the 10x cap
+            dead = stream.dead[0]
+            er = to_host(grp.er[1])
+            assert np.all(er[dead] == 0.0) if t <= 5 else True
+    assert rel_fro(to_host(grp.W[1]), free["W"]) < 3e-2
