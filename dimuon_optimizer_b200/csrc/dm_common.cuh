@@ -31,6 +31,18 @@ __device__ __forceinline__ float round_to(float v, int dt) {
   return dt == DT_BF16 ? __bfloat162float(__float2bfloat16_rn(v)) : v;
 }
 
+// M_t = mu M_{t-1} + G evaluated in fp64 and rounded once to the storage
+// dtype.  The product of an fp32 and a bf16 / fp32 value is exact in fp64, so
+// this is the correctly rounded momentum (no fp32 -> bf16 double rounding).
+__device__ __forceinline__ float momentum_value(float mu, float mprev, float g, int dt) {
+  const double v = fma((double)mu, (double)mprev, (double)g);
+  return dt == DT_BF16 ? __bfloat162float(__double2bfloat16(v)) : __double2float_rn(v);
+}
+
+// Squared Frobenius norms below this floor give a zero update (fp32 cannot
+// normalise them: the reciprocal square overflows).
+constexpr double NORM2_FLOOR = 1e-30;
+
 // 8 consecutive elements (16-byte aligned for bf16, 32-byte for fp32).
 __device__ __forceinline__ void ld8(const void* p, int64_t i, int dt, float v[8]) {
   if (dt == DT_BF16) {

@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(256) k1_momentum(const __grid_constant__ K1Par
         ld8(mt.M, base, mt.mdt, m8);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          m8[q] = round_to(fmaf(p.mu, m8[q], g8[q]), mt.mdt);
+          m8[q] = momentum_value(p.mu, m8[q], g8[q], mt.mdt);
           x8[q] = round_to(rs * m8[q] * cscale[q], mt.xdt);
           rsum += m8[q] * m8[q];
           csum[q] += m8[q] * m8[q];
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(256) k1_momentum(const __grid_constant__ K1Par
         const int64_t c = c0 + q;
         if (c < mt.cols) {
           const float gv = ld_elem(mt.G, base + q, mt.gdt);
-          const float mv = round_to(fmaf(p.mu, ld_elem(mt.M, base + q, mt.mdt), gv), mt.mdt);
+          const float mv = momentum_value(p.mu, ld_elem(mt.M, base + q, mt.mdt), gv, mt.mdt);
           const float xv = round_to(rs * mv * cscale[q], mt.xdt);
           st_elem(mt.M, base + q, mt.mdt, mv);
           st_elem(mt.X0, r * mt.ldx + c, mt.xdt, xv);
@@ -141,14 +141,16 @@ __global__ void __launch_bounds__(K1B_THREADS) k1b_reduce(const __grid_constant_
     for (int i = threadIdx.x; i < nt; i += blockDim.x) s += (double)mt.part_sumsq[i];
     s = block_sum_d(s, red);
     if (threadIdx.x == 0) {
-      const bool ok = isfinite(s);
-      const double nrm = sqrt(s);
-      const double inv = ok ? 1.0 / fmax(nrm, 1e-30) : 0.0;
+      // A non-finite norm is reported; a norm below the floor is a zero
+      // update.  Either way the update of this matrix is forced to zero.
+      const bool finite = isfinite(s);
+      const bool ok = finite && s >= NORM2_FLOOR;
+      const double inv = ok ? 1.0 / sqrt(s) : 0.0;
       mt.scal[SC_SUMSQ] = (float)s;
       mt.scal[SC_INV_S] = (float)inv;
       mt.scal[SC_INV_S2] = (float)(inv * inv);
       mt.scal[SC_VALID] = ok ? 1.f : 0.f;
-      if (!ok) raise_status(p.status, ST_NONFINITE);
+      if (!finite) raise_status(p.status, ST_NONFINITE);
     }
     return;
   }
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(256) k3_apply(const __grid_constant__ K3Params
         ld8(mt.W, base, mt.wdt, w8);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          o8[q] = rs * x8[q] * cs[q];
+          o8[q] = f != 0.f ? rs * x8[q] * cs[q] : 0.f;
           w8[q] = p.decay * w8[q] - p.lr * o8[q];
         }
         st8(mt.W, base, mt.wdt, w8);
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(256) k3_apply(const __grid_constant__ K3Params
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (c0 + q < mt.cols) {
-          const float o = rs * ld_elem(mt.X5, r * mt.ldx + c0 + q, mt.xdt) * cs[q];
+          const float o = f != 0.f ? rs * ld_elem(mt.X5, r * mt.ldx + c0 + q, mt.xdt) * cs[q] : 0.f;
           st_elem(mt.W, base + q, mt.wdt, p.decay * ld_elem(mt.W, base + q, mt.wdt) - p.lr * o);
           if (mt.upd) mt.upd[base + q] = o;
         }

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(256) thin_step(const __grid_constant__ ThinPar
       float m = 0.f;
       if (i < r && kk < cw) {
         const int64_t o = off(i, k0 + kk);
-        m = round_to(fmaf(p.mu, ld_elem(mt.M, o, mt.mdt), ld_elem(mt.G, o, mt.gdt)), mt.mdt);
+        m = momentum_value(p.mu, ld_elem(mt.M, o, mt.mdt), ld_elem(mt.G, o, mt.gdt), mt.mdt);
         st_elem(mt.M, o, mt.mdt, m);
       }
       s.ms[i][kk] = m;
@@ -170,8 +170,9 @@ __global__ void __launch_bounds__(256) thin_step(const __grid_constant__ ThinPar
   }
   __syncthreads();
   const double s2 = s.sc[0];
-  const bool valid = isfinite(s2);
-  const double inv_s2 = s2 > 0.0 ? 1.0 / s2 : 0.0;
+  const bool finite = isfinite(s2);
+  const bool valid = finite && s2 >= NORM2_FLOOR;  // else the update is zero
+  const double inv_s2 = valid ? 1.0 / s2 : 0.0;
   for (int idx = tid; idx < RP * RP; idx += 256) {
     const int i = idx / RP, j = idx % RP;
     s.u.it.A[i][j] = valid ? s.G[i][j] * inv_s2 : 0.0;
@@ -206,11 +207,10 @@ __global__ void __launch_bounds__(256) thin_step(const __grid_constant__ ThinPar
   ny = block_sum_d(ny, s.red);
   double factor = 0.0;
   if (valid) {
-    factor = (double)mt.kappa / fmax(sqrt(s2), 1e-30);
+    factor = (double)mt.kappa / sqrt(s2);
     if (on) factor = ny > 0.0 ? factor * sqrt(nx / ny) : 0.0;
-  } else if (tid == 0) {
-    raise_status(p.status, ST_NONFINITE);
   }
+  if (!finite && tid == 0) raise_status(p.status, ST_NONFINITE);
   for (int idx = tid; idx < RP * RP; idx += 256) {
     const int i = idx / RP, j = idx % RP;
     s.u.it.T[i][j] = factor * s.u.it.P[i][j];
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(256) thin_step(const __grid_constant__ ThinPar
       double acc = 0.0;
 #pragma unroll 8
       for (int j = 0; j < RP; ++j) acc = fma(s.u.it.T[i][j], s.xs[j][kk_o], acc);
-      s.ms[i][kk_o] = (float)((double)s.Rv[i] * acc * (double)s.Cc[kk_o]);
+      s.ms[i][kk_o] = factor != 0.0 ? (float)((double)s.Rv[i] * acc * (double)s.Cc[kk_o]) : 0.f;
     }
     __syncthreads();
     for (int idx = tid; idx < RP * CH; idx += 256) {

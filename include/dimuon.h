@@ -63,7 +63,9 @@ typedef enum {
   DM_ERR_CUDA = 4,            /* a CUDA runtime / driver call failed          */
   DM_ERR_DEVICE_TIMEOUT = 5,  /* device status: a bounded wait gave up        */
   DM_ERR_NONFINITE = 6        /* device status: non-finite ||X_0||_F; that
-                                 matrix got O = 0 (its W was only decayed)    */
+                                 matrix got O = 0 (its W was only decayed).
+                                 A norm below 1e-15 also gives O = 0, without
+                                 a status (nothing to normalise).             */
 } dm_status_t;
 
 typedef enum { DM_BF16 = 0, DM_FP32 = 1 } dm_dtype_t;

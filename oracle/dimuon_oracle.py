@@ -39,9 +39,10 @@ the repository's design notes):
     ([MuonNote], "Scaling up": AdamW's weight decay).
   * Tall matrices are orthogonalised on their short side: X is transposed so
     that rows <= cols; R and C swap roles; the result is transposed back.
-  * The Frobenius normalisation divides by max(||X_0||_F, 1e-30); a
-    non-finite norm makes the update O_t zero (W is only decayed) and is
-    reported as a flag.
+  * Degenerate norms: when ||X_0||_F is non-finite, or below 1e-15 (its
+    square below 1e-30, where fp32 cannot form 1/||X_0||^2), the update O_t
+    is zero and W is only decayed; a non-finite norm is also reported as a
+    flag.
   * Hyper-parameters reach the CUDA library as float32; the oracle rounds each
     scalar through float32 before using it in fp64 arithmetic.
 
@@ -62,7 +63,7 @@ NS_C = 2.0315
 NS_STEPS = 5
 COND_EPS = 1e-4          # [Dimuon], Problem 4: (relative energy + 1e-4)^(-1/4)
 MOONSHOT_COEF = 0.2      # RMS-matching coefficient (see module docstring)
-NORM_FLOOR = 1e-30
+NORM_FLOOR = 1e-15      # ||X_0||_F below this: zero update (see module docstring)
 
 SCALE_NONE = 0
 SCALE_MOONSHOT = 1
@@ -166,7 +167,7 @@ def frobenius_normalise(X):
     """X / ||X||_F ([Sitech], "Instead of SVD - Newton-Schulz")."""
     X = np.asarray(X, np.float64)
     nrm = math.sqrt(float((X * X).sum()))
-    return X / max(nrm, NORM_FLOOR), nrm
+    return (X / nrm if nrm > 0.0 else X), nrm
 
 
 def newton_schulz(X, steps: int = NS_STEPS, a: float = NS_A, b: float = NS_B,
@@ -247,7 +248,7 @@ def optimizer_step(W_prev, G, M_prev, hp: HParams, *, conditioned: bool,
 
     X, nrm = frobenius_normalise(X0)
     nonfinite = not math.isfinite(nrm)
-    if nonfinite:
+    if nonfinite or nrm < NORM_FLOOR:
         Y = np.zeros_like(X0)
     else:
         X5 = newton_schulz(X, hp.ns_steps, hp.a, hp.b, hp.c)

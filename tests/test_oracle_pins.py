@@ -417,6 +417,18 @@ def test_nonfinite_gradient_only_decays():
     np.testing.assert_array_equal(r.O, 0.0)
 
 
+def test_negligible_norm_zero_update():
+    """A momentum whose Frobenius norm is below the 1e-15 floor gives a zero
+    update rather than an amplified one."""
+    rng = np.random.default_rng(21)
+    W = rng.standard_normal((6, 9))
+    r = orc.muon_step(W, 1e-20 * rng.standard_normal((6, 9)), np.zeros((6, 9)), orc.HParams())
+    assert not r.nonfinite
+    np.testing.assert_array_equal(r.O, 0.0)
+    r = orc.muon_step(W, 1e-12 * rng.standard_normal((6, 9)), np.zeros((6, 9)), orc.HParams())
+    assert np.abs(r.O).max() > 0.01
+
+
 def test_zero_gradient_zero_update():
     W = np.full((3, 5), 2.0)
     r = orc.muon_step(W, np.zeros((3, 5)), np.zeros((3, 5)), orc.HParams())
