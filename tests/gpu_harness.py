@@ -118,10 +118,10 @@ def step_and_compare(grp: Group, grads_host, hp, o_tol, *, ws=None, check_sv=Tru
                                  e_col_prev=ec0, momentum_dtype=sname(grp.mdt),
                                  weight_dtype=sname(grp.wdt))
         Mg, Wg, Og = to_host(grp.M[i]), to_host(grp.W[i]), to_host(grp.upd[i])
-        # momentum: at most one storage ulp (double rounding fp32 -> bf16)
+        # momentum: both sides round the fp64 value of mu M + G once -> equal
         dM = np.abs(Mg - res.M)
-        assert np.all(dM <= storage_ulp(res.M, grp.mdt) * 1.0001), (i, dM.max())
         rep.m_mismatch.append(int((dM > 0).sum()))
+        assert rep.m_mismatch[-1] == 0, (i, dM.max())
         # the update
         e = rel_fro(Og, res.O)
         rep.o_err.append(e)
