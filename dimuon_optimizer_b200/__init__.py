@@ -11,7 +11,7 @@ PyTorch supplies device memory and streams.
                      device="cuda")
     dm.check(dm.dm_muon_step(mats, hp, ws))
 
-The shared library must have been built (python -m dimuon_optimizer_b200.build,
+The shared library must have been built (python dimuon_optimizer_b200/build.py,
 or __graft_entry__.build()); importing fails loudly otherwise.
 """
 from __future__ import annotations
@@ -40,8 +40,10 @@ DM_SCALE_MOONSHOT = 1
 DM_THIN_MAX = 32
 DM_DBG_NO_THIN = 0x1
 
+DM_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
+
 EXPORTED = ("dm_default_hparams", "dm_workspace_size", "dm_muon_step", "dm_dimuon_step",
-            "dm_read_device_status", "dm_status_string", "dm_version")
+            "dm_read_device_status", "dm_step_noalloc", "dm_status_string", "dm_version")
 
 
 class dm_matrix_t(ctypes.Structure):
@@ -67,7 +69,7 @@ class DimuonError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m dimuon_optimizer_b200.build`")
+            f"{LIB_PATH} is missing: build it with `python dimuon_optimizer_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER
     lib.dm_default_hparams.argtypes = [P(dm_hparams_t)]
@@ -79,6 +81,9 @@ def _load():
         fn = getattr(lib, name)
         fn.argtypes = [P(dm_matrix_t), c_int, P(dm_hparams_t), c_void_p, c_size_t, c_void_p]
         fn.restype = c_int
+    lib.dm_step_noalloc.argtypes = [P(dm_matrix_t), c_int, P(dm_hparams_t), c_int, c_void_p,
+                                    c_void_p]
+    lib.dm_step_noalloc.restype = c_int
     lib.dm_read_device_status.argtypes = [c_void_p, c_void_p, P(c_int32)]
     lib.dm_read_device_status.restype = c_int
     lib.dm_status_string.argtypes = [c_int32]
@@ -184,6 +189,15 @@ def dm_dimuon_step(mats, hp, workspace, stream=None):
     arr, n = _array(mats)
     ptr, nbytes = _ws(workspace)
     return _lib.dm_dimuon_step(arr, n, ctypes.byref(hp), ptr, nbytes, _stream_handle(stream))
+
+
+def dm_step_noalloc(mats, hp, conditioned, device_status_out=None, stream=None):
+    """The step with the library's own fixed scratch array instead of a
+    workspace (for callers that cannot allocate device memory); see
+    include/dimuon.h.  device_status_out: optional int32 CUDA tensor."""
+    arr, n = _array(mats)
+    return _lib.dm_step_noalloc(arr, n, ctypes.byref(hp), int(conditioned),
+                                _ptr(device_status_out), _stream_handle(stream))
 
 
 def dm_read_device_status(workspace, stream=None):

@@ -1,6 +1,6 @@
 """Builds libdimuon.so in-tree with nvcc for sm_100a.
 
-    python -m dimuon_optimizer_b200.build [--debug]
+    python dimuon_optimizer_b200/build.py [--debug]
 
 The library is compiled for B200 only (-gencode arch=compute_100a,code=sm_100a)
 and links the CUDA runtime statically; the driver's tensor-map encoder is
@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdimuon.so")
-SOURCES = ["api.cu", "k_elementwise.cu", "k_ns_simt.cu", "k_ns_tc.cu", "k_thin.cu"]
+SOURCES = ["api.cu", "api_noalloc.cu", "k_elementwise.cu", "k_ns_simt.cu", "k_ns_tc.cu", "k_thin.cu"]
 HEADERS = ["dm_common.cuh", "dm_internal.h", "dm_sm100.cuh", "dm_tiles.cuh"]
 
 

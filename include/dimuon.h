@@ -156,6 +156,36 @@ dm_status_t dm_dimuon_step(const dm_matrix_t* mats, int n,
 dm_status_t dm_read_device_status(const void* workspace, void* stream,
                                   int32_t* out);
 
+/* Size of the scratch array behind dm_step_noalloc: 32 MiB per GPU that
+ * loads the library, held until the process exits. */
+#define DM_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
+
+/* The step (conditioned = 0: as dm_muon_step, 1: as dm_dimuon_step) without
+ * a caller-provided workspace.  The pages have no counterpart: this exists
+ * for callers that cannot allocate device memory, such as code running
+ * inside a framework whose caching allocator has reserved the whole device,
+ * or a latency-critical path where cudaMalloc / cudaFree would synchronise
+ * the device.  Its scratch memory is one fixed array of
+ * DM_NOALLOC_MAX_BYTES in the library's device code; the caller still passes
+ * every input and output.
+ *   - Groups whose dm_workspace_size exceeds DM_NOALLOC_MAX_BYTES are
+ *     rejected with DM_ERR_WORKSPACE before any device work.  Thin factors
+ *     (short side <= DM_THIN_MAX) need no scratch, so any number of them fits.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress); make that first call before
+ *     any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; the step
+ *     zeroes its status word itself and needs nothing else zeroed.  Calls whose
+ *     device work overlaps (different streams or threads without ordering)
+ *     race on the array: order them on the device.
+ *   - device_status_out (nullable, device int32) receives the step's device
+ *     status word (as dm_read_device_status would report it), asynchronously.
+ *   - Calls no allocating routine (no cudaMalloc, cudaFree or library
+ *     allocator). */
+dm_status_t dm_step_noalloc(const dm_matrix_t* mats, int n,
+                            const dm_hparams_t* hp, int conditioned,
+                            int32_t* device_status_out, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* dm_status_string(int32_t status);
 
