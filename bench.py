@@ -2,7 +2,8 @@
 """Throughput of the B200 Muon / Dimuon step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large_batch|gpt2_small|square1024|lora_r2|lora_r8|lora_r32]
+                    [--workload large_batch|large_batch_quarter|gpt2_small|square1024|
+                               lora_r2|lora_r8|lora_r32]
 
 One step = one optimizer step (momentum, normalisation, five Newton-Schulz
 iterations, scale, decay, apply) over every matrix of the workload.  The
@@ -37,6 +38,10 @@ def workload_spec(name):
         return dict(shapes=workloads.large_batch_shapes(), cond=False, mdt="bf16", lr=0.02,
                     wd=0.0, moonshot=False, seed=3,
                     desc="8x4096^2 + 4x4096x14336 + 4x14336x4096 bf16, Muon, 5 NS5 iterations")
+    if name == "large_batch_quarter":  # same shapes, a quarter of the matrices
+        return dict(shapes=[(4096, 4096)] * 2 + [(4096, 14336), (14336, 4096)], cond=False,
+                    mdt="bf16", lr=0.02, wd=0.0, moonshot=False, seed=3,
+                    desc="2x4096^2 + 4096x14336 + 14336x4096 bf16, Muon, 5 NS5 iterations")
     if name == "gpt2_small":
         return dict(shapes=workloads.gpt2_small_shapes(), cond=False, mdt="bf16", lr=0.02,
                     wd=0.1, moonshot=True, seed=2,

@@ -330,12 +330,28 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
   if (n == 0) return DM_OK;
 
   // ---------------------------- thin factors -------------------------------
+  // Launches group factors by padded short side (2..32) and cluster size.
   {
-    std::vector<int> groups[3];  // pad 8 / 16 / 32
-    for (const MatPlan& p : L.mats)
-      if (p.thin) groups[p.m <= 8 ? 0 : (p.m <= 16 ? 1 : 2)].push_back(p.idx);
-    const int pads[3] = {8, 16, 32};
-    for (int gi = 0; gi < 3; ++gi) {
+    std::vector<std::pair<int, int>> keys;
+    std::vector<std::vector<int>> groups;
+    for (const MatPlan& p : L.mats) {
+      if (!p.thin) continue;
+      int pad = 2;
+      while (pad < p.m) pad *= 2;
+      const int64_t elems = (int64_t)p.m * p.n;
+      int cl = elems >= 65536 ? 8 : elems >= 32768 ? 4 : elems >= 16384 ? 2 : 1;
+      const int64_t chunks = ceil_div(p.n, 4096 / pad);  // 4096-element chunks
+      while (cl > 1 && chunks < cl) cl /= 2;
+      const std::pair<int, int> key(pad, cl);
+      size_t g = 0;
+      while (g < keys.size() && keys[g] != key) ++g;
+      if (g == keys.size()) {
+        keys.push_back(key);
+        groups.emplace_back();
+      }
+      groups[g].push_back(p.idx);
+    }
+    for (size_t gi = 0; gi < groups.size(); ++gi) {
       const std::vector<int>& idx = groups[gi];
       const int nchunks = (int)ceil_div((int64_t)idx.size(), THIN_MAX);
       for (int ch = 0; ch < nchunks; ++ch) {
@@ -344,7 +360,8 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
         static thread_local ThinParams tp;
         std::memset(&tp, 0, sizeof(tp));
         tp.count = (int)(e - b);
-        tp.pad = pads[gi];
+        tp.pad = keys[gi].first;
+        tp.cluster = keys[gi].second;
         tp.conditioned = cond;
         tp.ns_steps = hp->ns_steps;
         tp.mu = hp->mu;
@@ -370,6 +387,8 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
           t.mdt = um.momentum_dtype;
           t.wdt = um.weight_dtype;
           t.kappa = kappa_of(hp, um.rows, um.cols);
+          auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+          t.vec = al16(um.grad) && al16(um.momentum) && al16(um.weight) && al16(um.update_out);
         }
         DM_CUDA(launch_thin(tp, s));
       }

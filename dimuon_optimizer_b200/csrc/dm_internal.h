@@ -185,12 +185,14 @@ struct ThinMat {
   float* e_col;
   int64_t rows, cols;
   int gdt, mdt, wdt;
+  int vec;                // G, M, W, upd all 16-byte aligned
   float kappa;
 };
 constexpr int THIN_MAX = 256;
 struct ThinParams {
   int count;
-  int pad;                // padded short side of every factor in the launch
+  int pad;                // padded short side of every factor in the launch (2..32)
+  int cluster;            // CTAs per factor (thread-block cluster size, 1..8)
   int conditioned;
   int ns_steps;
   float mu, lr, decay, a, b, c, eps;
