@@ -106,8 +106,9 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
       p.ldm = (int64_t)round_up((size_t)p.m, 8);
       p.k1_rt = (int)ceil_div(p.rows, K1_ROWS);
       p.k1_ct = (int)ceil_div(p.cols, K1_COLS);
-      if (L.tc)
-        p.n_part = (int)(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN)) * 4;
+      if (L.tc)  // enough (sum x^2, sum y^2) slots for either tensor-core kernel
+        p.n_part = (int)std::max(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN) * 4,
+                                 ceil_div(p.rows, TC2_BM) * ceil_div(p.cols, TC2_BN) * 8);
       else
         p.n_part = (int)(ceil_div(p.rows, 128) * ceil_div(p.cols, 128));
       p.off_scal = take(SC_COUNT * sizeof(float), 256);
@@ -491,38 +492,58 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     }
   }
   // Newton-Schulz products
+  std::vector<int> final_npart(n, 0);  // partial slots the last product wrote
   if (L.tc) {
     std::vector<MatMaps> maps;
     if (!get_maps(L, ws, dev, maps)) return DM_ERR_CUDA;
     const int nsm = sm_count(dev);
     static thread_local TcParams pt;
+    auto build = [&](size_t b, int ph, int k, int bm, int bn) {
+      std::memset(&pt, 0, sizeof(pt));
+      pt.status = status;
+      pt.lr = hp->lr;
+      pt.decay = decay;
+      pt.debug = hp->debug_flags;
+      int tiles = 0;
+      for (size_t q = b; q < std::min(big.size(), b + TC_MAX); ++q) {
+        const MatPlan& p = *big[q];
+        TcMat& tm = pt.mats[pt.count];
+        const OperandSrc src = fill_gemm(tm.g, p, mats[p.idx], hp, ws, ph, k, cond != 0,
+                                         kappa_of(hp, p.rows, p.cols), bm, bn);
+        const MatMaps& mm = maps[p.idx];
+        auto pick = [&](int buf) -> const CUtensorMap& {
+          return buf < 2 ? mm.X[buf] : (buf == 2 ? mm.A : mm.B);
+        };
+        tm.ta = pick(src.a_buf);
+        tm.tb = pick(src.b_buf);
+        pt.starts[pt.count++] = tiles;
+        tiles += gemm_tile_count(tm.g, bm, bn);
+      }
+      pt.starts[pt.count] = tiles;
+      pt.total_tiles = tiles;
+      return tiles;
+    };
     for (int k = 1; k <= hp->ns_steps; ++k)
       for (int ph = 0; ph < 3; ++ph)
         for (size_t b = 0; b < big.size(); b += TC_MAX) {
-          std::memset(&pt, 0, sizeof(pt));
-          pt.status = status;
-          pt.lr = hp->lr;
-          pt.decay = decay;
-          pt.debug = hp->debug_flags;
-          int tiles = 0;
-          for (size_t q = b; q < std::min(big.size(), b + TC_MAX); ++q) {
-            const MatPlan& p = *big[q];
-            TcMat& tm = pt.mats[pt.count];
-            const OperandSrc src =
-                fill_gemm(tm.g, p, mats[p.idx], hp, ws, ph, k, cond != 0,
-                          kappa_of(hp, p.rows, p.cols), TC_BM, TC_BN);
-            const MatMaps& mm = maps[p.idx];
-            auto pick = [&](int buf) -> const CUtensorMap& {
-              return buf < 2 ? mm.X[buf] : (buf == 2 ? mm.A : mm.B);
-            };
-            tm.ta = pick(src.a_buf);
-            tm.tb = pick(src.b_buf);
-            pt.starts[pt.count++] = tiles;
-            tiles += gemm_tile_count(tm.g, TC_BM, TC_BN);
+          // CTA pairs when there are at least two 256 x 256 tiles per pair
+          const int pair_tiles = build(b, ph, k, TC2_BM, TC2_BN);
+          bool pair = pair_tiles >= nsm;
+          if (hp->debug_flags & DM_DBG_TC_PAIR) pair = true;
+          if (hp->debug_flags & DM_DBG_TC_SINGLE) pair = false;
+          if (pair) {
+            DM_CUDA(launch_tc_pair(pt, std::min(pair_tiles, nsm / 2), s));
+          } else {
+            const int tiles = build(b, ph, k, TC_BM, TC_BN);
+            DM_CUDA(launch_tc(pt, std::min(tiles, nsm), s));
           }
-          pt.starts[pt.count] = tiles;
-          pt.total_tiles = tiles;
-          DM_CUDA(launch_tc(pt, std::min(tiles, nsm), s));
+          if (k == hp->ns_steps && ph == PH_GEMM)
+            for (size_t q = b; q < std::min(big.size(), b + TC_MAX); ++q) {
+              const MatPlan& p = *big[q];
+              final_npart[p.idx] =
+                  pair ? (int)(ceil_div(p.rows, TC2_BM) * ceil_div(p.cols, TC2_BN) * 8)
+                       : (int)(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN) * 4);
+            }
         }
   } else {
     static thread_local SimtParams ps;
@@ -581,7 +602,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
         k.wdt = um.weight_dtype;
         k.vec = (p.cols % 8 == 0) && !(reinterpret_cast<uintptr_t>(um.weight) & 15u) &&
                 !(reinterpret_cast<uintptr_t>(um.update_out) & 15u);
-        k.n_part = p.n_part;
+        k.n_part = L.tc ? final_npart[p.idx] : p.n_part;
         k.n_rt = p.k1_rt;
         k.n_ct = p.k1_ct;
         k.kappa = kappa_of(hp, p.rows, p.cols);

@@ -209,6 +209,9 @@ cudaError_t launch_k3(const K3Params& p, int total_tiles, cudaStream_t s);
 cudaError_t launch_simt(const SimtParams& p, int total_tiles, cudaStream_t s);
 cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s);
 int tc_smem_bytes();
+constexpr int TC2_BM = 256, TC2_BN = 256;  // CTA-pair output tile
+cudaError_t launch_tc_pair(const TcParams& p, int pairs, cudaStream_t s);
+int tc_pair_smem_bytes();
 cudaError_t launch_thin(const ThinParams& p, cudaStream_t s);
 
 }  // namespace dm

@@ -1,0 +1,285 @@
+// Tensor-core Newton-Schulz products on CTA pairs (tcgen05 cta_group::2):
+// the same three products and fused epilogues as tc_ns_product
+//   A = X X^T, B = b A + c A A (symmetric), X' = a X + B X
+// (sitech.ge Muon post, "Instead of SVD - Newton-Schulz"; coefficients from
+// "Muon Optimizer 정리", "Why orthogonalise"), with 256 x 256 output tiles
+// computed by a pair of CTAs (a cluster of 2 on two SMs):
+//   - each CTA loads its own 128 rows of the A operand and its own 128
+//     columns of the B operand (TMA, 64 x 64 boxes, 128-byte swizzle, no
+//     multicast), 32 KB per stage, 6 stages; both CTAs' loads complete on
+//     the leader's "full" barrier;
+//   - one thread of the leader issues tcgen05.mma.cta_group::2 with M = 256,
+//     N = 256: the accumulator's rows 0..127 live in the leader's tensor
+//     memory, rows 128..255 in the peer's; per k-block the MMA reads half of
+//     B from each CTA, so each SM streams 2/3 of the bytes a 128 x 256 tile
+//     needs per flop;
+//   - the MMA's completion frees the stage in both CTAs and hands each CTA's
+//     epilogue warps its half of the accumulator;
+//   - the peer's epilogue warps report a drained accumulator to the leader.
+// Every wait is bounded; the kernel ends with a cluster barrier so neither
+// CTA leaves while the other still addresses its shared memory.
+#include "dm_common.cuh"
+#include "dm_sm100.cuh"
+#include "dm_tc_epilogue.cuh"
+#include "dm_tiles.cuh"
+
+namespace dm {
+namespace {
+
+using namespace sm100;
+using namespace tcepi;
+
+constexpr int PAIR_BM = 256;                     // output tile rows (both CTAs)
+constexpr int PAIR_BN = 256;                     // output tile columns
+constexpr int HALF = 128;                        // rows (A) / columns (B) per CTA
+constexpr int STAGES = 6;
+constexpr int BOX_BYTES = 64 * 64 * 2;
+constexpr int A_BYTES = HALF * TC_BK * 2;        // 16 KB
+constexpr int B_BYTES = HALF * TC_BK * 2;        // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB per CTA
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;              // two 128-lane x 256-column accumulators
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
+constexpr uint16_t PAIR_MASK = 0x3;
+
+struct Tile {
+  int g, lt, tm, tn;
+};
+
+__device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
+  Tile tl;
+  tl.g = find_group(p.starts, p.count, t);
+  tl.lt = t - p.starts[tl.g];
+  gemm_tile_coord(p.mats[tl.g].g, tl.lt, PAIR_BM, PAIR_BN, tl.tm, tl.tn);
+  return tl;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0 = leader, 1 = peer
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);   // leader: its own arrive.expect_tx; peer: unused
+      mbar_init(&empty[s], 1);  // one multicast commit per consumed stage
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // leader: 4 local + 4 peer epilogue warps
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {  // the same warp of both CTAs allocates collectively
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers initialised in both CTAs, TMEM address published
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ----------------------------- TMA producer -----------------------------
+    if (lane == 0) {
+      for (int g = 0; g < p.count; ++g) {
+        tma_prefetch_map(&p.mats[g].ta);
+        tma_prefetch_map(&p.mats[g].tb);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      for (int t = pair; t < p.total_tiles && !*abort; t += npairs) {
+        const Tile tl = decode_tile(p, t);
+        const TcMat& mt = p.mats[tl.g];
+        const int a_mn = mt.g.flags & GF_A_MN, b_mn = mt.g.flags & GF_B_MN;
+        const int m0 = tl.tm * PAIR_BM + (int)rank * HALF;
+        const int n0 = tl.tn * PAIR_BN + (int)rank * HALF;
+        const int nkb = (mt.g.K + TC_BK - 1) / TC_BK;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort, p.status, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          if (rank == 0) {
+            mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);  // both CTAs' bytes
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+          const int k0 = kb * TC_BK;
+#pragma unroll
+          for (int q = 0; q < HALF / 64; ++q) {
+            if (a_mn)
+              tma_load_2d_pair(sa + q * BOX_BYTES, &mt.ta, bar, m0 + 64 * q, k0);
+            else
+              tma_load_2d_pair(sa + q * BOX_BYTES, &mt.ta, bar, k0, m0 + 64 * q);
+            if (b_mn)
+              tma_load_2d_pair(sb + q * BOX_BYTES, &mt.tb, bar, n0 + 64 * q, k0);
+            else
+              tma_load_2d_pair(sb + q * BOX_BYTES, &mt.tb, bar, k0, n0 + 64 * q);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort && rank == 0) {
+        // Both CTAs' copies in flight complete on the leader's barriers.
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s))
+            mbar_wait_bounded(&full[s], (armed_par >> s) & 1u, abort, nullptr, DRAIN_LIMIT_NS);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------- MMA issuer (leader only) -------------------------
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int t = pair; t < p.total_tiles && !*abort; t += npairs, ++local) {
+        const Tile tl = decode_tile(p, t);
+        const GemmMat& g = p.mats[tl.g].g;
+        const int a_mn = (g.flags & GF_A_MN) ? 1 : 0, b_mn = (g.flags & GF_B_MN) ? 1 : 0;
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort, p.status, WAIT_LIMIT_NS)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PAIR_BN);
+        const uint32_t idesc = idesc_bf16(PAIR_BM, PAIR_BN, a_mn, b_mn);
+        const int nkb = (g.K + TC_BK - 1) / TC_BK;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort, p.status, WAIT_LIMIT_NS)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+            const uint64_t ad = a_mn ? smem_desc(sa + kk * 2048, BOX_BYTES, 1024)
+                                     : smem_desc(sa + kk * 32, 16, 1024);
+            const uint64_t bd = b_mn ? smem_desc(sb + kk * 2048, BOX_BYTES, 1024)
+                                     : smem_desc(sb + kk * 32, 16, 1024);
+            mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[stage], PAIR_MASK);  // frees the stage in both CTAs
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc], PAIR_MASK);  // accumulator ready in both CTAs
+      }
+      mma_commit_pair(drain, 0x1);
+      mbar_wait_bounded(drain, 0, abort, nullptr, DRAIN_LIMIT_NS);
+    }
+  } else {
+    // ------------------------------- epilogue -------------------------------
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int row_in_half = quarter * 32 + lane;
+    int local = 0;
+    for (int t = pair; t < p.total_tiles; t += npairs, ++local) {
+      const Tile tl = decode_tile(p, t);
+      const GemmMat& g = p.mats[tl.g].g;
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort, p.status, WAIT_LIMIT_NS)) break;
+      tc_fence_after();
+      const int r = tl.tm * PAIR_BM + (int)rank * HALF + row_in_half;
+      const bool row_ok = r < g.M;
+      const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
+      const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
+      float sx = 0.f, sy = 0.f;
+      const int nch = min(PAIR_BN, g.N - tl.tn * PAIR_BN + 31) / 32;
+#pragma unroll 1
+      for (int ch = 0; ch < PAIR_BN / 32; ++ch) {
+        float v[32];
+        tmem_ld32(tmem_base + (uint32_t)(acc * PAIR_BN + ch * 32) + ((uint32_t)(quarter * 32) << 16),
+                  v);
+        if (row_ok && ch < nch)
+          epilogue32(g, p.lr, p.decay, r, tl.tn * PAIR_BN + ch * 32, v, S, valid, sx, sy);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(&tempty[acc]);
+        else
+          mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
+      }
+      if (g.epi == EPI_FINAL_DIMUON) {
+        sx = warp_sum(sx);
+        sy = warp_sum(sy);
+        if (lane == 0) {
+          const int slot = (tl.tm * g.tiles_n + tl.tn) * 8 + (int)rank * 4 + quarter;
+          g.part[2 * slot] = sx;
+          g.part[2 * slot + 1] = sy;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no CTA of the pair is still addressed by the other
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+int tc_pair_smem_bytes() { return SMEM_BYTES; }
+
+cudaError_t launch_tc_pair(const TcParams& p, int pairs, cudaStream_t s) {
+  if (p.total_tiles <= 0 || pairs <= 0) return cudaSuccess;
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(tc_ns_product_pair,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_ns_product_pair, p);
+}
+
+}  // namespace dm

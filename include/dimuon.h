@@ -123,6 +123,10 @@ typedef struct {
 /* debug_flags bits (test hooks; none of them changes the arithmetic) */
 #define DM_DBG_NO_THIN 0x1u       /* send short-side <= DM_THIN_MAX matrices
                                      down the Newton-Schulz path as well   */
+#define DM_DBG_TC_SINGLE 0x2u     /* tensor-core products on single CTAs
+                                     (128 x 256 tiles) only                */
+#define DM_DBG_TC_PAIR 0x4u       /* tensor-core products on CTA pairs
+                                     (256 x 256 tiles) only                */
 
 /* Fills *hp with the defaults: mu 0.95, lr 0.02, wd 0, ns_steps 5,
  * (a,b,c) = (3.4445, -4.7750, 2.0315), cond_eps 1e-4, DM_SCALE_NONE,

@@ -64,10 +64,14 @@ def test_fp32_mode_ns_path(cond, dts):
 TC_SHAPES = [(384, 640), (700, 260), (257, 513), (40, 100), (128, 256), (520, 136)]
 
 
+@pytest.mark.parametrize("kernel", [0, dm.DM_DBG_TC_SINGLE, dm.DM_DBG_TC_PAIR])
 @pytest.mark.parametrize("cond", [False, True])
-def test_tc_mode_ns_path(cond):
+def test_tc_mode_ns_path(cond, kernel):
+    """Tensor-core products: the planner's choice, single-CTA 128 x 256 tiles
+    and CTA-pair 256 x 256 tiles."""
     grp = Group(TC_SHAPES, BF, BF, BF, cond=cond, seed=12)
-    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.1, scale_mode=dm.DM_SCALE_MOONSHOT)
+    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.1, scale_mode=dm.DM_SCALE_MOONSHOT,
+                 debug_flags=kernel)
     ws = None
     for t in range(3):
         rep, ws = step_and_compare(grp, gaussian(TC_SHAPES, 200 + t, scale_cols=True), hp,
@@ -87,9 +91,10 @@ def test_tc_mode_fp32_storage():
 @pytest.mark.parametrize("ns_steps", [1, 2, 6])
 def test_ns_step_counts(ns_steps):
     shapes = [(200, 330), (330, 200)]
-    for prec, tol in ((dm.DM_PREC_FP32, TOL_FP32), (dm.DM_PREC_BF16_TC, TOL_BF16)):
+    for prec, tol, dbg in ((dm.DM_PREC_FP32, TOL_FP32, 0), (dm.DM_PREC_BF16_TC, TOL_BF16, 0),
+                           (dm.DM_PREC_BF16_TC, TOL_BF16, dm.DM_DBG_TC_PAIR)):
         grp = Group(shapes, BF, BF, F32, cond=True, seed=14)
-        hp = hparams(prec, ns_steps=ns_steps)
+        hp = hparams(prec, ns_steps=ns_steps, debug_flags=dbg)
         ws = None
         for t in range(2):
             _, ws = step_and_compare(grp, gaussian(shapes, 400 + t), hp, tol, ws=ws)
