@@ -107,8 +107,8 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
       p.k1_rt = (int)ceil_div(p.rows, K1_ROWS);
       p.k1_ct = (int)ceil_div(p.cols, K1_COLS);
       if (L.tc)  // enough (sum x^2, sum y^2) slots for either tensor-core kernel
-        p.n_part = (int)std::max(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN) * 4,
-                                 ceil_div(p.rows, TC2_BM) * ceil_div(p.cols, TC2_BN) * 8);
+        p.n_part = (int)std::max(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN) * 8,
+                                 ceil_div(p.rows, TC2_BM) * ceil_div(p.cols, TC2_BN) * 16);
       else
         p.n_part = (int)(ceil_div(p.rows, 128) * ceil_div(p.cols, 128));
       p.off_scal = take(SC_COUNT * sizeof(float), 256);
@@ -541,8 +541,8 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
             for (size_t q = b; q < std::min(big.size(), b + TC_MAX); ++q) {
               const MatPlan& p = *big[q];
               final_npart[p.idx] =
-                  pair ? (int)(ceil_div(p.rows, TC2_BM) * ceil_div(p.cols, TC2_BN) * 8)
-                       : (int)(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN) * 4);
+                  pair ? (int)(ceil_div(p.rows, TC2_BM) * ceil_div(p.cols, TC2_BN) * 16)
+                       : (int)(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN) * 8);
             }
         }
   } else {

@@ -4,9 +4,14 @@
 #pragma once
 
 #include "dm_common.cuh"
+#include "dm_sm100.cuh"
 
 namespace dm {
 namespace tcepi {
+
+__device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, float v[32]) {
+  sm100::tmem_ld32(taddr, v);
+}
 
 __device__ __forceinline__ void ld_bf16x8(const void* p, float v[8]) {
   ld8(p, 0, DT_BF16, v);
@@ -64,10 +69,13 @@ __device__ __forceinline__ void store_sym32(const GemmMat& g, int r, int c0, con
   }
 }
 
-// Fused epilogue for 32 accumulator columns of one output row.
+__device__ __forceinline__ bool needs_aux(int epi) { return epi != EPI_SYRK; }
+
+// Fused epilogue for 32 accumulator columns of one output row; `ax` holds
+// the same 32 columns of the aux matrix (unused for EPI_SYRK).
 __device__ __forceinline__ void epilogue32(const GemmMat& g, float lr, float decay, int r, int c0,
-                                           float v[32], float S, float valid, float& sx,
-                                           float& sy) {
+                                           float v[32], const float ax[32], float S, float valid,
+                                           float& sx, float& sy) {
   switch (g.epi) {
     case EPI_SYRK: {
 #pragma unroll
@@ -76,24 +84,18 @@ __device__ __forceinline__ void epilogue32(const GemmMat& g, float lr, float dec
       break;
     }
     case EPI_POLY: {
-      float ax[32];
-      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
 #pragma unroll
       for (int q = 0; q < 32; ++q) v[q] = fmaf(g.coef_acc, v[q], g.coef_aux * ax[q]);
       store_sym32(g, r, c0, v);
       break;
     }
     case EPI_GEMM: {
-      float ax[32];
-      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
 #pragma unroll
       for (int q = 0; q < 32; ++q) v[q] = fmaf(g.coef_aux, ax[q], v[q]) * S;
       store_row32(reinterpret_cast<__nv_bfloat16*>(g.out), g.ldo, r, c0, g.N, v);
       break;
     }
     case EPI_FINAL_MUON: {
-      float ax[32];
-      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
       const float ks = valid != 0.f ? g.kappa * S : 0.f;
 #pragma unroll
       for (int q = 0; q < 32; ++q) v[q] = (valid != 0.f) ? fmaf(g.coef_aux, ax[q], v[q]) * ks : 0.f;
@@ -129,8 +131,6 @@ __device__ __forceinline__ void epilogue32(const GemmMat& g, float lr, float dec
       break;
     }
     case EPI_FINAL_DIMUON: {
-      float ax[32];
-      load_row32(reinterpret_cast<const __nv_bfloat16*>(g.aux), g.ldaux, r, c0, g.N, ax);
       const float rr = g.R[r];
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
@@ -144,6 +144,31 @@ __device__ __forceinline__ void epilogue32(const GemmMat& g, float lr, float dec
       store_row32(reinterpret_cast<__nv_bfloat16*>(g.out), g.ldo, r, c0, g.N, v);
       break;
     }
+  }
+}
+
+// Epilogue of chunks [ch_begin, ch_end) (32 columns each) of one accumulator
+// row: tcgen05.ld of each chunk, with the next chunk's aux row in flight while
+// the current one is processed.  Must be executed by all 32 lanes of the warp
+// (tcgen05.ld is warp-collective); rows outside the matrix only skip stores.
+__device__ __forceinline__ void epilogue_row(const GemmMat& g, float lr, float decay, int r,
+                                             bool row_ok, int col0, uint32_t taddr, int ch_begin,
+                                             int ch_end, int nch, float& sx, float& sy) {
+  const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
+  const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
+  const bool aux = needs_aux(g.epi);
+  const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(g.aux);
+  float axn[32];
+  if (aux && row_ok && ch_begin < nch) load_row32(ab, g.ldaux, r, col0 + ch_begin * 32, g.N, axn);
+#pragma unroll 1
+  for (int ch = ch_begin; ch < ch_end; ++ch) {
+    float v[32], ax[32];
+    tmem_ld32_at(taddr + (uint32_t)(ch * 32), v);
+#pragma unroll
+    for (int q = 0; q < 32; ++q) ax[q] = axn[q];
+    if (aux && row_ok && ch + 1 < ch_end && ch + 1 < nch)
+      load_row32(ab, g.ldaux, r, col0 + (ch + 1) * 32, g.N, axn);
+    if (row_ok && ch < nch) epilogue32(g, lr, decay, r, col0 + ch * 32, v, ax, S, valid, sx, sy);
   }
 }
 

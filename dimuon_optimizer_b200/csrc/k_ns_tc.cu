@@ -32,7 +32,7 @@ constexpr int BOX_BYTES = 64 * 64 * 2;
 constexpr int A_BYTES = TC_BM * TC_BK * 2;      // 16 KB
 constexpr int B_BYTES = TC_BN * TC_BK * 2;      // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t TMEM_COLS = 512;             // two 128 x 256 fp32 accumulators
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 8);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -192,8 +192,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
     }
   } else {
     // ------------------------------- epilogue -------------------------------
+    // Warps 2..9: two warps per TMEM lane quarter, each taking half of the
+    // accumulator's columns.
+    const int ew = warp - 2;
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-    const int row_in_tile = quarter * 32 + lane;
+    const int half = ew >> 2;
+    const int row_in_half = quarter * 32 + lane;
     int local = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++local) {
       const Tile tl = decode_tile(p, t);
@@ -202,27 +206,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort, p.status, WAIT_LIMIT_NS)) break;
       tc_fence_after();
-      const int r = tl.tm * TC_BM + row_in_tile;
-      const bool row_ok = r < g.M;
-      const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
-      const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
-      float sx = 0.f, sy = 0.f;
+      const int r = tl.tm * TC_BM + row_in_half;
       const int nch = min(TC_BN, g.N - tl.tn * TC_BN + 31) / 32;  // chunks holding columns < N
-#pragma unroll 1
-      for (int ch = 0; ch < TC_BN / 32; ++ch) {
-        float v[32];
-        tmem_ld32(tmem_base + (uint32_t)(acc * TC_BN + ch * 32) + ((uint32_t)(quarter * 32) << 16),
-                  v);
-        if (row_ok && ch < nch) epilogue32(g, p.lr, p.decay, r, tl.tn * TC_BN + ch * 32, v, S, valid, sx, sy);
-      }
+      constexpr int CH_PER = TC_BN / 32 / 2;
+      float sx = 0.f, sy = 0.f;
+      epilogue_row(g, p.lr, p.decay, r, r < g.M, tl.tn * TC_BN,
+                   tmem_base + (uint32_t)(acc * TC_BN) + ((uint32_t)(quarter * 32) << 16),
+                   half * CH_PER, half * CH_PER + CH_PER, nch, sx, sy);
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tempty[acc]);
+      }
       if (g.epi == EPI_FINAL_DIMUON) {
-        // One (sum x^2, sum y^2) pair per epilogue warp; no barrier needed.
+        // one (sum x^2, sum y^2) pair per epilogue warp; no barrier needed
         sx = warp_sum(sx);
         sy = warp_sum(sy);
         if (lane == 0) {
-          const int slot = (tl.tm * g.tiles_n + tl.tn) * 4 + quarter;
+          const int slot = (tl.tm * g.tiles_n + tl.tn) * 8 + ew;
           g.part[2 * slot] = sx;
           g.part[2 * slot + 1] = sy;
         }

@@ -37,7 +37,7 @@ constexpr int BOX_BYTES = 64 * 64 * 2;
 constexpr int A_BYTES = HALF * TC_BK * 2;        // 16 KB
 constexpr int B_BYTES = HALF * TC_BK * 2;        // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB per CTA
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t TMEM_COLS = 512;              // two 128-lane x 256-column accumulators
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);  // leader: 4 local + 4 peer epilogue warps
+      mbar_init(&tempty[a], 16);  // leader: 8 local + 8 peer epilogue warps
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -200,7 +200,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
     }
   } else {
     // ------------------------------- epilogue -------------------------------
+    // Warps 2..9: two warps per TMEM lane quarter, each taking half of the
+    // accumulator's columns.
+    const int ew = warp - 2;
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int half = ew >> 2;
     const int row_in_half = quarter * 32 + lane;
     int local = 0;
     for (int t = pair; t < p.total_tiles; t += npairs, ++local) {
@@ -211,19 +215,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort, p.status, WAIT_LIMIT_NS)) break;
       tc_fence_after();
       const int r = tl.tm * PAIR_BM + (int)rank * HALF + row_in_half;
-      const bool row_ok = r < g.M;
-      const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
-      const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
+      const int nch = min(PAIR_BN, g.N - tl.tn * PAIR_BN + 31) / 32;  // chunks holding columns < N
+      constexpr int CH_PER = PAIR_BN / 32 / 2;
       float sx = 0.f, sy = 0.f;
-      const int nch = min(PAIR_BN, g.N - tl.tn * PAIR_BN + 31) / 32;
-#pragma unroll 1
-      for (int ch = 0; ch < PAIR_BN / 32; ++ch) {
-        float v[32];
-        tmem_ld32(tmem_base + (uint32_t)(acc * PAIR_BN + ch * 32) + ((uint32_t)(quarter * 32) << 16),
-                  v);
-        if (row_ok && ch < nch)
-          epilogue32(g, p.lr, p.decay, r, tl.tn * PAIR_BN + ch * 32, v, S, valid, sx, sy);
-      }
+      epilogue_row(g, p.lr, p.decay, r, r < g.M, tl.tn * PAIR_BN,
+                   tmem_base + (uint32_t)(acc * PAIR_BN) + ((uint32_t)(quarter * 32) << 16),
+                   half * CH_PER, half * CH_PER + CH_PER, nch, sx, sy);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -233,10 +230,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
           mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
       }
       if (g.epi == EPI_FINAL_DIMUON) {
+        // one (sum x^2, sum y^2) pair per epilogue warp; no barrier needed
         sx = warp_sum(sx);
         sy = warp_sum(sy);
         if (lane == 0) {
-          const int slot = (tl.tm * g.tiles_n + tl.tn) * 8 + (int)rank * 4 + quarter;
+          const int slot = (tl.tm * g.tiles_n + tl.tn) * 16 + (int)rank * 8 + ew;
           g.part[2 * slot] = sx;
           g.part[2 * slot + 1] = sy;
         }
