@@ -75,6 +75,23 @@ def step_bytes(spec):
     return sum(r * c for r, c in spec["shapes"]) * (2 + 2 * mb + 4)
 
 
+# DRAM traffic of the tensor-core product per launch (ncu dram__bytes_read.sum +
+# dram__bytes_write.sum), valid only for the kernel build it was taken from:
+# profiles/tc_ns_product_pair_large_batch_quarter.md (quarter batch x 4).
+TRAFFIC_CAPTURED = {"large_batch": 2855e6}
+TRAFFIC_BUILD = "d1e95b408d4906e0"
+TRAFFIC_SOURCES = ["k_ns_tc2.cu", "dm_tc_epilogue.cuh", "dm_sm100.cuh"]
+
+
+def kernel_build_hash():
+    import hashlib
+    parts = []
+    for f in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "dimuon_optimizer_b200", "csrc", f), "rb") as fh:
+            parts.append(hashlib.sha256(fh.read()).hexdigest())
+    return hashlib.sha256("".join(parts).encode()).hexdigest()[:16]
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -298,9 +315,14 @@ def main():
     if per_iter_flops > 0 and t5 > t1:
         achieved = 4 * per_iter_flops / (t5 - t1) / 1e12
         peak = peaks.get("bf16_tflops_sustained", 1400.0)
+        traffic = None
+        if args.workload in TRAFFIC_CAPTURED and kernel_build_hash() == TRAFFIC_BUILD:
+            traffic = TRAFFIC_CAPTURED[args.workload]
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
-                    "kernel": "tc_ns_product", "avg_launch_ms": (t5 - t1) / tc_launches * 1e3,
+                    "frac": achieved / peak, "traffic": traffic,
+                    "kernel": "tc_ns_product_pair" if args.workload.startswith("large_batch")
+                    else "tc_ns_product(_pair)",
+                    "avg_launch_ms": (t5 - t1) / tc_launches * 1e3,
                     "peak_kind": f"{peak_kind} bf16 dense, sustained"}
     else:
         gbs = step_bytes(spec) / (ms_step / 1e3) / 1e9
