@@ -59,7 +59,8 @@ class dm_hparams_t(ctypes.Structure):
     _fields_ = [("mu", c_float), ("lr", c_float), ("weight_decay", c_float),
                 ("ns_steps", c_int32), ("a", c_float), ("b", c_float), ("c", c_float),
                 ("cond_eps", c_float), ("scale_mode", c_int32), ("scale_coef", c_float),
-                ("precision", c_int32), ("debug_flags", c_uint32)]
+                ("precision", c_int32), ("debug_flags", c_uint32), ("nesterov", c_int32),
+                ("reserved", c_int32 * 3)]
 
 
 class DimuonError(RuntimeError):

@@ -66,6 +66,8 @@ dm_status_t validate(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int
   for (float v : scalars)
     if (!(v == v) || v > 3.0e38f || v < -3.0e38f) return DM_ERR_INVALID_ARG;
   if (cond && !(hp->cond_eps >= 0.f)) return DM_ERR_INVALID_ARG;
+  if (hp->nesterov != 0 && hp->nesterov != 1) return DM_ERR_INVALID_ARG;
+  if (hp->reserved[0] || hp->reserved[1] || hp->reserved[2]) return DM_ERR_INVALID_ARG;
   for (int i = 0; i < n; ++i) {
     const dm_matrix_t& m = mats[i];
     if (m.rows < 1 || m.cols < 1 || m.rows > MAX_DIM || m.cols > MAX_DIM ||
@@ -364,6 +366,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
         tp.pad = keys[gi].first;
         tp.cluster = keys[gi].second;
         tp.conditioned = cond;
+        tp.nesterov = hp->nesterov;
         tp.ns_steps = hp->ns_steps;
         tp.mu = hp->mu;
         tp.lr = hp->lr;
@@ -433,6 +436,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     for (size_t b = 0; b < big.size(); b += K1_MAX) {
       std::memset(&p1, 0, sizeof(p1));
       p1.mu = hp->mu;
+      p1.nesterov = hp->nesterov;
       int tiles = 0;
       for (size_t q = b; q < std::min(big.size(), b + K1_MAX); ++q) {
         const MatPlan& p = *big[q];
@@ -635,6 +639,8 @@ void dm_default_hparams(dm_hparams_t* hp) {
   hp->scale_coef = 0.2f;
   hp->precision = DM_PREC_BF16_TC;
   hp->debug_flags = 0;
+  hp->nesterov = 0;
+  hp->reserved[0] = hp->reserved[1] = hp->reserved[2] = 0;
 }
 
 dm_status_t dm_workspace_size(const dm_matrix_t* mats, int n, const dm_hparams_t* hp,

@@ -61,6 +61,7 @@ constexpr int K1_MAX = 200;
 struct K1Params {
   int count;
   float mu;
+  int nesterov;           // X_0 from B_t = G + mu M_t instead of M_t
   int starts[K1_MAX + 1];
   K1Mat mats[K1_MAX];
 };
@@ -194,6 +195,7 @@ struct ThinParams {
   int pad;                // padded short side of every factor in the launch (2..32)
   int cluster;            // CTAs per factor (thread-block cluster size, 1..8)
   int conditioned;
+  int nesterov;
   int ns_steps;
   float mu, lr, decay, a, b, c, eps;
   int* status;

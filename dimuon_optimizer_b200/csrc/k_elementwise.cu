@@ -4,7 +4,7 @@
 //       Problem 4: (relative energy + eps)^(-1/4); off when M_{t-1} = 0,
 //       "Why the *last* momentum").
 //   K1  M_t = mu M_{t-1} + G ("Muon Optimizer 정리", "Update rule", eq. (1)),
-//       X_0 = R M_t C, per-tile sums of squares of X_0 and partial row /
+//       X_0 = R M_t C (R B_t C with B_t = G + mu M_t under Nesterov), per-tile sums of squares of X_0 and partial row /
 //       column energies of the stored M_t.
 //   K1b deterministic reduction of the K1 partials: energies of M_t (output
 //       for the next Dimuon step) and the Frobenius-norm scalars.
@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(256) k1_momentum(const __grid_constant__ K1Par
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           m8[q] = momentum_value(p.mu, m8[q], g8[q], mt.mdt);
-          x8[q] = round_to(rs * m8[q] * cscale[q], mt.xdt);
+          const float b = p.nesterov ? fmaf(p.mu, m8[q], g8[q]) : m8[q];
+          x8[q] = round_to(rs * b * cscale[q], mt.xdt);
           rsum += m8[q] * m8[q];
           csum[q] += m8[q] * m8[q];
           xsq += x8[q] * x8[q];
@@ -94,7 +95,8 @@ __global__ void __launch_bounds__(256) k1_momentum(const __grid_constant__ K1Par
         if (c < mt.cols) {
           const float gv = ld_elem(mt.G, base + q, mt.gdt);
           const float mv = momentum_value(p.mu, ld_elem(mt.M, base + q, mt.mdt), gv, mt.mdt);
-          const float xv = round_to(rs * mv * cscale[q], mt.xdt);
+          const float bv = p.nesterov ? fmaf(p.mu, mv, gv) : mv;
+          const float xv = round_to(rs * bv * cscale[q], mt.xdt);
           st_elem(mt.M, base + q, mt.mdt, mv);
           st_elem(mt.X0, r * mt.ldx + c, mt.xdt, xv);
           rsum += mv * mv;

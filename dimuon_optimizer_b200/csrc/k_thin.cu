@@ -236,9 +236,10 @@ __global__ void __launch_bounds__(THREADS, 2) thin_step(const __grid_constant__ 
   // loads of one chunk: a = first operand (G in pass 1, M in pass 2), b = second
   // (M in pass 1, W in pass 2)
   float av[NVEC][VEC], bv[NVEC][VEC];
-  auto load_chunk = [&](int64_t k0, const void* pa, int dta, const void* pb, int dtb) {
+  // second operand optional (with_b = false loads only pa)
+  auto load_chunk_pair = [&](int64_t k0, const void* pa, int dta, const void* pb, int dtb,
+                             float (&oa)[NVEC][VEC], float (&ob)[NVEC][VEC], bool with_b) {
     const int cw = (int)min((int64_t)CH, k_hi - k0);
-    load_energies(k0);
 #pragma unroll
     for (int q = 0; q < NVEC; ++q) {
       int i, kk;
@@ -246,11 +247,11 @@ __global__ void __launch_bounds__(THREADS, 2) thin_step(const __grid_constant__ 
       if (vec) {
         const bool ok = k0 < k_hi && i < r && kk < cw;  // vectors never straddle cw
         if (ok) {
-          ld4(pa, off(i, k0 + kk), dta, av[q]);
-          ld4(pb, off(i, k0 + kk), dtb, bv[q]);
+          ld4(pa, off(i, k0 + kk), dta, oa[q]);
+          if (with_b) ld4(pb, off(i, k0 + kk), dtb, ob[q]);
         } else {
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) av[q][e] = bv[q][e] = 0.f;
+          for (int e = 0; e < VEC; ++e) oa[q][e] = ob[q][e] = 0.f;
         }
       } else {
 #pragma unroll
@@ -259,11 +260,16 @@ __global__ void __launch_bounds__(THREADS, 2) thin_step(const __grid_constant__ 
           ecoord(i, kk, e, ie, ke);
           const bool ok = k0 < k_hi && ie < r && ke < cw;
           const int64_t o = ok ? off(ie, k0 + ke) : 0;
-          av[q][e] = ok ? ld_elem(pa, o, dta) : 0.f;
-          bv[q][e] = ok ? ld_elem(pb, o, dtb) : 0.f;
+          oa[q][e] = ok ? ld_elem(pa, o, dta) : 0.f;
+          ob[q][e] = (ok && with_b) ? ld_elem(pb, o, dtb) : 0.f;
         }
       }
     }
+  };
+
+  auto load_chunk = [&](int64_t k0, const void* pa, int dta, const void* pb, int dtb) {
+    load_energies(k0);
+    load_chunk_pair(k0, pa, dta, pb, dtb, av, bv, true);
   };
 
   // ---- pass 1 ----------------------------------------------------------------
@@ -292,7 +298,10 @@ __global__ void __launch_bounds__(THREADS, 2) thin_step(const __grid_constant__ 
         const bool ok = ie < r && ke < cw;
         m4[e] = ok ? momentum_value(p.mu, bv[q][e], av[q][e], mt.mdt) : 0.f;
         s.u.pass.ms[ie][ke] = m4[e];
-        s.u.pass.xs[ie][ke] = (double)s.Rv[ie] * (double)m4[e] * (double)s.Cc[ke];
+        // orthogonaliser input: M_t, or B_t = G + mu M_t under Nesterov
+        const double b = p.nesterov ? fma((double)p.mu, (double)m4[e], (double)av[q][e])
+                                    : (double)m4[e];
+        s.u.pass.xs[ie][ke] = (double)s.Rv[ie] * b * (double)s.Cc[ke];
         if (!vec && ok) st_elem(mt.M, off(ie, k0 + ke), mt.mdt, m4[e]);
       }
       if (vec && i < r && kk < cw) st4(mt.M, off(i, k0 + kk), mt.mdt, m4);
@@ -469,6 +478,13 @@ __global__ void __launch_bounds__(THREADS, 2) thin_step(const __grid_constant__ 
   const bool zero_update = s.sc[1] == 0.0;
 
   // ---- pass 2 ----------------------------------------------------------------
+  // Under Nesterov, X_0 needs G again: cv holds a chunk's G.
+  float cv[NVEC][VEC];
+  auto load_grad = [&](int64_t k0) {
+    if (!p.nesterov) return;
+    load_chunk_pair(k0, mt.G, mt.gdt, mt.G, mt.gdt, cv, cv, false);
+  };
+  load_grad(k_lo);
   load_chunk(k_lo, mt.M, mt.mdt, mt.W, mt.wdt);
   for (int64_t k0 = k_lo; k0 < k_hi; k0 += CH) {
     const int cw = (int)min((int64_t)CH, k_hi - k0);
@@ -484,10 +500,13 @@ __global__ void __launch_bounds__(THREADS, 2) thin_step(const __grid_constant__ 
         int ie, ke;
         ecoord(i, kk, e, ie, ke);
         s.u.pass.ms[ie][ke] = av[q][e];
-        s.u.pass.xs[ie][ke] = (double)s.Rv[ie] * (double)av[q][e] * (double)s.Cc[ke];
+        const double b = p.nesterov ? fma((double)p.mu, (double)av[q][e], (double)cv[q][e])
+                                    : (double)av[q][e];
+        s.u.pass.xs[ie][ke] = (double)s.Rv[ie] * b * (double)s.Cc[ke];
         wcur[q][e] = bv[q][e];
       }
     }
+    load_grad(k0 + CH);
     load_chunk(k0 + CH, mt.M, mt.mdt, mt.W, mt.wdt);  // in flight during the apply
     __syncthreads();
     if (cond) {

@@ -6,6 +6,8 @@
  * The step, per matrix (sources: web pages, cited by title and section):
  *   1. M_t = mu M_{t-1} + G
  *        "Muon Optimizer 정리" (dongju923.github.io), "Update rule", eq. (1).
+ *      With hp.nesterov the orthogonaliser's input is B_t = G + mu M_t in
+ *      place of M_t below (M_t is still what is stored).
  *   2. Dimuon only: R = diag((e_row/mean(e_row) + eps)^(-1/4)),
  *      C = diag((e_col/mean(e_col) + eps)^(-1/4)) from the row / column sums
  *      of squares of the PREVIOUS momentum M_{t-1}; X_0 = R M_t C.
@@ -118,6 +120,10 @@ typedef struct {
   float scale_coef;     /* DM_SCALE_MOONSHOT coefficient, default 0.2   */
   int32_t precision;    /* dm_precision_t                               */
   uint32_t debug_flags; /* 0 in production; bits below are test hooks   */
+  int32_t nesterov;     /* 1: orthogonalise B_t = G + mu M_t instead of
+                           M_t ("From PCG to Muon", section 3: the
+                           momentum-and-Nesterov combination)           */
+  int32_t reserved[3];  /* must be zero                                 */
 } dm_hparams_t;
 
 /* debug_flags bits (test hooks; none of them changes the arithmetic) */
@@ -130,7 +136,7 @@ typedef struct {
 
 /* Fills *hp with the defaults: mu 0.95, lr 0.02, wd 0, ns_steps 5,
  * (a,b,c) = (3.4445, -4.7750, 2.0315), cond_eps 1e-4, DM_SCALE_NONE,
- * scale_coef 0.2, DM_PREC_BF16_TC, debug_flags 0. */
+ * scale_coef 0.2, DM_PREC_BF16_TC, debug_flags 0, nesterov 0. */
 void dm_default_hparams(dm_hparams_t* hp);
 
 /* Bytes of device workspace a step over `mats[0..n)` needs with these

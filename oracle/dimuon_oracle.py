@@ -45,6 +45,12 @@ the repository's design notes):
     flag.
   * Hyper-parameters reach the CUDA library as float32; the oracle rounds each
     scalar through float32 before using it in fp64 arithmetic.
+  * Nesterov (optional, off by default): the matrix fed to the
+    orthogonaliser is B_t = G + mu M_t, with M_t the stored momentum
+    ([PCG2Muon], section 3 "Adam and Muon Optimizer": the orthogonaliser
+    takes the momentum-and-Nesterov combination B_t; its formula is not
+    printed, this is the standard look-ahead form).  M_t itself, and the
+    energies Dimuon reads, are unchanged.
 
 Parity pins for every function here live in tests/test_oracle_pins.py.
 """
@@ -87,6 +93,7 @@ class HParams:
     cond_eps: float = COND_EPS
     scale_mode: int = SCALE_NONE
     scale_coef: float = MOONSHOT_COEF
+    nesterov: bool = False
 
     def as_f32(self) -> "HParams":
         return HParams(mu=f32(self.mu), lr=f32(self.lr),
@@ -95,7 +102,7 @@ class HParams:
                        b=f32(self.b), c=f32(self.c),
                        cond_eps=f32(self.cond_eps),
                        scale_mode=int(self.scale_mode),
-                       scale_coef=f32(self.scale_coef))
+                       scale_coef=f32(self.scale_coef), nesterov=bool(self.nesterov))
 
 
 # ----------------------------------------------------------------------------
@@ -214,7 +221,8 @@ def optimizer_step(W_prev, G, M_prev, hp: HParams, *, conditioned: bool,
     """One Muon (conditioned=False) or Dimuon (conditioned=True) step on one
     matrix, in the page's order:
 
-      1. M_t = mu M_{t-1} + G, stored                ([MuonNote] eq. (1))
+      1. M_t = mu M_{t-1} + G, stored                ([MuonNote] eq. (1));
+         with Nesterov the orthogonaliser's input is B_t = G + mu M_t
       2. orient so rows <= cols
       3. Dimuon: R, C from the energies of M_{t-1}; X_0 = R M_t C  ([Dimuon])
       4. X <- X_0 / ||X_0||_F                          ([Sitech])
@@ -241,7 +249,8 @@ def optimizer_step(W_prev, G, M_prev, hp: HParams, *, conditioned: bool,
         if R is None or C is None:
             R = C = None
 
-    X0 = M_t if R is None else R[:, None] * M_t * C[None, :]
+    B_t = G + hp.mu * M_t if hp.nesterov else M_t
+    X0 = B_t if R is None else R[:, None] * B_t * C[None, :]
     transposed = rows > cols
     if transposed:
         X0 = X0.T

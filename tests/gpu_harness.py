@@ -77,7 +77,7 @@ def run_gpu_step(grp: Group, grads_host, hp, ws=None):
 def oracle_hp(hp):
     return orc.HParams(mu=hp.mu, lr=hp.lr, weight_decay=hp.weight_decay, ns_steps=hp.ns_steps,
                        a=hp.a, b=hp.b, c=hp.c, cond_eps=hp.cond_eps, scale_mode=hp.scale_mode,
-                       scale_coef=hp.scale_coef)
+                       scale_coef=hp.scale_coef, nesterov=bool(hp.nesterov))
 
 
 def rel_fro(x, y):

@@ -29,9 +29,10 @@ def test_every_declared_symbol_is_exported():
 
 def test_struct_layouts():
     assert ctypes.sizeof(dm.dm_matrix_t) == 80
-    assert ctypes.sizeof(dm.dm_hparams_t) == 48
+    assert ctypes.sizeof(dm.dm_hparams_t) == 64
     assert dm.dm_matrix_t.update_out.offset == 72
     assert dm.dm_hparams_t.debug_flags.offset == 44
+    assert dm.dm_hparams_t.nesterov.offset == 48
 
 
 def test_defaults_and_strings():

@@ -130,6 +130,21 @@ def test_thin_threshold_hook_matches_ns_path():
                                  ws=ws)
 
 
+@pytest.mark.parametrize("prec,tol", [(dm.DM_PREC_FP32, TOL_FP32), (dm.DM_PREC_BF16_TC, TOL_BF16)])
+@pytest.mark.parametrize("cond", [False, True])
+def test_nesterov(prec, tol, cond):
+    """B_t = G + mu M_t feeds the orthogonaliser on every path (Newton-Schulz
+    and thin)."""
+    shapes = [(200, 330), (330, 200), (8, 600), (600, 16)]
+    grp = Group(shapes, BF, BF, F32, cond=cond, seed=21)
+    hp = hparams(prec, nesterov=1, weight_decay=0.02)
+    ws = None
+    for t in range(3):
+        thin_tol = [tol, tol, TOL_FP32, TOL_FP32]
+        _, ws = step_and_compare(grp, gaussian(shapes, 900 + t, scale_cols=True), hp,
+                                 max(thin_tol), ws=ws)
+
+
 # --------------------------------------------------------------------------
 # invariants and edge cases
 # --------------------------------------------------------------------------

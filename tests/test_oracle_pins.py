@@ -41,7 +41,7 @@ def bf_transpose(A):
 
 
 def brute_force_step(W, G, M, mu, lr, wd, a, b, c, steps, eps, kappa_coef,
-                     moonshot, e_row=None, e_col=None):
+                     moonshot, e_row=None, e_col=None, nesterov=False):
     """Pure-Python restatement of one step on a tiny matrix (lists of floats).
     Orientation is handled by transposing when rows > cols."""
     rows, cols = len(G), len(G[0])
@@ -54,7 +54,9 @@ def brute_force_step(W, G, M, mu, lr, wd, a, b, c, steps, eps, kappa_coef,
         mc = sum(e_col) / cols
         Rv = [(e / mr + eps) ** -0.25 for e in e_row]
         Cv = [(e / mc + eps) ** -0.25 for e in e_col]
-    X0 = [[Mt[i][j] * (Rv[i] * Cv[j] if Rv else 1.0) for j in range(cols)]
+    Bt = [[G[i][j] + mu * Mt[i][j] if nesterov else Mt[i][j] for j in range(cols)]
+          for i in range(rows)]
+    X0 = [[Bt[i][j] * (Rv[i] * Cv[j] if Rv else 1.0) for j in range(cols)]
           for i in range(rows)]
     tall = rows > cols
     if tall:
@@ -435,3 +437,40 @@ def test_zero_gradient_zero_update():
     assert not r.nonfinite
     np.testing.assert_array_equal(r.O, 0.0)
     np.testing.assert_array_equal(r.W, W)
+
+
+@pytest.mark.parametrize("cond", [False, True])
+def test_nesterov_brute_force(cond):
+    """Nesterov: the orthogonaliser takes B_t = G + mu M_t (From PCG to Muon,
+    section 3, momentum-and-Nesterov combination); M_t and the energies are
+    those of the plain momentum."""
+    rng = np.random.default_rng(31)
+    shape = (5, 8)
+    W = rng.standard_normal(shape) * 0.02
+    G = rng.standard_normal(shape)
+    M = rng.standard_normal(shape)
+    e_r = rng.exponential(1.0, shape[0])
+    e_c = rng.exponential(1.0, shape[1])
+    hp = orc.HParams(mu=0.9, lr=0.03, nesterov=True)
+    h = hp.as_f32()
+    want = brute_force_step(W.tolist(), G.tolist(), M.tolist(), h.mu, h.lr, 0.0, h.a, h.b,
+                            h.c, h.ns_steps, h.cond_eps, h.scale_coef, False,
+                            e_r.tolist() if cond else None, e_c.tolist() if cond else None,
+                            nesterov=True)
+    got = orc.optimizer_step(W, G, M, hp, conditioned=cond, e_row_prev=e_r, e_col_prev=e_c)
+    np.testing.assert_allclose(got.O, want[2], rtol=1e-10, atol=1e-13)
+    plain = orc.optimizer_step(W, G, M, orc.HParams(mu=0.9, lr=0.03), conditioned=cond,
+                               e_row_prev=e_r, e_col_prev=e_c)
+    np.testing.assert_array_equal(got.M, plain.M)
+    assert np.abs(got.O - plain.O).max() > 1e-3
+
+
+def test_nesterov_without_momentum_is_plain():
+    """With mu = 0, B_t = G = M_t: Nesterov changes nothing."""
+    rng = np.random.default_rng(32)
+    W = rng.standard_normal((6, 9))
+    G = rng.standard_normal((6, 9)).astype(np.float32).astype(np.float64)  # = stored M_t
+    Z = np.zeros((6, 9))
+    a = orc.muon_step(W, G, Z, orc.HParams(mu=0.0, nesterov=True))
+    b = orc.muon_step(W, G, Z, orc.HParams(mu=0.0))
+    np.testing.assert_array_equal(a.O, b.O)
