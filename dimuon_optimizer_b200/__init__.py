@@ -41,6 +41,7 @@ DM_THIN_MAX = 32
 DM_DBG_NO_THIN = 0x1
 DM_DBG_TC_SINGLE = 0x2
 DM_DBG_TC_PAIR = 0x4
+DM_DBG_FORCE_TIMEOUT = 0x8
 
 DM_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 

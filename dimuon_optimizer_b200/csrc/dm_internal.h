@@ -23,6 +23,10 @@ enum {
 // Device status codes (mirror dm_status_t).
 enum { ST_OK = 0, ST_TIMEOUT = 5, ST_NONFINITE = 6 };
 
+// debug_flags bit read inside the tensor-core kernels (mirrors the public
+// DM_DBG_FORCE_TIMEOUT).
+constexpr unsigned DBG_FORCE_TIMEOUT = 0x8u;
+
 // ------------------------------- K0 ---------------------------------------
 // Dimuon conditioning vectors R, C from the previous momentum's energies.
 struct K0Mat {

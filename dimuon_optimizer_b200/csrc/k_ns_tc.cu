@@ -38,6 +38,7 @@ constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // any single wait > 2 s is a hang
 constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
+constexpr uint64_t FORCED_LIMIT_NS = 20000000ull;   // forced-timeout hook: 20 ms
 
 struct Tile {
   int g, lt, tm, tn;
@@ -60,7 +61,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* never = drain + 1;  // nothing ever arrives (forced-timeout hook)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -75,6 +77,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
       mbar_init(&tempty[a], 8);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
+    mbar_init(never, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -86,6 +89,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+
+  if (p.debug & DBG_FORCE_TIMEOUT) {
+    // Test hook: one thread waits, with a short limit, on a barrier nothing
+    // arrives on.  Its expiry takes the ordinary timeout path (abort flag,
+    // status word) before any copy or product is issued, so every role then
+    // leaves at its first abort check.
+    if (threadIdx.x == 0) mbar_wait_bounded(never, 0, abort, p.status, FORCED_LIMIT_NS);
+    __syncthreads();
+  }
 
   if (warp == 0) {
     // ----------------------------- TMA producer -----------------------------
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
         // Let the copies already in flight land before the CTA exits.
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s))
-            mbar_wait_bounded(&full[s], (armed_par >> s) & 1u, abort, nullptr, DRAIN_LIMIT_NS);
+            mbar_wait_drain(&full[s], (armed_par >> s) & 1u, DRAIN_LIMIT_NS);
       }
     }
   } else if (warp == 1) {
@@ -188,7 +200,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
       }
       // Every MMA this thread issued has completed once `drain` flips.
       mma_commit(drain);
-      mbar_wait_bounded(drain, 0, abort, nullptr, DRAIN_LIMIT_NS);
+      mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);
     }
   } else {
     // ------------------------------- epilogue -------------------------------

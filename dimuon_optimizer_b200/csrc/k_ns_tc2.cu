@@ -43,6 +43,7 @@ constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
+constexpr uint64_t FORCED_LIMIT_NS = 20000000ull;   // forced-timeout hook: 20 ms
 constexpr uint16_t PAIR_MASK = 0x3;
 
 struct Tile {
@@ -66,7 +67,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* never = drain + 1;  // nothing ever arrives (forced-timeout hook)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -83,6 +85,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
       mbar_init(&tempty[a], 16);  // leader: 8 local + 8 peer epilogue warps
     }
     mbar_init(drain, 1);
+    mbar_init(never, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -94,6 +97,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
   cluster_sync_all();  // barriers initialised in both CTAs, TMEM address published
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+
+  if (p.debug & DBG_FORCE_TIMEOUT) {
+    // Test hook: one leader thread waits, with a short limit, on a barrier
+    // nothing arrives on.  Its expiry takes the ordinary timeout path (abort
+    // flag, status word); the abort is copied into the peer before the
+    // cluster barrier, so no copy or product is issued in either CTA and
+    // every role leaves at its first abort check.
+    if (threadIdx.x == 0 && rank == 0) {
+      mbar_wait_bounded(never, 0, abort, p.status, FORCED_LIMIT_NS);
+      st_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(abort)), 1), 1u);
+    }
+    cluster_sync_all();
+  }
 
   if (warp == 0) {
     // ----------------------------- TMA producer -----------------------------
@@ -149,7 +165,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
         // Both CTAs' copies in flight complete on the leader's barriers.
         for (int s = 0; s < STAGES; ++s)
           if (armed & (1u << s))
-            mbar_wait_bounded(&full[s], (armed_par >> s) & 1u, abort, nullptr, DRAIN_LIMIT_NS);
+            mbar_wait_drain(&full[s], (armed_par >> s) & 1u, DRAIN_LIMIT_NS);
       }
     }
   } else if (warp == 1) {
@@ -196,7 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
         mma_commit_pair(&tfull[acc], PAIR_MASK);  // accumulator ready in both CTAs
       }
       mma_commit_pair(drain, 0x1);
-      mbar_wait_bounded(drain, 0, abort, nullptr, DRAIN_LIMIT_NS);
+      mbar_wait_drain(drain, 0, DRAIN_LIMIT_NS);
     }
   } else {
     // ------------------------------- epilogue -------------------------------

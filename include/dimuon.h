@@ -133,6 +133,15 @@ typedef struct {
                                      (128 x 256 tiles) only                */
 #define DM_DBG_TC_PAIR 0x4u       /* tensor-core products on CTA pairs
                                      (256 x 256 tiles) only                */
+#define DM_DBG_FORCE_TIMEOUT 0x8u /* failure-detection hook: each
+                                     tensor-core product launch makes one
+                                     bounded wait run out (20 ms, on a
+                                     barrier nothing arrives on) before it
+                                     issues any copy or product; the launch
+                                     then leaves without writing and the
+                                     device status reads
+                                     DM_ERR_DEVICE_TIMEOUT.  The step's
+                                     outputs are then meaningless.         */
 
 /* Fills *hp with the defaults: mu 0.95, lr 0.02, wd 0, ns_steps 5,
  * (a,b,c) = (3.4445, -4.7750, 2.0315), cond_eps 1e-4, DM_SCALE_NONE,
