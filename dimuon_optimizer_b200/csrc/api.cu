@@ -3,7 +3,8 @@
 //
 // Step order (one stream, no host synchronisation):
 //   status word cleared
-//   thin factors (short side <= DM_THIN_MAX): one CTA per factor, whole step
+//   thin factors (short side <= DM_THIN_MAX): thin_gram, thin_iterate,
+//        thin_apply per padded short side (Gram route, whole step)
 //   other matrices:
 //     K0   (Dimuon) R, C from the previous momentum's energies
 //     K1   momentum, X_0 = R M_t C, partial norms / energies
@@ -49,8 +50,24 @@ struct MatPlan {
   size_t off_X[2], off_A, off_B;
 };
 
+// One group of thin factors launched together (same padded short side).
+struct ThinLaunch {
+  int pad;
+  int combo;                // storage combination of the staged path, -1 = register path
+  std::vector<int> idx;     // matrix indices
+  std::vector<int> starts;  // first slab of each factor, plus the total
+  size_t off_mats, off_starts, off_unit_f, off_part, off_rpart, off_T, off_fsc;
+};
+
+// Header of the workspace: the device status word at 0, the thin slab
+// counters (two per group) from THIN_CTR_OFFSET; zeroed at the start of a step.
+constexpr size_t THIN_CTR_OFFSET = 64;
+
+int thin_pad(int r) { return r <= 4 ? r : r <= 8 ? 8 : r <= 16 ? 16 : 32; }
+
 struct Layout {
   std::vector<MatPlan> mats;
+  std::vector<ThinLaunch> thin;
   size_t bytes = 0;
   bool tc = false;
   bool cond = false;
@@ -127,6 +144,48 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
       p.off_B = take((size_t)p.m * p.ldm * esz, 1024);
     }
     L.mats.push_back(p);
+  }
+  // thin factors: one launch group per padded short side and path (staged
+  // path for r == pad, long side a multiple of 8, 16-byte aligned buffers and
+  // a supported storage combination; register path otherwise)
+  auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+  std::vector<std::pair<int, int>> pads;
+  std::vector<std::vector<int>> members;
+  for (const MatPlan& p : L.mats) {
+    if (!p.thin) continue;
+    const int pad = thin_pad(p.m);
+    const dm_matrix_t& um = mats[p.idx];
+    int combo = thin_bulk_combo(um.grad_dtype, um.momentum_dtype, um.weight_dtype);
+    const bool ok = p.m == pad && pad >= 2 && pad != 3 && p.n % 8 == 0 && al16(um.grad) &&
+                    al16(um.momentum) && al16(um.weight) && al16(um.update_out) &&
+                    (!cond || (al16(um.row_energy) && al16(um.col_energy)));
+    if (!ok || (hp->debug_flags & DM_DBG_THIN_REGS)) combo = -1;
+    const std::pair<int, int> key(pad, combo);
+    size_t g = 0;
+    while (g < pads.size() && pads[g] != key) ++g;
+    if (g == pads.size()) {
+      pads.push_back(key);
+      members.emplace_back();
+    }
+    members[g].push_back(p.idx);
+  }
+  for (size_t g = 0; g < pads.size(); ++g) {
+    ThinLaunch tl;
+    tl.pad = pads[g].first;
+    tl.combo = pads[g].second;
+    tl.idx = members[g];
+    const int slab = thin_slab(tl.pad);
+    tl.starts.push_back(0);
+    for (int i : tl.idx) tl.starts.push_back(tl.starts.back() + (int)ceil_div(L.mats[i].n, slab));
+    const size_t units = (size_t)tl.starts.back(), count = tl.idx.size();
+    tl.off_mats = take(count * sizeof(ThinMat), 256);
+    tl.off_starts = take((count + 1) * sizeof(int), 256);
+    tl.off_unit_f = take(units * sizeof(int), 256);
+    tl.off_part = take(units * 2 * thin_part_doubles(tl.pad) * sizeof(double), 256);
+    tl.off_rpart = take(units * tl.pad * sizeof(float), 256);
+    tl.off_T = take(count * tl.pad * tl.pad * sizeof(double), 256);
+    tl.off_fsc = take(count * 4 * sizeof(double), 256);
+    L.thin.push_back(std::move(tl));
   }
   L.bytes = round_up(cur, 1024);
   return L;
@@ -329,74 +388,76 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
   DM_CUDA(cudaGetDevice(&dev));
   const float decay = 1.f - hp->lr * hp->weight_decay;
 
-  DM_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  // status word and thin slab counters
+  DM_CUDA(cudaMemsetAsync(ws, 0, THIN_CTR_OFFSET + 2 * sizeof(int) * L.thin.size(), s));
   if (n == 0) return DM_OK;
 
   // ---------------------------- thin factors -------------------------------
-  // Launches group factors by padded short side (2..32) and cluster size.
-  {
-    std::vector<std::pair<int, int>> keys;
-    std::vector<std::vector<int>> groups;
-    for (const MatPlan& p : L.mats) {
-      if (!p.thin) continue;
-      int pad = 2;
-      while (pad < p.m) pad *= 2;
-      const int64_t elems = (int64_t)p.m * p.n;
-      int cl = elems >= 65536 ? 8 : elems >= 32768 ? 4 : elems >= 16384 ? 2 : 1;
-      const int64_t chunks = ceil_div(p.n, 4096 / pad);  // 4096-element chunks
-      while (cl > 1 && chunks < cl) cl /= 2;
-      const std::pair<int, int> key(pad, cl);
-      size_t g = 0;
-      while (g < keys.size() && keys[g] != key) ++g;
-      if (g == keys.size()) {
-        keys.push_back(key);
-        groups.emplace_back();
+  for (size_t gi = 0; gi < L.thin.size(); ++gi) {
+    const ThinLaunch& tl = L.thin[gi];
+    ThinMat* mats_dev = reinterpret_cast<ThinMat*>(ws + tl.off_mats);
+    int* starts_dev = reinterpret_cast<int*>(ws + tl.off_starts);
+    double* fsc = reinterpret_cast<double*>(ws + tl.off_fsc);
+    const int count = (int)tl.idx.size();
+    for (int first = 0; first < count; first += THIN_MAX) {
+      static thread_local ThinSetupParams sp;
+      std::memset(&sp, 0, sizeof(sp));
+      sp.count = std::min(THIN_MAX, count - first);
+      sp.first = first;
+      sp.conditioned = cond;
+      sp.mats_dst = mats_dev;
+      sp.starts_dst = starts_dev;
+      sp.unit_f_dst = reinterpret_cast<int*>(ws + tl.off_unit_f);
+      sp.fsc = fsc;
+      for (int q = 0; q <= sp.count; ++q) sp.starts[q] = tl.starts[first + q];
+      for (int q = 0; q < sp.count; ++q) {
+        const dm_matrix_t& um = mats[tl.idx[first + q]];
+        ThinMat& t = sp.mats[q];
+        t.G = um.grad;
+        t.M = um.momentum;
+        t.W = um.weight;
+        t.upd = um.update_out;
+        t.e_row = cond ? um.row_energy : nullptr;
+        t.e_col = cond ? um.col_energy : nullptr;
+        t.rows = um.rows;
+        t.cols = um.cols;
+        t.gdt = um.grad_dtype;
+        t.mdt = um.momentum_dtype;
+        t.wdt = um.weight_dtype;
+        t.kappa = kappa_of(hp, um.rows, um.cols);
+        auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+        t.vec = al16(um.grad) && al16(um.momentum) && al16(um.weight) && al16(um.update_out);
       }
-      groups[g].push_back(p.idx);
+      DM_CUDA(launch_thin_setup(sp, s));
     }
-    for (size_t gi = 0; gi < groups.size(); ++gi) {
-      const std::vector<int>& idx = groups[gi];
-      const int nchunks = (int)ceil_div((int64_t)idx.size(), THIN_MAX);
-      for (int ch = 0; ch < nchunks; ++ch) {
-        // split evenly so launches are balanced
-        const size_t b = idx.size() * ch / nchunks, e = idx.size() * (ch + 1) / nchunks;
-        static thread_local ThinParams tp;
-        std::memset(&tp, 0, sizeof(tp));
-        tp.count = (int)(e - b);
-        tp.pad = keys[gi].first;
-        tp.cluster = keys[gi].second;
-        tp.conditioned = cond;
-        tp.nesterov = hp->nesterov;
-        tp.ns_steps = hp->ns_steps;
-        tp.mu = hp->mu;
-        tp.lr = hp->lr;
-        tp.decay = decay;
-        tp.a = hp->a;
-        tp.b = hp->b;
-        tp.c = hp->c;
-        tp.eps = hp->cond_eps;
-        tp.status = status;
-        for (size_t q = b; q < e; ++q) {
-          const dm_matrix_t& um = mats[idx[q]];
-          ThinMat& t = tp.mats[q - b];
-          t.G = um.grad;
-          t.M = um.momentum;
-          t.W = um.weight;
-          t.upd = um.update_out;
-          t.e_row = cond ? um.row_energy : nullptr;
-          t.e_col = cond ? um.col_energy : nullptr;
-          t.rows = um.rows;
-          t.cols = um.cols;
-          t.gdt = um.grad_dtype;
-          t.mdt = um.momentum_dtype;
-          t.wdt = um.weight_dtype;
-          t.kappa = kappa_of(hp, um.rows, um.cols);
-          auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
-          t.vec = al16(um.grad) && al16(um.momentum) && al16(um.weight) && al16(um.update_out);
-        }
-        DM_CUDA(launch_thin(tp, s));
-      }
-    }
+    ThinParams tp;
+    std::memset(&tp, 0, sizeof(tp));
+    tp.count = count;
+    tp.pad = tl.pad;
+    tp.units = tl.starts.back();
+    tp.conditioned = cond;
+    tp.nesterov = hp->nesterov;
+    tp.ns_steps = hp->ns_steps;
+    tp.mu = hp->mu;
+    tp.lr = hp->lr;
+    tp.decay = decay;
+    tp.a = hp->a;
+    tp.b = hp->b;
+    tp.c = hp->c;
+    tp.eps = hp->cond_eps;
+    tp.status = status;
+    tp.mats = mats_dev;
+    tp.starts = starts_dev;
+    tp.unit_f = reinterpret_cast<const int*>(ws + tl.off_unit_f);
+    tp.part = reinterpret_cast<double*>(ws + tl.off_part);
+    tp.rpart = reinterpret_cast<float*>(ws + tl.off_rpart);
+    tp.T = reinterpret_cast<double*>(ws + tl.off_T);
+    tp.fsc = fsc;
+    tp.counters = reinterpret_cast<int*>(ws + THIN_CTR_OFFSET) + 2 * gi;
+    if (tl.combo >= 0)
+      DM_CUDA(launch_thin_bulk(tp, tl.combo, sm_count(dev), s));
+    else
+      DM_CUDA(launch_thin(tp, sm_count(dev), s));
   }
 
   // -------------------------- Newton-Schulz path ---------------------------

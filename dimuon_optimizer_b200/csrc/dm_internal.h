@@ -180,7 +180,12 @@ struct K3Params {
 };
 
 // ------------------------------ thin --------------------------------------
-// Whole step of one short-side <= 32 factor in one CTA (Gram route).
+// Whole step of short-side <= 32 factors (Gram route): per padded short
+// side, thin_setup copies the factor descriptors into the workspace (up to
+// THIN_MAX per launch) and sums the previous energies; thin_gram,
+// thin_iterate and thin_apply then cover every factor of that padded side,
+// the streaming two in slabs of thin_slab(pad) long-side columns handed out
+// by a device counter.
 struct ThinMat {
   const void* G;
   void* M;
@@ -194,17 +199,39 @@ struct ThinMat {
   float kappa;
 };
 constexpr int THIN_MAX = 256;
+struct ThinSetupParams {
+  int count;              // factors in this launch (<= THIN_MAX)
+  int first;              // their first index in the group
+  int conditioned;
+  ThinMat* mats_dst;      // group descriptor table (device)
+  int* starts_dst;        // group slab starts (device), count + 1 entries written
+  int* unit_f_dst;        // group slab -> factor table (device)
+  double* fsc;            // group per-factor scalars (device)
+  int starts[THIN_MAX + 1];
+  ThinMat mats[THIN_MAX];
+};
 struct ThinParams {
-  int count;
-  int pad;                // padded short side of every factor in the launch (2..32)
-  int cluster;            // CTAs per factor (thread-block cluster size, 1..8)
+  int count;              // factors in the group
+  int pad;                // padded short side (1, 2, 3, 4, 8, 16, 32)
+  int units;              // slabs over all factors
+  int grid_gram, grid_apply;  // persistent grid sizes
   int conditioned;
   int nesterov;
   int ns_steps;
   float mu, lr, decay, a, b, c, eps;
   int* status;
-  ThinMat mats[THIN_MAX];
+  const ThinMat* mats;    // [count]
+  const int* starts;      // [count + 1]: first slab of each factor
+  const int* unit_f;      // [units]: factor of each slab
+  double* part;           // [units][2][thin_part_doubles(pad)]: S_1, S_2 slab partials
+  float* rpart;           // [units][pad]: short-side energy partials
+  double* T;              // [count][pad * pad]: apply matrices
+  double* fsc;            // [count][4]: sums of the previous long- / short-side
+                          // energies, conditioning on, zero update
+  int* counters;          // [2]: next slab of thin_gram / thin_apply (zero at the start)
 };
+int thin_part_doubles(int pad);
+int thin_slab(int pad);
 
 // ------------------------------ launches ----------------------------------
 cudaError_t launch_k0(const K0Params& p, cudaStream_t s);
@@ -218,6 +245,11 @@ int tc_smem_bytes();
 constexpr int TC2_BM = 256, TC2_BN = 256;  // CTA-pair output tile
 cudaError_t launch_tc_pair(const TcParams& p, int pairs, cudaStream_t s);
 int tc_pair_smem_bytes();
-cudaError_t launch_thin(const ThinParams& p, cudaStream_t s);
+cudaError_t launch_thin_setup(const ThinSetupParams& p, cudaStream_t s);
+cudaError_t launch_thin(ThinParams& p, int nsm, cudaStream_t s);
+cudaError_t launch_thin_iterate(const ThinParams& p, cudaStream_t s);
+// shared-memory staged thin path (k_thin_bulk.cu)
+int thin_bulk_combo(int gdt, int mdt, int wdt);
+cudaError_t launch_thin_bulk(ThinParams& p, int combo, int nsm, cudaStream_t s);
 
 }  // namespace dm

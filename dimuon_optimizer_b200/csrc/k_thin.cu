@@ -1,106 +1,388 @@
 // Whole Muon / Dimuon step for thin factors (short side r <= 32, e.g. LoRA A
-// (r x n) and B (n x r)), one thread-block cluster per factor.
+// (r x n) and B (n x r)), per padded short side RP.
 //
 // The Newton-Schulz iterate is a left-multiple of the start matrix: each step
 // X <- (aI + bA + cA^2) X with A = X X^T, so X_k = P_k X_0 with an r x r
-// polynomial P_k in the Gram matrix A_0 = X_0 X_0^T; A_{k+1} = Q_k A_k Q_k.
-// ("From PCG to Muon", section 6 "Muon's Gram Matrix": the orthogonaliser
-// normalises the global Gram matrix G^T G; sitech.ge, "Instead of SVD -
-// Newton-Schulz" for the iteration itself.)  The factor is streamed twice and
-// the iteration runs in r x r space:
-//   pass 1   M_t = mu M_{t-1} + G (stored), X_0 = R M_t C in fp64,
-//            A_0 += X_0 X_0^T and H += X_0 C^2 X_0^T in fp64 (exact products),
-//            row energies of M_t
-//   reduce   Gram partials of the cluster's CTAs through distributed shared
-//            memory, in rank order (deterministic)
-//   iterate  rank 0: P <- Q P, A <- Q A Q in fp64; the Frobenius norms of
-//            X_5 = P X_0 / s and Y = R X_5 C follow from A_0 and H; T = factor P
-//   pass 2   reload M_t (L2-resident), O = R (T X_0) C, W update, column
-//            energies of M_t
-// The fp64 products (Gram matrices, r x r iteration, apply) run on the fp64
-// tensor-core MMA (mma.sync m8n8k4) for r > 4; r <= 4 uses plain fp64 FMAs.
-// Each CTA of the cluster owns a contiguous run of 4096-element chunks of the
-// long side; the next chunk's loads are in flight during the current chunk's
-// arithmetic.
+// polynomial P_k in the Gram matrix A_0 = X_0 X_0^T ("From PCG to Muon",
+// section 6 "Muon's Gram Matrix": the orthogonaliser normalises the global
+// Gram matrix; sitech.ge, "Instead of SVD - Newton-Schulz" for the iteration).
+// With X_0 = R B C (B = M_t, or G + mu M_t under Nesterov; R = C = I in Muon
+// mode) and b_j the j-th long-side column of B:
+//   A_0 = R S_1 R,  S_1 = sum_j C_j^2 b_j b_j^T
+//   H   = X_0 C^2 X_0^T = R S_2 R,  S_2 = sum_j C_j^4 b_j b_j^T
+//   O(:, j) = C_j^2 T b_j,  T = f R P_5 R,
+// f = kappa / ||X_0||_F, times ||X_5||_F / ||R X_5 C||_F when Dimuon
+// conditioning is on; both norms follow from A_0 and H.  Launches:
+//   thin_setup   one CTA per factor (up to THIN_MAX per launch): descriptor
+//                into the workspace, sums of the previous energies
+//   thin_gram    persistent CTAs taking slabs of long-side columns from a
+//                device counter: M_t = mu M_{t-1} + G (fp64, one rounding,
+//                stored), the slab's S_1 / S_2 partials (fp64), short-side
+//                energy partials
+//   thin_iterate one CTA per factor: partials summed in slab order, R, the
+//                r x r iteration, T, the new short-side energies
+//   thin_apply   persistent CTAs over slabs: O = C^2 T B, W update, the new
+//                long-side energies
+// fp64 products use the fp64 tensor-core MMA (mma.sync m8n8k4) for RP >= 8
+// (RP = 8, 16, 32); RP <= 4 (RP == r) uses fp64 FMAs, one lane per four
+// long-side columns.  The streaming loops keep everything in registers, with
+// the next step's loads in flight while the current step computes; each warp
+// walks its own columns of the slab with no block-wide barrier.
 // Dimuon conditioning, renormalisation, scale and decay follow "Dimuon: LoRA
 // 에 맞춰 다시 짠 Muon" ("-1/4 power from both sides", "Why the *last*
 // momentum", Problem 4) and "Muon Optimizer 정리" (eq. (1)-(3), "Scaling up").
-#include <cooperative_groups.h>
+#include <algorithm>
 
 #include "dm_common.cuh"
-
-namespace cg = cooperative_groups;
+#include "dm_thin.cuh"
 
 namespace dm {
 namespace {
 
-constexpr int THREADS = 256;
-constexpr int WARPS = THREADS / 32;
-constexpr int CHUNK_ELEMS = 4096;  // RP x CH elements per chunk
-constexpr int VEC = 4;             // elements per vector access
-constexpr int NVEC = CHUNK_ELEMS / VEC / THREADS;  // vectors per thread per chunk (4)
+using namespace thin;
 
+// Next slab for this CTA from the device counter (the same for every thread).
+__device__ __forceinline__ int next_unit(int* counter, int* slot) {
+  __syncthreads();  // every thread is done with the previous slab's shared state
+  if (threadIdx.x == 0) *slot = atomicAdd(counter, 1);
+  __syncthreads();
+  return *slot;
+}
+
+// Runs step() over this warp's long-side positions c0, c0 + stride, ... < c_hi,
+// with the loads of the next position issued before the current one computes
+// (DB) or one position at a time.
+template <bool DB, typename Frag, typename Load, typename Step>
+__device__ __forceinline__ void stream_positions(int64_t c0, int64_t stride, int64_t c_hi,
+                                                 Load&& load, Step&& step) {
+  if (c0 >= c_hi) return;
+  Frag fa, fb;
+  load(fa, c0);
+  if constexpr (DB) {
+    for (int64_t c = c0;;) {
+      const int64_t c1 = c + stride;
+      if (c1 < c_hi) load(fb, c1);
+      step(fa, c);
+      if (c1 >= c_hi) break;
+      const int64_t c2 = c1 + stride;
+      if (c2 < c_hi) load(fa, c2);
+      step(fb, c1);
+      if (c2 >= c_hi) break;
+      c = c2;
+    }
+  } else {
+    for (int64_t c = c0; c < c_hi; c += stride) {
+      if (c != c0) load(fa, c);
+      step(fa, c);
+    }
+  }
+}
+
+// ===========================================================================
+// thin_setup: descriptors into the workspace, sums of the previous energies
+// ===========================================================================
+__global__ void __launch_bounds__(256) thin_setup(const __grid_constant__ ThinSetupParams p) {
+  __shared__ double red[32];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const ThinMat& mt = p.mats[b];
+  const int f = p.first + b;
+  if (tid == 0) {
+    p.mats_dst[f] = mt;
+    p.starts_dst[f] = p.starts[b];
+    if (b == p.count - 1) p.starts_dst[f + 1] = p.starts[b + 1];
+  }
+  for (int u = p.starts[b] + tid; u < p.starts[b + 1]; u += blockDim.x) p.unit_f_dst[u] = f;
+  const Geo q = geometry(mt, p.conditioned);
+  double sc = 0.0, sr = 0.0;
+  if (q.cond) {
+    for (int i = tid; i < q.r; i += blockDim.x) sr += (double)q.e_r[i];
+    for (int64_t k = tid; k < q.n; k += blockDim.x) sc += (double)q.e_c[k];
+  }
+  sc = block_sum_d(sc, red);
+  sr = block_sum_d(sr, red);
+  if (tid == 0) {
+    p.fsc[4 * f] = sc;
+    p.fsc[4 * f + 1] = sr;
+  }
+}
+
+// ===========================================================================
+// thin_gram: momentum, Gram partials, short-side energy partials
+// ===========================================================================
 template <int RP>
-struct Cfg {
-  static constexpr bool MMA = RP >= 8;                // fp64 tensor-core path
-  static constexpr int CH = CHUNK_ELEMS / RP;         // columns per chunk
-  static constexpr int XLD = CH + 4;                  // padded fp64 row (8-bank shift)
-  static constexpr int MLD = CH + 1;                  // padded fp32 row
-  static constexpr int SLD = RP + 1;                  // padded r x r row
-  static constexpr int NBD = RP / 8;                  // 8-row blocks (MMA path)
-  static constexpr int NUB = NBD * (NBD + 1) / 2;     // upper-triangle 8x8 blocks
-  // per-warp partials (MMA path: one RP x RP matrix per warp) or per-thread
-  // partials (small path: two per thread)
-  static constexpr int PARTN =
-      WARPS * RP * RP > 2 * THREADS ? WARPS * RP * RP : 2 * THREADS;
+struct GramFrag {
+  static constexpr int ROWS = TCfg<RP>::MMA ? TCfg<RP>::NB : RP;
+  float m[ROWS][4], g[ROWS][4];
+  float ec[4];  // previous long-side energies of the four columns
 };
 
 template <int RP>
-struct ThinSmem {
-  union {
-    struct {
-      double xs[RP][Cfg<RP>::XLD];   // X_0 chunk (fp64)
-      float ms[RP][Cfg<RP>::MLD];    // stored momentum chunk, then the update chunk
-    } pass;
-    double part[Cfg<RP>::PARTN];     // Gram / H partials
-    struct {
-      double G[RP][Cfg<RP>::SLD], H[RP][Cfg<RP>::SLD], P[RP][Cfg<RP>::SLD],
-          A[RP][Cfg<RP>::SLD], Q[RP][Cfg<RP>::SLD], S[RP][Cfg<RP>::SLD];
-    } it;
-  } u;
-  double Gc[RP * RP];  // this CTA's Gram partial (rank 0 reads it over DSMEM)
-  double Hc[RP * RP];
-  double T[RP][Cfg<RP>::SLD];  // factor * P, broadcast from rank 0
-  float rowp[RP];              // row-energy partial of this CTA's slice
-  float Rv[RP];
-  float Cc[Cfg<RP>::CH];
-  float red32[THREADS];
+__global__ void __launch_bounds__(TT) thin_gram(const __grid_constant__ ThinParams p) {
+  using Cf = TCfg<RP>;
+  using Frag = GramFrag<RP>;
+  __shared__ double red_s[TW][2][Cf::PART];
+  __shared__ float red_e[TW][RP];
+  __shared__ int s_unit;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float mu = p.mu, eps = p.eps;
+
+  for (int u = next_unit(p.counters, &s_unit); u < p.units; u = next_unit(p.counters, &s_unit)) {
+    const int f = p.unit_f[u];
+    const ThinMat mt = p.mats[f];  // by value: stores cannot alias it
+    const Geo q = geometry(mt, p.conditioned);
+    const int r = q.r;
+    const int mdt = mt.mdt, gdt = mt.gdt;
+    const int64_t c_lo = (int64_t)(u - p.starts[f]) * Cf::SLAB;
+    const int64_t c_hi = min(q.n, c_lo + Cf::SLAB);
+    const bool on = q.cond && p.fsc[4 * f] > 0.0 && p.fsc[4 * f + 1] > 0.0;
+    const float inv_mc = on ? (float)((double)q.n / p.fsc[4 * f]) : 0.f;
+
+    if constexpr (Cf::MMA) {
+      constexpr int NB = Cf::NB, NUB = Cf::NUB;
+      const int g = lane >> 2, t = lane & 3;
+      double s1[NUB][2], s2[NUB][2];
+      float er[NB];
+#pragma unroll
+      for (int b = 0; b < NUB; ++b) s1[b][0] = s1[b][1] = s2[b][0] = s2[b][1] = 0.0;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) er[b] = 0.f;
+      const bool quad = !q.tall && q.vec;
+      // lane (g, t) holds rows g + 8 blk at long-side columns col(e), e = 0..3:
+      // wide c + 4t + e (one 4-vector per row), tall c + t + 4e
+      auto col_of = [&](int64_t c, int e) -> int64_t { return q.tall ? c + t + 4 * e : c + 4 * t + e; };
+      auto load = [&](Frag& fr, int64_t c) {
+#pragma unroll
+        for (int blk = 0; blk < NB; ++blk) {
+          const int row = g + 8 * blk;
+          if (quad) {
+            if (row < r && c + 4 * t < c_hi) {
+              ld4(mt.M, q.off(row, c + 4 * t), mdt, fr.m[blk]);
+              ld4(mt.G, q.off(row, c + 4 * t), gdt, fr.g[blk]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) fr.m[blk][e] = fr.g[blk][e] = 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int64_t col = col_of(c, e);
+              const bool ok = row < r && col < c_hi;
+              const int64_t o = ok ? q.off(row, col) : 0;
+              fr.m[blk][e] = ok ? ld_elem(mt.M, o, mdt) : 0.f;
+              fr.g[blk][e] = ok ? ld_elem(mt.G, o, gdt) : 0.f;
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int64_t col = col_of(c, e);
+          fr.ec[e] = (on && col < c_hi) ? q.e_c[col] : 0.f;
+        }
+      };
+      auto step = [&](Frag& fr, int64_t c) {
+        // momentum (invalid positions hold zeros and stay zero)
+        double bx[NB][4];
+#pragma unroll
+        for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float m = momentum_value(mu, fr.m[blk][e], fr.g[blk][e], mdt);
+            fr.m[blk][e] = m;
+            bx[blk][e] = p.nesterov ? fma((double)mu, (double)m, (double)fr.g[blk][e]) : (double)m;
+            er[blk] = fmaf(m, m, er[blk]);
+          }
+#pragma unroll
+        for (int blk = 0; blk < NB; ++blk) {
+          const int row = g + 8 * blk;
+          if (quad) {
+            if (row < r && c + 4 * t < c_hi) st4(mt.M, q.off(row, c + 4 * t), mdt, fr.m[blk]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int64_t col = col_of(c, e);
+              if (row < r && col < c_hi) st_elem(mt.M, q.off(row, col), mdt, fr.m[blk][e]);
+            }
+          }
+        }
+        // Gram partials: the DMMA's k slot t is column col(e)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const double w =
+              on ? (col_of(c, e) < c_hi ? (double)col_weight(fr.ec[e], inv_mc, eps) : 0.0) : 1.0;
+          double xw[NB], xw2[NB];
+#pragma unroll
+          for (int blk = 0; blk < NB; ++blk) {
+            xw[blk] = w * bx[blk][e];
+            xw2[blk] = w * xw[blk];
+          }
+          int ub = 0;
+#pragma unroll
+          for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+            for (int bj = bi; bj < NB; ++bj, ++ub) {
+              dmma(s1[ub][0], s1[ub][1], bx[bi][e], xw[bj]);
+              if (on) dmma(s2[ub][0], s2[ub][1], bx[bi][e], xw2[bj]);
+            }
+        }
+      };
+      stream_positions<Cf::DB, Frag>(c_lo + 16 * warp, 16 * TW, c_hi, load, step);
+      // block ub's entry (g, 2t + h) -> slot ub * 64 + g * 8 + 2t + h
+#pragma unroll
+      for (int ub = 0; ub < NUB; ++ub)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          red_s[warp][0][ub * 64 + g * 8 + 2 * t + h] = s1[ub][h];
+          red_s[warp][1][ub * 64 + g * 8 + 2 * t + h] = s2[ub][h];
+        }
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+        float e = er[blk];
+        e += __shfl_xor_sync(0xffffffffu, e, 1);
+        e += __shfl_xor_sync(0xffffffffu, e, 2);
+        if (t == 0) red_e[warp][g + 8 * blk] = e;
+      }
+    } else {
+      // RP == r <= 4: lane owns long-side columns c .. c + 3
+      double s1[RP][RP], s2[RP][RP];
+      float er[RP];
+#pragma unroll
+      for (int i = 0; i < RP; ++i) {
+        er[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < RP; ++k) s1[i][k] = s2[i][k] = 0.0;
+      }
+      auto load = [&](Frag& fr, int64_t c) {
+        const bool full = q.vec && c + 4 <= c_hi;
+        if (full && q.tall) {
+          float fm[4 * RP], fg[4 * RP];  // four long-side columns, r each
+#pragma unroll
+          for (int s = 0; s < RP; ++s) {
+            ld4(mt.M, c * RP + 4 * s, mdt, &fm[4 * s]);
+            ld4(mt.G, c * RP + 4 * s, gdt, &fg[4 * s]);
+          }
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              fr.m[i][e] = fm[e * RP + i];
+              fr.g[i][e] = fg[e * RP + i];
+            }
+        } else if (full) {
+#pragma unroll
+          for (int i = 0; i < RP; ++i) {
+            ld4(mt.M, q.off(i, c), mdt, fr.m[i]);
+            ld4(mt.G, q.off(i, c), gdt, fr.g[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const bool ok = c + e < c_hi;
+              const int64_t o = ok ? q.off(i, c + e) : 0;
+              fr.m[i][e] = ok ? ld_elem(mt.M, o, mdt) : 0.f;
+              fr.g[i][e] = ok ? ld_elem(mt.G, o, gdt) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) fr.ec[e] = (on && c + e < c_hi) ? q.e_c[c + e] : 0.f;
+      };
+      auto step = [&](Frag& fr, int64_t c) {
+        const bool full = q.vec && c + 4 <= c_hi;
+        double bx[RP][4];
+#pragma unroll
+        for (int i = 0; i < RP; ++i)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float m = momentum_value(mu, fr.m[i][e], fr.g[i][e], mdt);
+            fr.m[i][e] = m;
+            bx[i][e] = p.nesterov ? fma((double)mu, (double)m, (double)fr.g[i][e]) : (double)m;
+            er[i] = fmaf(m, m, er[i]);
+          }
+        if (full && q.tall) {
+          float fm[4 * RP];
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) fm[e * RP + i] = fr.m[i][e];
+#pragma unroll
+          for (int s = 0; s < RP; ++s) st4(mt.M, c * RP + 4 * s, mdt, &fm[4 * s]);
+        } else if (full) {
+#pragma unroll
+          for (int i = 0; i < RP; ++i) st4(mt.M, q.off(i, c), mdt, fr.m[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (c + e < c_hi) st_elem(mt.M, q.off(i, c + e), mdt, fr.m[i][e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const double w = on ? (c + e < c_hi ? (double)col_weight(fr.ec[e], inv_mc, eps) : 0.0) : 1.0;
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int k = i; k < RP; ++k) {
+              const double xk = w * bx[k][e];
+              s1[i][k] = fma(bx[i][e], xk, s1[i][k]);
+              if (on) s2[i][k] = fma(bx[i][e], w * xk, s2[i][k]);
+            }
+        }
+      };
+      stream_positions<Cf::DB, Frag>(c_lo + 4 * (lane + 32 * warp), 4 * TT, c_hi, load, step);
+#pragma unroll
+      for (int i = 0; i < RP; ++i) {
+#pragma unroll
+        for (int k = i; k < RP; ++k) {
+          const double a = warp_sum_d(s1[i][k]), b = warp_sum_d(s2[i][k]);
+          if (lane == 0) {
+            red_s[warp][0][i * RP + k] = red_s[warp][0][k * RP + i] = a;
+            red_s[warp][1][i * RP + k] = red_s[warp][1][k * RP + i] = b;
+          }
+        }
+        const float e = warp_sum(er[i]);
+        if (lane == 0) red_e[warp][i] = e;
+      }
+    }
+    __syncthreads();
+    double* dst = p.part + (size_t)u * 2 * Cf::PART;
+    for (int i = tid; i < 2 * Cf::PART; i += TT) {
+      double s = 0.0;
+#pragma unroll
+      for (int w = 0; w < TW; ++w) s += (&red_s[w][0][0])[i];
+      dst[i] = s;
+    }
+    if (q.cond)
+      for (int i = tid; i < RP; i += TT) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < TW; ++w) s += red_e[w][i];
+        p.rpart[(size_t)u * RP + i] = s;
+      }
+  }
+}
+
+// ===========================================================================
+// thin_iterate: one CTA per factor
+// ===========================================================================
+template <int RP>
+struct IterSmem {
+  double G[RP][TCfg<RP>::SLD], H[RP][TCfg<RP>::SLD], P[RP][TCfg<RP>::SLD],
+      A[RP][TCfg<RP>::SLD], Q[RP][TCfg<RP>::SLD], S[RP][TCfg<RP>::SLD];
+  double R[RP];
   double red[32];
-  double sc[8];  // [0] slice sum of previous long-side energies, [1] factor, [4] ||X_0||^2
 };
-
-// D (8x8, two values per lane) += A (8x4) * B (4x8) in fp64.
-// Lane l = 4g + t holds A[g][t], B[t][g], D[g][2t], D[g][2t+1].
-__device__ __forceinline__ void dmma(double& d0, double& d1, double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-               : "+d"(d0), "+d"(d1)
-               : "d"(a), "d"(b));
-}
-
-// (relative energy + eps)^(-1/4) as 1 / sqrt(sqrt(.)).
-__device__ __forceinline__ float cond_value(float rel_plus_eps) {
-  return rsqrtf(sqrtf(rel_plus_eps));
-}
 
 // C = A * B for RP x RP fp64 matrices in shared memory (padded rows).
 template <int RP>
-__device__ __forceinline__ void mm(double (*C)[Cfg<RP>::SLD], double (*A)[Cfg<RP>::SLD],
-                                   double (*B)[Cfg<RP>::SLD]) {
-  if constexpr (Cfg<RP>::MMA) {
-    constexpr int NBD = Cfg<RP>::NBD;
+__device__ __forceinline__ void mm(double (*C)[TCfg<RP>::SLD], double (*A)[TCfg<RP>::SLD],
+                                   double (*B)[TCfg<RP>::SLD]) {
+  if constexpr (TCfg<RP>::MMA) {
+    constexpr int NB = TCfg<RP>::NB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    for (int blk = warp; blk < NBD * NBD; blk += WARPS) {
-      const int rb = blk / NBD, cb = blk % NBD;
+    for (int blk = warp; blk < NB * NB; blk += TW) {
+      const int rb = blk / NB, cb = blk % NB;
       double d0 = 0.0, d1 = 0.0;
 #pragma unroll
       for (int kb = 0; kb < RP / 4; ++kb)
@@ -109,7 +391,7 @@ __device__ __forceinline__ void mm(double (*C)[Cfg<RP>::SLD], double (*A)[Cfg<RP
       C[rb * 8 + g][cb * 8 + 2 * t + 1] = d1;
     }
   } else {
-    for (int idx = threadIdx.x; idx < RP * RP; idx += THREADS) {
+    for (int idx = threadIdx.x; idx < RP * RP; idx += TT) {
       const int i = idx / RP, j = idx % RP;
       double s = 0.0;
 #pragma unroll
@@ -120,506 +402,564 @@ __device__ __forceinline__ void mm(double (*C)[Cfg<RP>::SLD], double (*A)[Cfg<RP
   __syncthreads();
 }
 
-// 4 consecutive elements (aligned) <-> floats.
-__device__ __forceinline__ void ld4(const void* p, int64_t i, int dt, float v[4]) {
-  if (dt == DT_BF16) {
-    const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p) + i);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-    const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-  } else {
-    const float4 f = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + i);
-    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-  }
-}
-
-__device__ __forceinline__ void st4(void* p, int64_t i, int dt, const float v[4]) {
-  if (dt == DT_BF16) {
-    uint2 u;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-    h[0] = __floats2bfloat162_rn(v[0], v[1]);
-    h[1] = __floats2bfloat162_rn(v[2], v[3]);
-    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p) + i) = u;
-  } else {
-    *reinterpret_cast<float4*>(reinterpret_cast<float*>(p) + i) = make_float4(v[0], v[1], v[2], v[3]);
-  }
-}
-
 template <int RP>
-__global__ void __launch_bounds__(THREADS, 2) thin_step(const __grid_constant__ ThinParams p) {
-  using Cf = Cfg<RP>;
-  constexpr int CH = Cf::CH;
+__global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinParams p) {
+  using Cf = TCfg<RP>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  ThinSmem<RP>& s = *reinterpret_cast<ThinSmem<RP>*>(smem_raw);
-  cg::cluster_group cluster = cg::this_cluster();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cs = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
+  IterSmem<RP>& s = *reinterpret_cast<IterSmem<RP>*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int f = blockIdx.x;
+  const ThinMat mt = p.mats[f];  // by value: stores cannot alias it
+  const Geo q = geometry(mt, p.conditioned);
+  const int r = q.r;
+  const int u0 = p.starts[f], nu = p.starts[f + 1] - p.starts[f];
 
-  const ThinMat& mt = p.mats[blockIdx.x / cs];
-  const bool tall = mt.rows > mt.cols;
-  const int r = (int)(tall ? mt.cols : mt.rows);
-  const int64_t n = tall ? mt.rows : mt.cols;
-  const int64_t nck = (n + CH - 1) / CH;  // chunks of the factor
-  const int64_t k_lo = (nck * rank / cs) * CH;
-  const int64_t k_hi = min(n, (nck * (rank + 1) / cs) * CH);
-  float* e_r = tall ? mt.e_col : mt.e_row;  // energies along the short side
-  float* e_c = tall ? mt.e_row : mt.e_col;  // energies along the long side
-  const bool cond = p.conditioned && e_r != nullptr && e_c != nullptr;
-  // Vector path: each 4-vector lies in one row (wide) or the chunk is one
-  // contiguous run (tall with RP == r).
-  // (tall r = 2 vectors span two columns: the long side must be even)
-  const bool vec = mt.vec && (tall ? (RP == r && (RP >= 4 || n % 2 == 0)) : (n % VEC) == 0);
-
-  // element (i, k) of X (short side i) in storage
-  auto off = [&](int i, int64_t k) -> int64_t { return tall ? k * r + i : (int64_t)i * n + k; };
-  // vector v of a chunk -> first element's (row, column); tall vectors run
-  // along the flat (column-major in X) order
-  auto vcoord = [&](int v, int& i, int& kk) {
-    if (tall) {
-      kk = (v * VEC) / RP;
-      i = (v * VEC) % RP;
-    } else {
-      i = v / (CH / VEC);
-      kk = (v % (CH / VEC)) * VEC;
-    }
-  };
-  // element e (0..3) of a vector starting at (i, kk)
-  auto ecoord = [&](int i, int kk, int e, int& ie, int& ke) {
-    if (tall) {
-      ie = (i + e) % RP;
-      ke = kk + (i + e) / RP;
-    } else {
-      ie = i;
-      ke = kk + e;
-    }
-  };
-
-  // ---- means of the previous energies.  Every read of e_r / e_c for them
-  //      happens before the first cluster barrier; in-place writes come later.
-  double sr = 0.0, sl = 0.0;
-  if (cond) {
-    for (int i = tid; i < r; i += THREADS) sr += (double)e_r[i];
-    for (int64_t k = k_lo + tid; k < k_hi; k += THREADS) sl += (double)e_c[k];
-  }
-  sr = block_sum_d(sr, s.red);
-  sl = block_sum_d(sl, s.red);
-  if (tid == 0) s.sc[0] = sl;
-  cluster.sync();
-  double sc_tot = 0.0;
-  for (int q = 0; q < cs; ++q) sc_tot += *cluster.map_shared_rank(&s.sc[0], q);
-  const bool on = cond && sr > 0.0 && sc_tot > 0.0;
-  const float inv_mr = on ? (float)((double)r / sr) : 0.f;
-  const float inv_mc = on ? (float)((double)n / sc_tot) : 0.f;
-  if (tid < RP) {
-    s.Rv[tid] = tid < r ? (on ? cond_value(e_r[tid] * inv_mr + p.eps) : 1.f) : 0.f;
-    s.rowp[tid] = 0.f;
-  }
-
-  // previous long-side energies of a chunk ride along with its loads
-  constexpr int ECP = (CH + THREADS - 1) / THREADS;
-  float ecv[ECP];
-  auto load_energies = [&](int64_t k0) {
-#pragma unroll
-    for (int q = 0; q < ECP; ++q) {
-      const int kk = tid + THREADS * q;
-      ecv[q] = (on && kk < CH && k0 + kk < k_hi) ? e_c[k0 + kk] : 0.f;
-    }
-  };
-  auto conditioning_of_chunk = [&](int cw) {
-#pragma unroll
-    for (int q = 0; q < ECP; ++q) {
-      const int kk = tid + THREADS * q;
-      if (kk < CH) s.Cc[kk] = kk < cw ? (on ? cond_value(ecv[q] * inv_mc + p.eps) : 1.f) : 0.f;
-    }
-  };
-  // loads of one chunk: a = first operand (G in pass 1, M in pass 2), b = second
-  // (M in pass 1, W in pass 2)
-  float av[NVEC][VEC], bv[NVEC][VEC];
-  // second operand optional (with_b = false loads only pa)
-  auto load_chunk_pair = [&](int64_t k0, const void* pa, int dta, const void* pb, int dtb,
-                             float (&oa)[NVEC][VEC], float (&ob)[NVEC][VEC], bool with_b) {
-    const int cw = (int)min((int64_t)CH, k_hi - k0);
-#pragma unroll
-    for (int q = 0; q < NVEC; ++q) {
-      int i, kk;
-      vcoord(tid + THREADS * q, i, kk);
-      if (vec) {
-        const bool ok = k0 < k_hi && i < r && kk < cw;  // vectors never straddle cw
-        if (ok) {
-          ld4(pa, off(i, k0 + kk), dta, oa[q]);
-          if (with_b) ld4(pb, off(i, k0 + kk), dtb, ob[q]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < VEC; ++e) oa[q][e] = ob[q][e] = 0.f;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          int ie, ke;
-          ecoord(i, kk, e, ie, ke);
-          const bool ok = k0 < k_hi && ie < r && ke < cw;
-          const int64_t o = ok ? off(ie, k0 + ke) : 0;
-          oa[q][e] = ok ? ld_elem(pa, o, dta) : 0.f;
-          ob[q][e] = (ok && with_b) ? ld_elem(pb, o, dtb) : 0.f;
-        }
-      }
-    }
-  };
-
-  auto load_chunk = [&](int64_t k0, const void* pa, int dta, const void* pb, int dtb) {
-    load_energies(k0);
-    load_chunk_pair(k0, pa, dta, pb, dtb, av, bv, true);
-  };
-
-  // ---- pass 1 ----------------------------------------------------------------
-  // MMA path: warps 0..3 accumulate A_0, warps 4..7 accumulate H, each over a
-  // quarter of the chunk's 4-column steps; fragments are 8x8 upper blocks.
-  double acc[Cf::MMA ? Cf::NUB : 1][2];
-  // SIMT path (RP <= 4): thread t accumulates pair (t % (RP*RP)) over columns
-  double sacc_g = 0.0, sacc_h = 0.0;
-#pragma unroll
-  for (int b = 0; b < (Cf::MMA ? Cf::NUB : 1); ++b) acc[b][0] = acc[b][1] = 0.0;
-
-  load_chunk(k_lo, mt.G, mt.gdt, mt.M, mt.mdt);
-  for (int64_t k0 = k_lo; k0 < k_hi; k0 += CH) {
-    const int cw = (int)min((int64_t)CH, k_hi - k0);
-    conditioning_of_chunk(cw);
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < NVEC; ++q) {
-      int i, kk;
-      vcoord(tid + THREADS * q, i, kk);
-      float m4[VEC];
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        int ie, ke;
-        ecoord(i, kk, e, ie, ke);
-        const bool ok = ie < r && ke < cw;
-        m4[e] = ok ? momentum_value(p.mu, bv[q][e], av[q][e], mt.mdt) : 0.f;
-        s.u.pass.ms[ie][ke] = m4[e];
-        // orthogonaliser input: M_t, or B_t = G + mu M_t under Nesterov
-        const double b = p.nesterov ? fma((double)p.mu, (double)m4[e], (double)av[q][e])
-                                    : (double)m4[e];
-        s.u.pass.xs[ie][ke] = (double)s.Rv[ie] * b * (double)s.Cc[ke];
-        if (!vec && ok) st_elem(mt.M, off(ie, k0 + ke), mt.mdt, m4[e]);
-      }
-      if (vec && i < r && kk < cw) st4(mt.M, off(i, k0 + kk), mt.mdt, m4);
-    }
-    load_chunk(k0 + CH, mt.G, mt.gdt, mt.M, mt.mdt);  // in flight during the Gram
-    __syncthreads();
-    if (cond) {  // row energies: THREADS / RP threads per row
-      constexpr int TPR = THREADS / RP;
-      const int i = tid / TPR;
-      float e = 0.f;
-      if (i < r)
-        for (int kk = tid % TPR; kk < cw; kk += TPR) e = fmaf(s.u.pass.ms[i][kk], s.u.pass.ms[i][kk], e);
-      s.red32[tid] = e;
-    }
+  // S_1, S_2: slab partials in slab order; lower 8x8 blocks mirror upper ones
+  for (int idx = tid; idx < RP * RP; idx += TT) {
+    const int i = idx / RP, j = idx % RP;
+    int src;
     if constexpr (Cf::MMA) {
-      const int g = lane >> 2, t = lane & 3;
-      const bool hpart = warp >= 4;
-      for (int ks = warp & 3; ks < CH / 4; ks += 4) {
-        const int kk = ks * 4 + t;
-        const double c2 = hpart ? (double)s.Cc[kk] * (double)s.Cc[kk] : 1.0;
-        double f[Cf::NBD];
-#pragma unroll
-        for (int b = 0; b < Cf::NBD; ++b) f[b] = s.u.pass.xs[b * 8 + g][kk];
-        int ub = 0;
-#pragma unroll
-        for (int bi = 0; bi < Cf::NBD; ++bi)
-#pragma unroll
-          for (int bj = bi; bj < Cf::NBD; ++bj, ++ub) dmma(acc[ub][0], acc[ub][1], f[bi], f[bj] * c2);
-      }
+      constexpr int NB = Cf::NB;
+      const int bi = i >> 3, bj = j >> 3;
+      const int lo = bi <= bj ? bi : bj, hi = bi <= bj ? bj : bi;
+      const int ub = lo * NB - lo * (lo - 1) / 2 + (hi - lo);
+      src = ub * 64 + (bi <= bj ? (i & 7) * 8 + (j & 7) : (j & 7) * 8 + (i & 7));
     } else {
-      const int pr = tid % (RP * RP), i = pr / RP, j = pr % RP;
-      for (int kk = tid / (RP * RP); kk < cw; kk += THREADS / (RP * RP)) {
-        const double x = s.u.pass.xs[i][kk] * s.u.pass.xs[j][kk];
-        sacc_g += x;
-        sacc_h = fma(x, (double)s.Cc[kk] * (double)s.Cc[kk], sacc_h);
-      }
+      src = idx;
     }
-    __syncthreads();
-    if (cond && tid < r) {
-      constexpr int TPR = THREADS / RP;
-      float e = 0.f;
-      for (int q = 0; q < TPR; ++q) e += s.red32[tid * TPR + q];
-      s.rowp[tid] += e;
+    double g1 = 0.0, g2 = 0.0;
+    for (int v = 0; v < nu; ++v) {
+      const double* pp = p.part + (size_t)(u0 + v) * 2 * Cf::PART;
+      g1 += pp[src];
+      g2 += pp[Cf::PART + src];
     }
+    s.G[i][j] = g1;
+    s.H[i][j] = g2;
+  }
+  // R from the previous short-side energies (read before they are replaced)
+  const double sc = p.fsc[4 * f], sr = p.fsc[4 * f + 1];
+  const bool on = q.cond && sr > 0.0 && sc > 0.0;
+  if (tid < RP) {
+    double rv = tid < r ? 1.0 : 0.0;
+    if (on && tid < r) rv = 1.0 / sqrt(sqrt((double)q.e_r[tid] * ((double)r / sr) + (double)p.eps));
+    s.R[tid] = rv;
   }
   __syncthreads();
-
-  // ---- CTA-level reduction of the Gram partials (fixed order) -----------------
-  if constexpr (Cf::MMA) {
-    const int g = lane >> 2, t = lane & 3;
-    double* dst = s.u.part + warp * RP * RP;  // warps 0..3: A_0, warps 4..7: H
-    int ub = 0;
-#pragma unroll
-    for (int bi = 0; bi < Cf::NBD; ++bi)
-#pragma unroll
-      for (int bj = bi; bj < Cf::NBD; ++bj, ++ub) {
-        dst[(bi * 8 + g) * RP + bj * 8 + 2 * t] = acc[ub][0];
-        dst[(bi * 8 + g) * RP + bj * 8 + 2 * t + 1] = acc[ub][1];
-      }
-    __syncthreads();
-    for (int idx = tid; idx < RP * RP; idx += THREADS) {
+  if (q.cond && tid < r) {
+    float e = 0.f;
+    for (int v = 0; v < nu; ++v) e += p.rpart[(size_t)(u0 + v) * RP + tid];
+    q.e_r[tid] = e;
+  }
+  // A_0 = R S_1 R, H = R S_2 R; ||X_0||^2 = tr A_0
+  double tr = 0.0;
+  for (int idx = tid; idx < RP * RP; idx += TT) {
+    const int i = idx / RP, j = idx % RP;
+    const double rr = s.R[i] * s.R[j];
+    s.G[i][j] *= rr;
+    s.H[i][j] *= rr;
+    if (i == j) tr += s.G[i][j];
+  }
+  const double s2 = block_sum_d(tr, s.red);
+  const bool finite = isfinite(s2);
+  const bool valid = finite && s2 >= NORM2_FLOOR;  // else the update is zero
+  const double inv_s2 = valid ? 1.0 / s2 : 0.0;
+  for (int idx = tid; idx < RP * RP; idx += TT) {
+    const int i = idx / RP, j = idx % RP;
+    s.A[i][j] = valid ? s.G[i][j] * inv_s2 : 0.0;
+    s.P[i][j] = i == j ? 1.0 : 0.0;
+  }
+  __syncthreads();
+  const double a = p.a, b = p.b, c = p.c;
+  for (int it = 0; it < p.ns_steps; ++it) {
+    mm<RP>(s.Q, s.A, s.A);  // Q = A A
+    for (int idx = tid; idx < RP * RP; idx += TT) {
       const int i = idx / RP, j = idx % RP;
-      const int src = (i / 8 <= j / 8) ? idx : j * RP + i;  // lower blocks mirror upper ones
-      double gs = 0.0, hs = 0.0;
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        gs += s.u.part[w * RP * RP + src];
-        hs += s.u.part[(w + 4) * RP * RP + src];
-      }
-      s.Gc[idx] = gs;
-      s.Hc[idx] = hs;
+      s.Q[i][j] = c * s.Q[i][j] + b * s.A[i][j] + (i == j ? a : 0.0);
     }
-  } else {
-    s.u.part[tid] = sacc_g;
-    s.u.part[THREADS + tid] = sacc_h;
     __syncthreads();
-    for (int idx = tid; idx < RP * RP; idx += THREADS) {
-      double gs = 0.0, hs = 0.0;
-      for (int q = idx; q < THREADS; q += RP * RP) {
-        gs += s.u.part[q];
-        hs += s.u.part[THREADS + q];
-      }
-      s.Gc[idx] = gs;
-      s.Hc[idx] = hs;
-    }
+    mm<RP>(s.S, s.Q, s.P);  // P <- Q P
+    for (int idx = tid; idx < RP * RP; idx += TT) s.P[idx / RP][idx % RP] = s.S[idx / RP][idx % RP];
+    __syncthreads();
+    mm<RP>(s.S, s.Q, s.A);  // A <- Q A Q
+    mm<RP>(s.A, s.S, s.Q);
   }
-  cluster.sync();  // every CTA's Gc / Hc / rowp are final
-
-  // ---- rank 0: cluster reduction and the r x r iteration -----------------------
-  if (rank == 0) {
-    for (int idx = tid; idx < RP * RP; idx += THREADS) {
-      double gv[8], hv[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        gv[q] = q < cs ? cluster.map_shared_rank(&s.Gc[0], q)[idx] : 0.0;
-        hv[q] = q < cs ? cluster.map_shared_rank(&s.Hc[0], q)[idx] : 0.0;
-      }
-      double g = 0.0, h = 0.0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        g += gv[q];
-        h += hv[q];
-      }
-      s.u.it.G[idx / RP][idx % RP] = g;
-      s.u.it.H[idx / RP][idx % RP] = h;
-    }
-    if (cond && tid < r) {
-      float e = 0.f;
-      for (int q = 0; q < cs; ++q) e += cluster.map_shared_rank(&s.rowp[0], q)[tid];
-      e_r[tid] = e;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      double tr = 0.0;
-      for (int i = 0; i < r; ++i) tr += s.u.it.G[i][i];
-      s.sc[4] = tr;
-    }
-    __syncthreads();
-    const double s2 = s.sc[4];
-    const bool finite = isfinite(s2);
-    const bool valid = finite && s2 >= NORM2_FLOOR;  // else the update is zero
-    const double inv_s2 = valid ? 1.0 / s2 : 0.0;
-    for (int idx = tid; idx < RP * RP; idx += THREADS) {
-      const int i = idx / RP, j = idx % RP;
-      s.u.it.A[i][j] = valid ? s.u.it.G[i][j] * inv_s2 : 0.0;
-      s.u.it.P[i][j] = i == j ? 1.0 : 0.0;
-    }
-    __syncthreads();
-    const double a = p.a, b = p.b, c = p.c;
-    for (int it = 0; it < p.ns_steps; ++it) {
-      mm<RP>(s.u.it.Q, s.u.it.A, s.u.it.A);  // Q = A A
-      for (int idx = tid; idx < RP * RP; idx += THREADS) {
-        const int i = idx / RP, j = idx % RP;
-        s.u.it.Q[i][j] = c * s.u.it.Q[i][j] + b * s.u.it.A[i][j] + (i == j ? a : 0.0);
-      }
-      __syncthreads();
-      mm<RP>(s.u.it.S, s.u.it.Q, s.u.it.P);  // P <- Q P
-      for (int idx = tid; idx < RP * RP; idx += THREADS)
-        s.u.it.P[idx / RP][idx % RP] = s.u.it.S[idx / RP][idx % RP];
-      __syncthreads();
-      mm<RP>(s.u.it.S, s.u.it.Q, s.u.it.A);  // A <- Q A Q
-      mm<RP>(s.u.it.A, s.u.it.S, s.u.it.Q);
-    }
-    // ||X_5||^2 s^2 = tr(P A_0 P^T); ||R X_5 C||^2 s^2 = sum_i R_i^2 (P H P^T)_ii
-    mm<RP>(s.u.it.S, s.u.it.P, s.u.it.G);
-    double nx = 0.0;
-    for (int idx = tid; idx < RP * RP; idx += THREADS)
-      nx += s.u.it.S[idx / RP][idx % RP] * s.u.it.P[idx / RP][idx % RP];
-    nx = block_sum_d(nx, s.red);
-    mm<RP>(s.u.it.Q, s.u.it.P, s.u.it.H);
-    double ny = 0.0;
-    for (int idx = tid; idx < RP * RP; idx += THREADS) {
-      const int i = idx / RP;
-      ny += (double)s.Rv[i] * s.Rv[i] * s.u.it.Q[i][idx % RP] * s.u.it.P[i][idx % RP];
-    }
-    ny = block_sum_d(ny, s.red);
-    double factor = 0.0;
-    if (valid) {
-      factor = (double)mt.kappa / sqrt(s2);
-      if (on) factor = ny > 0.0 ? factor * sqrt(nx / ny) : 0.0;
-    }
-    if (!finite && tid == 0) raise_status(p.status, ST_NONFINITE);
-    for (int idx = tid; idx < RP * RP; idx += THREADS)
-      s.T[idx / RP][idx % RP] = factor * s.u.it.P[idx / RP][idx % RP];
-    if (tid == 0) s.sc[1] = factor;
+  // ||X_5||^2 s^2 = tr(P A_0 P^T); ||R X_5 C||^2 s^2 = sum_i R_i^2 (P H P^T)_ii
+  mm<RP>(s.S, s.P, s.G);
+  double nx = 0.0;
+  for (int idx = tid; idx < RP * RP; idx += TT) nx += s.S[idx / RP][idx % RP] * s.P[idx / RP][idx % RP];
+  nx = block_sum_d(nx, s.red);
+  mm<RP>(s.Q, s.P, s.H);
+  double ny = 0.0;
+  for (int idx = tid; idx < RP * RP; idx += TT) {
+    const int i = idx / RP;
+    ny += s.R[i] * s.R[i] * s.Q[i][idx % RP] * s.P[i][idx % RP];
   }
-  cluster.sync();  // rank 0's T is final
-  if (rank != 0) {
-    const double* T0 = &cluster.map_shared_rank(&s.T[0][0], 0)[0];
-    for (int idx = tid; idx < RP * Cf::SLD; idx += THREADS) (&s.T[0][0])[idx] = T0[idx];
-    if (tid == 0) s.sc[1] = *cluster.map_shared_rank(&s.sc[1], 0);
+  ny = block_sum_d(ny, s.red);
+  double factor = 0.0;
+  if (valid) {
+    factor = (double)mt.kappa / sqrt(s2);
+    if (on) factor = ny > 0.0 ? factor * sqrt(nx / ny) : 0.0;
   }
-  cluster.sync();  // no CTA reads another CTA's shared memory after this point
-  const bool zero_update = s.sc[1] == 0.0;
-
-  // ---- pass 2 ----------------------------------------------------------------
-  // Under Nesterov, X_0 needs G again: cv holds a chunk's G.
-  float cv[NVEC][VEC];
-  auto load_grad = [&](int64_t k0) {
-    if (!p.nesterov) return;
-    load_chunk_pair(k0, mt.G, mt.gdt, mt.G, mt.gdt, cv, cv, false);
-  };
-  load_grad(k_lo);
-  load_chunk(k_lo, mt.M, mt.mdt, mt.W, mt.wdt);
-  for (int64_t k0 = k_lo; k0 < k_hi; k0 += CH) {
-    const int cw = (int)min((int64_t)CH, k_hi - k0);
-    conditioning_of_chunk(cw);
-    __syncthreads();
-    float wcur[NVEC][VEC];
-#pragma unroll
-    for (int q = 0; q < NVEC; ++q) {
-      int i, kk;
-      vcoord(tid + THREADS * q, i, kk);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        int ie, ke;
-        ecoord(i, kk, e, ie, ke);
-        s.u.pass.ms[ie][ke] = av[q][e];
-        const double b = p.nesterov ? fma((double)p.mu, (double)av[q][e], (double)cv[q][e])
-                                    : (double)av[q][e];
-        s.u.pass.xs[ie][ke] = (double)s.Rv[ie] * b * (double)s.Cc[ke];
-        wcur[q][e] = bv[q][e];
-      }
-    }
-    load_grad(k0 + CH);
-    load_chunk(k0 + CH, mt.M, mt.mdt, mt.W, mt.wdt);  // in flight during the apply
-    __syncthreads();
-    if (cond) {
-      for (int kk = tid; kk < cw; kk += THREADS) {
-        float e = 0.f;
-        for (int i = 0; i < r; ++i) e = fmaf(s.u.pass.ms[i][kk], s.u.pass.ms[i][kk], e);
-        e_c[k0 + kk] = e;
-      }
-    }
-    __syncthreads();
+  if (!finite && tid == 0) raise_status(p.status, ST_NONFINITE);
+  // T = f R P R; for RP >= 8 in MMA fragment order: T(8 bo + l/4, 4 kb + l%4)
+  // at ((bo * KB + kb) * 32 + l)
+  double* T = p.T + (size_t)f * RP * RP;
+  for (int idx = tid; idx < RP * RP; idx += TT) {
+    int i, j;
     if constexpr (Cf::MMA) {
-      // O block (rb, cb) = sum_kb T[rb, kb] X[kb, cb]; one warp per 8 columns
-      const int g = lane >> 2, t = lane & 3;
-      for (int cb = warp; cb < CH / 8; cb += WARPS) {
-        double o[Cf::NBD][2];
-#pragma unroll
-        for (int rb = 0; rb < Cf::NBD; ++rb) o[rb][0] = o[rb][1] = 0.0;
-#pragma unroll
-        for (int kb = 0; kb < RP / 4; ++kb) {
-          const double xb = s.u.pass.xs[kb * 4 + t][cb * 8 + g];
-#pragma unroll
-          for (int rb = 0; rb < Cf::NBD; ++rb)
-            dmma(o[rb][0], o[rb][1], s.T[rb * 8 + g][kb * 4 + t], xb);
-        }
-#pragma unroll
-        for (int rb = 0; rb < Cf::NBD; ++rb)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int i = rb * 8 + g, kk = cb * 8 + 2 * t + h;
-            s.u.pass.ms[i][kk] =
-                zero_update ? 0.f : (float)((double)s.Rv[i] * o[rb][h] * (double)s.Cc[kk]);
-          }
-      }
+      const int l = idx & 31, fr = idx >> 5;
+      const int bo = fr / Cf::KB, kb = fr % Cf::KB;
+      i = 8 * bo + (l >> 2);
+      j = 4 * kb + (l & 3);
     } else {
-      for (int o = tid; o < CH; o += THREADS) {
-        double x[RP];
-#pragma unroll
-        for (int j = 0; j < RP; ++j) x[j] = s.u.pass.xs[j][o];
-#pragma unroll
-        for (int i = 0; i < RP; ++i) {
-          double acc2 = 0.0;
-#pragma unroll
-          for (int j = 0; j < RP; ++j) acc2 = fma(s.T[i][j], x[j], acc2);
-          s.u.pass.ms[i][o] = zero_update ? 0.f : (float)((double)s.Rv[i] * acc2 * (double)s.Cc[o]);
-        }
-      }
+      i = idx / RP;
+      j = idx % RP;
     }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < NVEC; ++q) {
-      int i, kk;
-      vcoord(tid + THREADS * q, i, kk);
-      float u4[VEC], w4[VEC];
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        int ie, ke;
-        ecoord(i, kk, e, ie, ke);
-        u4[e] = s.u.pass.ms[ie][ke];
-        w4[e] = p.decay * wcur[q][e] - p.lr * u4[e];
-        if (!vec && ie < r && ke < cw) {
-          const int64_t o = off(ie, k0 + ke);
-          st_elem(mt.W, o, mt.wdt, w4[e]);
-          if (mt.upd) mt.upd[o] = u4[e];
-        }
-      }
-      if (vec && i < r && kk < cw) {
-        st4(mt.W, off(i, k0 + kk), mt.wdt, w4);
-        if (mt.upd) st4(mt.upd, off(i, k0 + kk), DT_FP32, u4);
-      }
-    }
-    __syncthreads();
+    T[idx] = factor * s.R[i] * s.P[i][j] * s.R[j];
+  }
+  if (tid == 0) {
+    p.fsc[4 * f + 2] = on ? 1.0 : 0.0;
+    p.fsc[4 * f + 3] = factor == 0.0 ? 1.0 : 0.0;
   }
 }
 
+// ===========================================================================
+// thin_apply: O = C^2 T B, W update, long-side energies
+// ===========================================================================
 template <int RP>
-cudaError_t launch_rp(const ThinParams& p, cudaStream_t st) {
-  const int bytes = (int)sizeof(ThinSmem<RP>);
+struct ApplyFrag {
+  static constexpr bool MMA = TCfg<RP>::MMA;
+  static constexpr int MR = MMA ? TCfg<RP>::KB : RP;  // B values per column slot
+  static constexpr int WR = MMA ? TCfg<RP>::NB : RP;
+  float m[MR][4], g[MR][4];
+  float w[WR][MMA ? 2 : 1][4];  // current weights at the lane's output positions
+  float ec[4];                  // previous long-side energies of the four column slots
+};
+
+template <int RP>
+__global__ void __launch_bounds__(TT) thin_apply(const __grid_constant__ ThinParams p) {
+  using Cf = TCfg<RP>;
+  using Frag = ApplyFrag<RP>;
+  __shared__ double Ts[RP * RP];
+  __shared__ int s_unit;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float mu = p.mu, lr = p.lr, decay = p.decay, eps = p.eps;
+  int f_loaded = -1;
+
+  for (int u = next_unit(p.counters + 1, &s_unit); u < p.units;
+       u = next_unit(p.counters + 1, &s_unit)) {
+    const int f = p.unit_f[u];
+    if (f != f_loaded) {  // uniform: every thread saw the same u
+      const double* Tg = p.T + (size_t)f * RP * RP;
+      for (int i = tid; i < RP * RP; i += TT) Ts[i] = Tg[i];
+      f_loaded = f;
+      __syncthreads();
+    }
+    const ThinMat mt = p.mats[f];  // by value: stores cannot alias it
+    const Geo q = geometry(mt, p.conditioned);
+    const int r = q.r;
+    const int64_t c_lo = (int64_t)(u - p.starts[f]) * Cf::SLAB;
+    const int64_t c_hi = min(q.n, c_lo + Cf::SLAB);
+    const bool on = p.fsc[4 * f + 2] != 0.0;
+    const bool zero = p.fsc[4 * f + 3] != 0.0;
+    const float inv_mc = on ? (float)((double)q.n / p.fsc[4 * f]) : 0.f;
+    const int mdt = mt.mdt, gdt = mt.gdt, wdt = mt.wdt;
+    const bool nest = p.nesterov != 0;
+
+    if constexpr (Cf::MMA) {
+      constexpr int NB = Cf::NB, KB = Cf::KB;
+      const int g = lane >> 2, t = lane & 3;
+      const bool quad = !q.tall && q.vec;
+      const bool pair = q.tall && mt.vec && (r & 1) == 0;  // two short-side neighbours aligned
+      // lane (g, t) holds B rows 4 kb + t at long-side column slots col(e):
+      // wide c + 4g + e (4-vectors), tall c + 8e + g.  Wide computes
+      // D = T B (output rows 8 bo + g, columns c + 8t .. c + 8t + 7); tall
+      // computes D = B^T T^T (output rows 8 bo + 2t, +1 at column c + 8e + g).
+      auto col_of = [&](int64_t c, int e) -> int64_t { return q.tall ? c + 8 * e + g : c + 4 * g + e; };
+      auto load = [&](Frag& fr, int64_t c) {
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+          const int row = 4 * kb + t;
+          if (quad) {
+            if (row < r && c + 4 * g < c_hi) {
+              ld4(mt.M, q.off(row, c + 4 * g), mdt, fr.m[kb]);
+              if (nest) {
+                ld4(mt.G, q.off(row, c + 4 * g), gdt, fr.g[kb]);
+              } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) fr.g[kb][e] = 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) fr.m[kb][e] = fr.g[kb][e] = 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int64_t col = col_of(c, e);
+              const bool ok = row < r && col < c_hi;
+              const int64_t o = ok ? q.off(row, col) : 0;
+              fr.m[kb][e] = ok ? ld_elem(mt.M, o, mdt) : 0.f;
+              fr.g[kb][e] = (ok && nest) ? ld_elem(mt.G, o, gdt) : 0.f;
+            }
+          }
+        }
+#pragma unroll
+        for (int bo = 0; bo < NB; ++bo) {
+          if (!q.tall) {
+            const int row = 8 * bo + g;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int64_t col0 = c + 8 * t + 4 * h;
+              if (quad) {
+                if (row < r && col0 < c_hi) {
+                  ld4(mt.W, q.off(row, col0), wdt, fr.w[bo][h]);
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) fr.w[bo][h][e] = 0.f;
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  fr.w[bo][h][e] =
+                      (row < r && col0 + e < c_hi) ? ld_elem(mt.W, q.off(row, col0 + e), wdt) : 0.f;
+              }
+            }
+          } else {
+            const int row0 = 8 * bo + 2 * t;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int64_t col = c + 8 * e + g;
+              if (pair && row0 + 1 < r && col < c_hi) {
+                ld2(mt.W, q.off(row0, col), wdt, fr.w[bo][0][e], fr.w[bo][1][e]);
+              } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                  fr.w[bo][h][e] =
+                      (row0 + h < r && col < c_hi) ? ld_elem(mt.W, q.off(row0 + h, col), wdt) : 0.f;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int64_t col = col_of(c, e);
+          fr.ec[e] = (on && col < c_hi) ? q.e_c[col] : 0.f;
+        }
+      };
+      auto step = [&](Frag& fr, int64_t c) {
+        float ce[4];
+        double x[KB][4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const double w =
+              on ? (col_of(c, e) < c_hi ? (double)col_weight(fr.ec[e], inv_mc, eps) : 0.0) : 1.0;
+          float sq = 0.f;
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb) {
+            const double m = (double)fr.m[kb][e];
+            x[kb][e] = w * (nest ? fma((double)mu, m, (double)fr.g[kb][e]) : m);
+            sq = fmaf(fr.m[kb][e], fr.m[kb][e], sq);
+          }
+          sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+          sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+          ce[e] = sq;
+        }
+        double acc[NB][4][2];
+#pragma unroll
+        for (int bo = 0; bo < NB; ++bo)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[bo][e][0] = acc[bo][e][1] = 0.0;
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+          double tf[NB];
+#pragma unroll
+          for (int bo = 0; bo < NB; ++bo) tf[bo] = Ts[(bo * KB + kb) * 32 + lane];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int bo = 0; bo < NB; ++bo) {
+              if (q.tall)
+                dmma(acc[bo][e][0], acc[bo][e][1], x[kb][e], tf[bo]);
+              else
+                dmma(acc[bo][e][0], acc[bo][e][1], tf[bo], x[kb][e]);
+            }
+        }
+        // W update (and O) at this lane's output positions
+#pragma unroll
+        for (int bo = 0; bo < NB; ++bo) {
+          if (!q.tall) {
+            // acc[bo][e][h] is column c + 8t + 4h + e of row 8 bo + g
+            const int row = 8 * bo + g;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float o4[4], n4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                o4[e] = zero ? 0.f : (float)acc[bo][e][h];
+                n4[e] = decay * fr.w[bo][h][e] - lr * o4[e];
+              }
+              const int64_t col0 = c + 8 * t + 4 * h;
+              if (quad) {
+                if (row < r && col0 < c_hi) {
+                  st4(mt.W, q.off(row, col0), wdt, n4);
+                  if (mt.upd) st4(mt.upd, q.off(row, col0), DT_FP32, o4);
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (row < r && col0 + e < c_hi) {
+                    st_elem(mt.W, q.off(row, col0 + e), wdt, n4[e]);
+                    if (mt.upd) mt.upd[q.off(row, col0 + e)] = o4[e];
+                  }
+              }
+            }
+          } else {
+            // acc[bo][e][h] is row 8 bo + 2t + h of column c + 8e + g
+            const int row0 = 8 * bo + 2 * t;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int64_t col = c + 8 * e + g;
+              float o2[2], n2[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                o2[h] = zero ? 0.f : (float)acc[bo][e][h];
+                n2[h] = decay * fr.w[bo][h][e] - lr * o2[h];
+              }
+              if (pair && row0 + 1 < r && col < c_hi) {
+                st2(mt.W, q.off(row0, col), wdt, n2[0], n2[1]);
+                if (mt.upd) st2(mt.upd, q.off(row0, col), DT_FP32, o2[0], o2[1]);
+              } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                  if (row0 + h < r && col < c_hi) {
+                    st_elem(mt.W, q.off(row0 + h, col), wdt, n2[h]);
+                    if (mt.upd) mt.upd[q.off(row0 + h, col)] = o2[h];
+                  }
+              }
+            }
+          }
+        }
+        if (q.cond) {
+          __syncwarp();  // every lane's read of these columns' previous energies is done
+          if (t == 0)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int64_t col = col_of(c, e);
+              if (col < c_hi) q.e_c[col] = ce[e];
+            }
+        }
+      };
+      stream_positions<Cf::DB, Frag>(c_lo + 32 * warp, 32 * TW, c_hi, load, step);
+    } else {
+      // RP == r <= 4: lane owns long-side columns c .. c + 3
+      auto load = [&](Frag& fr, int64_t c) {
+        const bool full = q.vec && c + 4 <= c_hi;
+        if (full && q.tall) {
+          float fm[4 * RP], fg[4 * RP], fw[4 * RP];
+#pragma unroll
+          for (int s = 0; s < RP; ++s) {
+            ld4(mt.M, c * RP + 4 * s, mdt, &fm[4 * s]);
+            if (nest) ld4(mt.G, c * RP + 4 * s, gdt, &fg[4 * s]);
+            ld4(mt.W, c * RP + 4 * s, wdt, &fw[4 * s]);
+          }
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              fr.m[i][e] = fm[e * RP + i];
+              fr.g[i][e] = nest ? fg[e * RP + i] : 0.f;
+              fr.w[i][0][e] = fw[e * RP + i];
+            }
+        } else if (full) {
+#pragma unroll
+          for (int i = 0; i < RP; ++i) {
+            ld4(mt.M, q.off(i, c), mdt, fr.m[i]);
+            if (nest) {
+              ld4(mt.G, q.off(i, c), gdt, fr.g[i]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) fr.g[i][e] = 0.f;
+            }
+            ld4(mt.W, q.off(i, c), wdt, fr.w[i][0]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const bool ok = c + e < c_hi;
+              const int64_t o = ok ? q.off(i, c + e) : 0;
+              fr.m[i][e] = ok ? ld_elem(mt.M, o, mdt) : 0.f;
+              fr.g[i][e] = (ok && nest) ? ld_elem(mt.G, o, gdt) : 0.f;
+              fr.w[i][0][e] = ok ? ld_elem(mt.W, o, wdt) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) fr.ec[e] = (on && c + e < c_hi) ? q.e_c[c + e] : 0.f;
+      };
+      auto step = [&](Frag& fr, int64_t c) {
+        const bool full = q.vec && c + 4 <= c_hi;
+        float ov[RP][4], wv[RP][4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const double w = on ? (c + e < c_hi ? (double)col_weight(fr.ec[e], inv_mc, eps) : 0.0) : 1.0;
+          double x[RP];
+          float sq = 0.f;
+#pragma unroll
+          for (int k = 0; k < RP; ++k) {
+            const double m = (double)fr.m[k][e];
+            x[k] = w * (nest ? fma((double)mu, m, (double)fr.g[k][e]) : m);
+            sq = fmaf(fr.m[k][e], fr.m[k][e], sq);
+          }
+#pragma unroll
+          for (int i = 0; i < RP; ++i) {
+            double y = 0.0;
+#pragma unroll
+            for (int k = 0; k < RP; ++k) y = fma(Ts[i * RP + k], x[k], y);
+            ov[i][e] = zero ? 0.f : (float)y;
+            wv[i][e] = decay * fr.w[i][0][e] - lr * ov[i][e];
+          }
+          if (q.cond && c + e < c_hi) q.e_c[c + e] = sq;  // this lane read it in load()
+        }
+        if (full && q.tall) {
+          float fw[4 * RP], fo[4 * RP];
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              fw[e * RP + i] = wv[i][e];
+              fo[e * RP + i] = ov[i][e];
+            }
+#pragma unroll
+          for (int s = 0; s < RP; ++s) {
+            st4(mt.W, c * RP + 4 * s, wdt, &fw[4 * s]);
+            if (mt.upd) st4(mt.upd, c * RP + 4 * s, DT_FP32, &fo[4 * s]);
+          }
+        } else if (full) {
+#pragma unroll
+          for (int i = 0; i < RP; ++i) {
+            st4(mt.W, q.off(i, c), wdt, wv[i]);
+            if (mt.upd) st4(mt.upd, q.off(i, c), DT_FP32, ov[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < RP; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (c + e < c_hi) {
+                st_elem(mt.W, q.off(i, c + e), wdt, wv[i][e]);
+                if (mt.upd) mt.upd[q.off(i, c + e)] = ov[i][e];
+              }
+        }
+      };
+      stream_positions<Cf::DB, Frag>(c_lo + 4 * (lane + 32 * warp), 4 * TT, c_hi, load, step);
+    }
+  }
+}
+
+template <typename K>
+int resident_ctas(K kernel, int smem) {
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, TT, smem) != cudaSuccess || occ < 1)
+    occ = 1;
+  return occ;
+}
+
+template <int RP>
+cudaError_t launch_iter_rp(const ThinParams& p, cudaStream_t st) {
+  const int iter_bytes = (int)sizeof(IterSmem<RP>);
   static int configured = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured != dev) {
-    cudaError_t e =
-        cudaFuncSetAttribute(thin_step<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = cudaFuncSetAttribute(thin_iterate<RP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, iter_bytes);
     if (e != cudaSuccess) return e;
     configured = dev;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.count * p.cluster), 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, thin_step<RP>, p);
+  thin_iterate<RP><<<p.count, TT, iter_bytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int RP>
+cudaError_t launch_rp(ThinParams& p, int nsm, cudaStream_t st) {
+  static int configured = -1;
+  static int occ_gram = 1, occ_apply = 1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured != dev) {
+    occ_gram = resident_ctas(thin_gram<RP>, 0);
+    occ_apply = resident_ctas(thin_apply<RP>, 0);
+    configured = dev;
+  }
+  p.grid_gram = std::min(p.units, nsm * occ_gram);
+  p.grid_apply = std::min(p.units, nsm * occ_apply);
+  thin_gram<RP><<<p.grid_gram, TT, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_iter_rp<RP>(p, st);
+  if (e != cudaSuccess) return e;
+  thin_apply<RP><<<p.grid_apply, TT, 0, st>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-// All factors of one launch share the padded short side p.pad (2..32) and
-// the cluster size p.cluster (1..8 CTAs per factor).
-cudaError_t launch_thin(const ThinParams& p, cudaStream_t s) {
-  if (p.count <= 0) return cudaSuccess;
+int thin_part_doubles(int pad) {
+  switch (pad) {
+    case 1: return TCfg<1>::PART;
+    case 2: return TCfg<2>::PART;
+    case 3: return TCfg<3>::PART;
+    case 4: return TCfg<4>::PART;
+    case 8: return TCfg<8>::PART;
+    case 16: return TCfg<16>::PART;
+    default: return TCfg<32>::PART;
+  }
+}
+
+int thin_slab(int pad) {
+  switch (pad) {
+    case 1: return TCfg<1>::SLAB;
+    case 2: return TCfg<2>::SLAB;
+    case 3: return TCfg<3>::SLAB;
+    case 4: return TCfg<4>::SLAB;
+    case 8: return TCfg<8>::SLAB;
+    case 16: return TCfg<16>::SLAB;
+    default: return TCfg<32>::SLAB;
+  }
+}
+
+cudaError_t launch_thin_iterate(const ThinParams& p, cudaStream_t s) {
   switch (p.pad) {
-    case 2: return launch_rp<2>(p, s);
-    case 4: return launch_rp<4>(p, s);
-    case 8: return launch_rp<8>(p, s);
-    case 16: return launch_rp<16>(p, s);
-    default: return launch_rp<32>(p, s);
+    case 1: return launch_iter_rp<1>(p, s);
+    case 2: return launch_iter_rp<2>(p, s);
+    case 3: return launch_iter_rp<3>(p, s);
+    case 4: return launch_iter_rp<4>(p, s);
+    case 8: return launch_iter_rp<8>(p, s);
+    case 16: return launch_iter_rp<16>(p, s);
+    default: return launch_iter_rp<32>(p, s);
+  }
+}
+
+cudaError_t launch_thin_setup(const ThinSetupParams& p, cudaStream_t s) {
+  if (p.count <= 0) return cudaSuccess;
+  thin_setup<<<p.count, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// All factors of one group share the padded short side p.pad (1, 2, 3, 4,
+// 8, 16 or 32); their descriptors are in p.mats (written by thin_setup).
+cudaError_t launch_thin(ThinParams& p, int nsm, cudaStream_t s) {
+  if (p.count <= 0 || p.units <= 0) return cudaSuccess;
+  switch (p.pad) {
+    case 1: return launch_rp<1>(p, nsm, s);
+    case 2: return launch_rp<2>(p, nsm, s);
+    case 3: return launch_rp<3>(p, nsm, s);
+    case 4: return launch_rp<4>(p, nsm, s);
+    case 8: return launch_rp<8>(p, nsm, s);
+    case 16: return launch_rp<16>(p, nsm, s);
+    default: return launch_rp<32>(p, nsm, s);
   }
 }
 

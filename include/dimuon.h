@@ -133,6 +133,8 @@ typedef struct {
                                      (128 x 256 tiles) only                */
 #define DM_DBG_TC_PAIR 0x4u       /* tensor-core products on CTA pairs
                                      (256 x 256 tiles) only                */
+#define DM_DBG_THIN_REGS 0x10u    /* thin factors always take the register
+                                     path (no shared-memory staging)       */
 #define DM_DBG_FORCE_TIMEOUT 0x8u /* failure-detection hook: each
                                      tensor-core product launch makes one
                                      bounded wait run out (20 ms, on a

@@ -61,7 +61,11 @@ def test_workspace_size_host_only():
     thin = dm.dm_workspace_size([fake_matrix(8, 4096)], hp, 1)
     big = dm.dm_workspace_size([fake_matrix(1024, 1024)], hp, 0)
     big_cond = dm.dm_workspace_size([fake_matrix(1024, 1024)], hp, 1)
-    assert thin == 1024                       # thin factors need no scratch
+    # thin factors: fp64 Gram partials (S_1, S_2) of the four 1024-column slabs
+    # of an 8 x 4096 factor (one 8x8 block each), plus small per-factor slots
+    assert 1024 + 4 * 2 * 64 * 8 <= thin <= 16 * 1024
+    thin32 = dm.dm_workspace_size([fake_matrix(4096, 32)] * 448, hp, 1)
+    assert thin32 <= dm.DM_NOALLOC_MAX_BYTES  # a LoRA r=32 set fits the static scratch
     assert big >= 2 * 1024 * 1024 * 2 + 2 * 1024 * 1024 * 2   # X ping-pong + A + B
     assert big_cond > big
     hp32 = dm.dm_default_hparams(precision=dm.DM_PREC_FP32)

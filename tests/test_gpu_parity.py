@@ -101,21 +101,36 @@ def test_ns_step_counts(ns_steps):
 
 
 # --------------------------------------------------------------------------
-# thin factors (Gram route, one CTA per factor)
+# thin factors (Gram route).  Shapes with r in {2, 4, 8, 16, 32} and a long
+# side divisible by 8 take the shared-memory staged kernels, the rest (and
+# everything under DM_DBG_THIN_REGS) the register kernels.
 # --------------------------------------------------------------------------
 THIN_SHAPES = [(4, 16), (2, 100), (8, 4096), (4096, 8), (17, 333), (32, 4096), (4096, 32),
-               (1, 50), (50, 1), (31, 31)]
+               (1, 50), (50, 1), (31, 31), (16, 1000), (2, 2056), (3000, 4), (8, 24)]
 
 
+@pytest.mark.parametrize("path", [0, dm.DM_DBG_THIN_REGS], ids=["staged", "regs"])
 @pytest.mark.parametrize("cond", [False, True])
 @pytest.mark.parametrize("mdt", [F32, BF])
-def test_thin_path(cond, mdt):
+def test_thin_path(cond, mdt, path):
     grp = Group(THIN_SHAPES, BF, BF, mdt, cond=cond, seed=15)
-    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.01)
+    hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.01, debug_flags=path)
     ws = None
     for t in range(3):
         _, ws = step_and_compare(grp, gaussian(THIN_SHAPES, 500 + t, scale_cols=True), hp,
                                  TOL_FP32, ws=ws)
+
+
+@pytest.mark.parametrize("cond", [False, True])
+def test_thin_path_fp32_storage(cond):
+    """fp32 gradients, momentum and weights (the third staged combination)."""
+    shapes = [(8, 512), (512, 16), (32, 256), (4, 96), (2, 40)]
+    grp = Group(shapes, F32, F32, F32, cond=cond, seed=17)
+    hp = hparams(dm.DM_PREC_FP32, nesterov=1)
+    ws = None
+    for t in range(3):
+        _, ws = step_and_compare(grp, gaussian(shapes, 700 + t, scale_cols=True), hp, TOL_FP32,
+                                 ws=ws)
 
 
 def test_thin_threshold_hook_matches_ns_path():
