@@ -328,7 +328,9 @@ def main():
         gbs = step_bytes(spec) / (ms_step / 1e3) / 1e9
         peak = peaks.get("hbm_gbs", 6650.0)
         roofline = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                    "frac": gbs / peak, "traffic": None, "kernel": "thin_step",
+                    "frac": gbs / peak, "traffic": None,
+                    "kernel": "thin path (thin_setup + thin_gram + thin_iterate + thin_apply), "
+                              "algorithmic bytes of the whole step over the step time",
                     "peak_kind": f"{peak_kind} HBM copy"}
 
     # end to end through the public API: pinned host gradients in, status out
@@ -361,9 +363,15 @@ def main():
     big = n_mat - thin
     launches = 0
     if thin:
-        launches += sum(math.ceil(sum(1 for s in shapes if min(s) <= dm.DM_THIN_MAX and
-                                      lo < min(s) <= hi) / 256)
-                        for lo, hi in ((0, 8), (8, 16), (16, 32)))
+        # per padded short side: thin_setup (448 factors per launch), then the
+        # Gram, r x r iteration and apply launches
+        pads = {}
+        for s in shapes:
+            r = min(s)
+            if r <= dm.DM_THIN_MAX:
+                pad = r if r <= 4 else 8 if r <= 8 else 16 if r <= 16 else 32
+                pads[pad] = pads.get(pad, 0) + 1
+        launches += sum(math.ceil(cnt / 448) + 3 for cnt in pads.values())
     if big:
         launches += 2 + 3 * hp.ns_steps + (3 if spec["cond"] else 0)
     cpu = None

@@ -34,16 +34,33 @@ def _stale():
 
 
 def build(force=False, verbose=False, extra=()):
+    """Compiles each source to an object in parallel (objects under a
+    temporary folder), then links the shared library."""
     if not force and not _stale():
         return LIB
-    cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
-           "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
-           "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp"]
-    cmd += list(extra)
-    cmd += [os.path.join(CSRC, f) for f in SOURCES]
-    if verbose:
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True)
+    import tempfile
+    from concurrent.futures import ThreadPoolExecutor
+
+    flags = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
+             "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
+    flags += list(extra)
+    with tempfile.TemporaryDirectory(prefix="dimuon_build_") as tmp:
+        def compile_one(src):
+            obj = os.path.join(tmp, src.replace(".cu", ".o"))
+            cmd = [nvcc_path()] + flags + ["-c", os.path.join(CSRC, src), "-o", obj]
+            if verbose:
+                print(" ".join(cmd), flush=True)
+            subprocess.run(cmd, check=True)
+            return obj
+
+        workers = max(1, min(len(SOURCES), os.cpu_count() or 1))
+        with ThreadPoolExecutor(max_workers=workers) as pool:
+            objs = list(pool.map(compile_one, SOURCES))
+        link = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                "-Xcompiler", "-fPIC", "-o", LIB + ".tmp"] + objs
+        if verbose:
+            print(" ".join(link), flush=True)
+        subprocess.run(link, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

@@ -419,14 +419,14 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
         t.upd = um.update_out;
         t.e_row = cond ? um.row_energy : nullptr;
         t.e_col = cond ? um.col_energy : nullptr;
-        t.rows = um.rows;
-        t.cols = um.cols;
-        t.gdt = um.grad_dtype;
-        t.mdt = um.momentum_dtype;
-        t.wdt = um.weight_dtype;
+        t.rows = (int32_t)um.rows;
+        t.cols = (int32_t)um.cols;
+        t.gdt = (uint8_t)um.grad_dtype;
+        t.mdt = (uint8_t)um.momentum_dtype;
+        t.wdt = (uint8_t)um.weight_dtype;
         t.kappa = kappa_of(hp, um.rows, um.cols);
         auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
-        t.vec = al16(um.grad) && al16(um.momentum) && al16(um.weight) && al16(um.update_out);
+        t.vec = (uint8_t)(al16(um.grad) && al16(um.momentum) && al16(um.weight) && al16(um.update_out));
       }
       DM_CUDA(launch_thin_setup(sp, s));
     }

@@ -186,19 +186,19 @@ struct K3Params {
 // thin_iterate and thin_apply then cover every factor of that padded side,
 // the streaming two in slabs of thin_slab(pad) long-side columns handed out
 // by a device counter.
-struct ThinMat {
+struct ThinMat {           // 64 bytes
   const void* G;
   void* M;
   void* W;
   float* upd;
   float* e_row;           // user orientation, null in Muon mode
   float* e_col;
-  int64_t rows, cols;
-  int gdt, mdt, wdt;
-  int vec;                // G, M, W, upd all 16-byte aligned
+  int32_t rows, cols;
+  uint8_t gdt, mdt, wdt;
+  uint8_t vec;            // G, M, W, upd all 16-byte aligned
   float kappa;
 };
-constexpr int THIN_MAX = 256;
+constexpr int THIN_MAX = 448;  // descriptors per setup launch (kernel parameter space)
 struct ThinSetupParams {
   int count;              // factors in this launch (<= THIN_MAX)
   int first;              // their first index in the group
@@ -230,6 +230,8 @@ struct ThinParams {
                           // energies, conditioning on, zero update
   int* counters;          // [2]: next slab of thin_gram / thin_apply (zero at the start)
 };
+static_assert(sizeof(ThinMat) == 64, "ThinMat packing");
+static_assert(sizeof(ThinSetupParams) <= 32764, "kernel parameter space");
 int thin_part_doubles(int pad);
 int thin_slab(int pad);
 

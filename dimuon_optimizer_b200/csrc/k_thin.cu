@@ -96,7 +96,18 @@ __global__ void __launch_bounds__(256) thin_setup(const __grid_constant__ ThinSe
   double sc = 0.0, sr = 0.0;
   if (q.cond) {
     for (int i = tid; i < q.r; i += blockDim.x) sr += (double)q.e_r[i];
-    for (int64_t k = tid; k < q.n; k += blockDim.x) sc += (double)q.e_c[k];
+    if ((reinterpret_cast<uintptr_t>(q.e_c) & 15u) == 0) {
+      const float4* e4 = reinterpret_cast<const float4*>(q.e_c);
+      const int64_t n4 = q.n >> 2;
+#pragma unroll 4
+      for (int64_t k = tid; k < n4; k += blockDim.x) {
+        const float4 v = e4[k];
+        sc += ((double)v.x + (double)v.y) + ((double)v.z + (double)v.w);
+      }
+      for (int64_t k = 4 * n4 + tid; k < q.n; k += blockDim.x) sc += (double)q.e_c[k];
+    } else {
+      for (int64_t k = tid; k < q.n; k += blockDim.x) sc += (double)q.e_c[k];
+    }
   }
   sc = block_sum_d(sc, red);
   sr = block_sum_d(sr, red);
@@ -400,6 +411,147 @@ __device__ __forceinline__ void mm(double (*C)[TCfg<RP>::SLD], double (*A)[TCfg<
     }
   }
   __syncthreads();
+}
+
+// ---- one warp per factor for RP <= 8 (no block-wide barriers) -------------
+template <int RP>
+struct WarpIterSmem {
+  double G[RP][RP + 1], H[RP][RP + 1], P[RP][RP + 1], A[RP][RP + 1], Q[RP][RP + 1], S[RP][RP + 1];
+  double R[RP];
+};
+
+template <int RP>
+__device__ __forceinline__ void mm_warp(double (*C)[RP + 1], double (*A)[RP + 1], double (*B)[RP + 1]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (RP == 8) {
+    const int g = lane >> 2, t = lane & 3;
+    double d0 = 0.0, d1 = 0.0;
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) dmma(d0, d1, A[g][kb * 4 + t], B[kb * 4 + t][g]);
+    __syncwarp();  // every lane has read A and B (C may alias neither, but keep order)
+    C[g][2 * t] = d0;
+    C[g][2 * t + 1] = d1;
+  } else {
+    if (lane < RP * RP) {
+      const int i = lane / RP, j = lane % RP;
+      double s = 0.0;
+#pragma unroll
+      for (int k = 0; k < RP; ++k) s = fma(A[i][k], B[k][j], s);
+      C[i][j] = s;
+    }
+  }
+  __syncwarp();
+}
+
+template <int RP>
+__global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ ThinParams p) {
+  using Cf = TCfg<RP>;
+  __shared__ WarpIterSmem<RP> sm[TW];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = blockIdx.x * TW + warp;
+  if (f >= p.count) return;  // the whole warp leaves; no block-wide barrier follows
+  WarpIterSmem<RP>& s = sm[warp];
+  const ThinMat mt = p.mats[f];
+  const Geo q = geometry(mt, p.conditioned);
+  const int r = q.r;
+  const int u0 = p.starts[f], nu = p.starts[f + 1] - p.starts[f];
+
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP, j = idx % RP;
+    int src;
+    if constexpr (Cf::MMA) {
+      src = (i & 7) * 8 + (j & 7);  // one 8x8 block
+    } else {
+      src = idx;
+    }
+    double g1 = 0.0, g2 = 0.0;
+    for (int v = 0; v < nu; ++v) {
+      const double* pp = p.part + (size_t)(u0 + v) * 2 * Cf::PART;
+      g1 += pp[src];
+      g2 += pp[Cf::PART + src];
+    }
+    s.G[i][j] = g1;
+    s.H[i][j] = g2;
+  }
+  const double sc = p.fsc[4 * f], sr = p.fsc[4 * f + 1];
+  const bool on = q.cond && sr > 0.0 && sc > 0.0;
+  if (lane < RP) {
+    double rv = lane < r ? 1.0 : 0.0;
+    if (on && lane < r) rv = 1.0 / sqrt(sqrt((double)q.e_r[lane] * ((double)r / sr) + (double)p.eps));
+    s.R[lane] = rv;
+  }
+  __syncwarp();
+  if (q.cond && lane < r) {
+    float e = 0.f;
+    for (int v = 0; v < nu; ++v) e += p.rpart[(size_t)(u0 + v) * RP + lane];
+    q.e_r[lane] = e;
+  }
+  double tr = 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP, j = idx % RP;
+    const double rr = s.R[i] * s.R[j];
+    s.G[i][j] *= rr;
+    s.H[i][j] *= rr;
+    if (i == j) tr += s.G[i][j];
+  }
+  const double s2 = warp_sum_d(tr);
+  const bool finite = isfinite(s2);
+  const bool valid = finite && s2 >= NORM2_FLOOR;
+  const double inv_s2 = valid ? 1.0 / s2 : 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP, j = idx % RP;
+    s.A[i][j] = valid ? s.G[i][j] * inv_s2 : 0.0;
+    s.P[i][j] = i == j ? 1.0 : 0.0;
+  }
+  __syncwarp();
+  const double a = p.a, b = p.b, c = p.c;
+  for (int it = 0; it < p.ns_steps; ++it) {
+    mm_warp<RP>(s.Q, s.A, s.A);
+    for (int idx = lane; idx < RP * RP; idx += 32) {
+      const int i = idx / RP, j = idx % RP;
+      s.Q[i][j] = c * s.Q[i][j] + b * s.A[i][j] + (i == j ? a : 0.0);
+    }
+    __syncwarp();
+    mm_warp<RP>(s.S, s.Q, s.P);
+    for (int idx = lane; idx < RP * RP; idx += 32) s.P[idx / RP][idx % RP] = s.S[idx / RP][idx % RP];
+    __syncwarp();
+    mm_warp<RP>(s.S, s.Q, s.A);
+    mm_warp<RP>(s.A, s.S, s.Q);
+  }
+  mm_warp<RP>(s.S, s.P, s.G);
+  double nx = 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) nx += s.S[idx / RP][idx % RP] * s.P[idx / RP][idx % RP];
+  nx = warp_sum_d(nx);
+  mm_warp<RP>(s.Q, s.P, s.H);
+  double ny = 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP;
+    ny += s.R[i] * s.R[i] * s.Q[i][idx % RP] * s.P[i][idx % RP];
+  }
+  ny = warp_sum_d(ny);
+  double factor = 0.0;
+  if (valid) {
+    factor = (double)mt.kappa / sqrt(s2);
+    if (on) factor = ny > 0.0 ? factor * sqrt(nx / ny) : 0.0;
+  }
+  if (!finite && lane == 0) raise_status(p.status, ST_NONFINITE);
+  double* T = p.T + (size_t)f * RP * RP;
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    int i, j;
+    if constexpr (Cf::MMA) {  // fragment order, KB = 2, one row block
+      const int l = idx & 31, kb = idx >> 5;
+      i = l >> 2;
+      j = 4 * kb + (l & 3);
+    } else {
+      i = idx / RP;
+      j = idx % RP;
+    }
+    T[idx] = factor * s.R[i] * s.P[i][j] * s.R[j];
+  }
+  if (lane == 0) {
+    p.fsc[4 * f + 2] = on ? 1.0 : 0.0;
+    p.fsc[4 * f + 3] = factor == 0.0 ? 1.0 : 0.0;
+  }
 }
 
 template <int RP>
@@ -868,6 +1020,10 @@ int resident_ctas(K kernel, int smem) {
 
 template <int RP>
 cudaError_t launch_iter_rp(const ThinParams& p, cudaStream_t st) {
+  if constexpr (RP <= 8) {
+    thin_iterate_warp<RP><<<(p.count + TW - 1) / TW, TT, 0, st>>>(p);
+    return cudaGetLastError();
+  }
   const int iter_bytes = (int)sizeof(IterSmem<RP>);
   static int configured = -1;
   int dev = 0;

@@ -8,8 +8,12 @@
 // One producer warp per CTA takes slabs from the device counter and streams
 // each slab through a ring of shared-memory stages with 1-D bulk async copies
 // (cp.async.bulk, completion on an mbarrier): the copies of the next stages
-// are in flight while four consumer warps work on the current one, so the
-// loads need neither registers nor per-lane address arithmetic.  Consumers
+// are in flight while the consumer warps (8, or 4 for r = 32) work on the
+// current one, so the loads need neither registers nor per-lane address
+// arithmetic.  Full steps run branch-free code specialised on the layout
+// (wide / tall), on whether Dimuon conditioning is on and on whether
+// energies are written; partial steps at a factor's end take a predicated
+// version.  Consumers
 // write their results (M_t, W, O, energies) straight to global memory.  Every
 // wait is bounded; the slab-end reduction of the Gram partials synchronises
 // the consumer warps through mbarriers, so a timeout can never leave a warp
@@ -26,11 +30,42 @@ namespace {
 using namespace thin;
 using namespace sm100;
 
-constexpr int BT = 160;          // 4 consumer warps + 1 producer warp
-constexpr int CW = 4;            // consumer warps
 constexpr int ROWPAD = 64;       // bytes after each staged wide row (bank shift)
 constexpr uint64_t WAIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
+
+// Bounded wait on an mbarrier phase whose try_wait carries a suspend-time
+// hint, so a waiting warp sleeps in the barrier unit instead of spinning
+// through issue slots the working warps need.  Same contract as
+// mbar_wait_bounded: false after an abort or after WAIT_NS (then the abort
+// flag and the timeout status are set).
+constexpr uint32_t SLEEP_NS = 20000;
+__device__ __forceinline__ bool try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(SLEEP_NS)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                           int* status) {
+  if (try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (try_wait_sleep(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > WAIT_NS) {
+      *abort = 1;
+      raise_status(status, ST_TIMEOUT);
+      return false;
+    }
+  }
+}
 
 // Element types of the staged operands.
 template <typename T>
@@ -89,7 +124,7 @@ struct El<__nv_bfloat16> {
 struct StageInfo {
   ThinMat mt;
   int u, f, c0, c1;  // slab, factor, long-side columns [c0, c1)
-  int first, last;   // first / last stage of the slab
+  int first, last;   // first / last stage of a run of slabs of one factor in this CTA
   int on, zero;      // Dimuon conditioning on; zero update (apply pass)
   float inv_mc;      // n / sum of the previous long-side energies
   int pad_;
@@ -112,68 +147,107 @@ __device__ __forceinline__ void drain_stages(uint64_t* full, int ns, uint32_t ar
     if (armed & (1u << s)) mbar_wait_drain(&full[s], (armed_par >> s) & 1u, DRAIN_NS);
 }
 
+// Per-slab values the producer needs (and hands to the consumers).
+struct SlabMeta {
+  ThinMat mt;
+  int f;
+  int on, zero;
+  float inv_mc;
+  int64_t c_lo, c_hi;
+};
+
+template <int RP, int KIND>
+__device__ __forceinline__ SlabMeta slab_meta(const ThinParams& p, int u) {
+  SlabMeta m;
+  m.f = p.unit_f[u];
+  m.mt = p.mats[m.f];
+  const Geo q = geometry(m.mt, p.conditioned);
+  m.c_lo = (int64_t)(u - p.starts[m.f]) * TCfg<RP>::SLAB;
+  m.c_hi = min(q.n, m.c_lo + TCfg<RP>::SLAB);
+  const double sc = p.fsc[4 * m.f];
+  if (KIND == 0) {
+    m.on = q.cond && sc > 0.0 && p.fsc[4 * m.f + 1] > 0.0;
+    m.zero = 0;
+  } else {
+    m.on = p.fsc[4 * m.f + 2] != 0.0;
+    m.zero = p.fsc[4 * m.f + 3] != 0.0;
+  }
+  m.inv_mc = m.on ? (float)((double)q.n / sc) : 0.f;
+  return m;
+}
+
 // ---------------------------------------------------------------------------
-// Producer: slabs from the counter, stages through the ring.  `kind` 0 =
-// gram pass (M, G, E), 1 = apply pass (M, G under Nesterov, W, E).
+// Producer: slabs blockIdx.x, blockIdx.x + gridDim.x, ... (the next slab's
+// descriptor is loaded while the current slab's stages are issued), stages
+// through the ring.  KIND 0 = gram pass (M, G, E), 1 = apply pass (M, G
+// under Nesterov, W, E).
 // ---------------------------------------------------------------------------
 template <int RP, int CH, int NS, typename TG, typename TM, typename TW, int KIND>
 __device__ void produce(const ThinParams& p, uint8_t* stages, int stage_bytes, int offG, int offW,
                         int offE, StageInfo* info, uint64_t* full, uint64_t* empty,
-                        volatile int* abort, int* counter) {
+                        volatile int* abort, int pw, int np) {
+  // np producer warps walk the same stage sequence; warp pw fills the
+  // stages whose ring index is pw modulo np (one warp's copy issue rate is
+  // far below what the memory system takes)
   const int lane = threadIdx.x & 31;
   int stage = 0;
   uint32_t ph = 0, armed = 0, armed_par = 0;
   bool ok = true;
-  const int slab_cols = TCfg<RP>::SLAB;
-  for (;;) {
-    int u = 0;
-    if (lane == 0) u = atomicAdd(counter, 1);
-    u = __shfl_sync(0xffffffffu, u, 0);
-    if (u >= p.units) break;
-    const int f = p.unit_f[u];
-    const int64_t c_lo = (int64_t)(u - p.starts[f]) * slab_cols;
-    // per-slab values, lane 0 only
-    ThinMat mt;
-    Geo q;
-    int64_t c_hi = 0;
-    int on = 0, zero = 0;
-    float inv_mc = 0.f;
-    if (lane == 0) {
-      mt = p.mats[f];
-      q = geometry(mt, p.conditioned);
-      c_hi = min(q.n, c_lo + slab_cols);
-      if (KIND == 0) {
-        on = q.cond && p.fsc[4 * f] > 0.0 && p.fsc[4 * f + 1] > 0.0;
-      } else {
-        on = p.fsc[4 * f + 2] != 0.0;
-        zero = p.fsc[4 * f + 3] != 0.0;
-      }
-      inv_mc = on ? (float)((double)q.n / p.fsc[4 * f]) : 0.f;
+  // contiguous slab range of this CTA (balanced to within one slab), so a
+  // CTA's slabs of one factor are consecutive and the Gram partials of such
+  // a run are reduced once
+  const int q = p.units / (int)gridDim.x, rem = p.units % (int)gridDim.x;
+  const int u_begin = (int)blockIdx.x * q + min((int)blockIdx.x, rem);
+  const int u_end = u_begin + q + ((int)blockIdx.x < rem ? 1 : 0);
+  int u = u_begin;
+  int prev_f = -1;
+  SlabMeta cur;
+  // every lane holds the slab values, so the loop control below is warp-uniform
+  if (u < u_end) cur = slab_meta<RP, KIND>(p, u);
+  while (u < u_end && ok) {
+    const int un = u + 1;
+    SlabMeta nxt;
+    if (un < u_end) nxt = slab_meta<RP, KIND>(p, un);
+    const bool run_first = cur.f != prev_f;
+    const bool run_last = un >= u_end || nxt.f != cur.f;
+    if (KIND == 0 && !run_last && pw == 0) {
+      // this slab's partial slot holds zeros: the run's sum goes to its last slab
+      constexpr int PART = TCfg<RP>::PART;
+      double* dst = p.part + (size_t)u * 2 * PART;
+      for (int i = lane; i < 2 * PART; i += 32) dst[i] = 0.0;
+      if (cur.mt.e_row != nullptr && p.conditioned)
+        for (int i = lane; i < RP; i += 32) p.rpart[(size_t)u * RP + i] = 0.f;
     }
-    for (int64_t c0 = c_lo;; c0 += CH) {
+    for (int64_t c0 = cur.c_lo;; c0 += CH) {
+      if (c0 >= cur.c_hi) break;
+      if (stage % np != pw) {  // another producer warp's stage
+        if (++stage == NS) {
+          stage = 0;
+          ph ^= 1;
+        }
+        continue;
+      }
       int go = 1;
       if (lane == 0) {
-        if (c0 >= c_hi) {
-          go = 0;
-        } else if (!mbar_wait_bounded(&empty[stage], ph ^ 1, abort, p.status, WAIT_NS)) {
+        if (!wait_phase(&empty[stage], ph ^ 1, abort, p.status)) {
           go = -1;
         } else {
           StageInfo& si = info[stage];
-          si.mt = mt;
+          si.mt = cur.mt;
           si.u = u;
-          si.f = f;
+          si.f = cur.f;
           si.c0 = (int)c0;
-          si.c1 = (int)min(c0 + CH, c_hi);
-          si.first = c0 == c_lo;
-          si.last = si.c1 == c_hi;
-          si.on = on;
-          si.zero = zero;
-          si.inv_mc = inv_mc;
+          si.c1 = (int)min(c0 + CH, cur.c_hi);
+          si.first = run_first && c0 == cur.c_lo;
+          si.last = run_last && si.c1 == cur.c_hi;
+          si.on = cur.on;
+          si.zero = cur.zero;
+          si.inv_mc = cur.inv_mc;
           const int w = si.c1 - si.c0;
           uint32_t bytes = (uint32_t)(RP * w) * (uint32_t)sizeof(TM);
           if (KIND == 0 || p.nesterov) bytes += (uint32_t)(RP * w) * (uint32_t)sizeof(TG);
           if (KIND == 1) bytes += (uint32_t)(RP * w) * (uint32_t)sizeof(TW);
-          if (si.on) bytes += (uint32_t)w * 4u;
+          if (cur.on) bytes += (uint32_t)w * 4u;
           mbar_arrive_expect_tx(&full[stage], bytes);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (ph << stage);
@@ -223,10 +297,12 @@ __device__ void produce(const ThinParams& p, uint8_t* stages, int stage_bytes, i
         ph ^= 1;
       }
     }
-    if (!ok) break;
+    prev_f = cur.f;
+    u = un;
+    cur = nxt;
   }
   if (lane == 0) {
-    if (ok && mbar_wait_bounded(&empty[stage], ph ^ 1, abort, p.status, WAIT_NS)) {
+    if (ok && stage % np == pw && wait_phase(&empty[stage], ph ^ 1, abort, p.status)) {
       info[stage].u = -1;  // end of the work
       mbar_arrive(&full[stage]);
     }
@@ -234,26 +310,270 @@ __device__ void produce(const ThinParams& p, uint8_t* stages, int stage_bytes, i
   }
 }
 
+// Column weights C_j^2 (and C_j^4) of the columns a consumer warp handles in
+// the current stage, computed once per column: the warp's k-th step of SW
+// columns starts at c0 + SW (warp + CW k); entry k SW + o holds column
+// o of that step (zero past c1).
+template <int SW, int CW, int NCOL>
+__device__ __forceinline__ void stage_weights(double* wmine, const float* Es, int c0, int c1, int warp,
+                                              int lane, float inv_mc, float eps) {
+  for (int idx = lane; idx < NCOL; idx += 32) {
+    const int k = idx / SW, o = idx % SW;
+    const int col = c0 + SW * (warp + CW * k) + o;
+    const double w = col < c1 ? (double)col_weight(Es[col - c0], inv_mc, eps) : 0.0;
+    wmine[idx] = w;
+    wmine[NCOL + idx] = w * w;
+  }
+  __syncwarp();
+}
+
 // ===========================================================================
-// thin_gram_bulk
+// thin_gram_bulk: momentum, Gram partials, short-side energy partials
 // ===========================================================================
 template <int RP, typename TG, typename TM>
 struct GramBulk {
-  static constexpr int CH = 2048 / RP;
+  static constexpr int CW = RP == 32 ? 4 : 8;  // consumer warps
+  static constexpr int NP = 2;                 // producer warps
+  static constexpr int BT = 32 * (CW + NP);
+  static constexpr int MINB = RP == 8 || RP == 16 ? 3 : 1;  // resident CTAs the registers allow
+  static constexpr int CH = RP <= 4 ? 1024 : RP == 8 ? 256 : RP == 16 ? 128 : 64;
   static constexpr int NS = 4;
+  // reduction at the end of a run of slabs: NSLOT > 0 = asynchronous (each
+  // warp drops its partial into one of NSLOT slots, the last warp to arrive
+  // sums); 0 = all consumer warps meet
+  static constexpr int NSLOT = 0;
+  static constexpr int NRED = NSLOT > 0 ? NSLOT : 1;
+  static constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH);
   static constexpr int OFF_G = opnd_bytes<TM>(RP, CH);
   static constexpr int OFF_E = OFF_G + opnd_bytes<TG>(RP, CH);
   static constexpr int STAGE_BYTES = (OFF_E + CH * 4 + 127) / 128 * 128;
-  static constexpr int RED_BYTES = CW * 2 * TCfg<RP>::PART * 8 + CW * RP * 4;
+  static constexpr int RED_BYTES = NRED * (CW * 2 * TCfg<RP>::PART * 8 + CW * RP * 4) + NRED * 16;
+  static constexpr int NCOL = TCfg<RP>::MMA ? CH / CW : 0;  // columns of one consumer warp per stage
+  static constexpr int WS_BYTES = CW * 2 * NCOL * 8;
   static constexpr int SMEM = NS * STAGE_BYTES + NS * (int)sizeof(StageInfo) +
-                              (2 * NS + 2) * 8 + 16 + RED_BYTES + 128;
+                              (2 * NS + 2 + NRED) * 8 + 16 + RED_BYTES + WS_BYTES + 128;
 };
 
+// Accumulators of one consumer lane for one slab.
+template <int RP>
+struct GramAcc {
+  static constexpr bool MMA = TCfg<RP>::MMA;
+  double s1[MMA ? TCfg<RP>::NUB : RP][MMA ? 2 : RP];
+  double s2[MMA ? TCfg<RP>::NUB : RP][MMA ? 2 : RP];
+  float er[MMA ? TCfg<RP>::NB : RP];
+};
+
+// 16 long-side columns c .. c + 15, all inside the stage (RP >= 8).
+// Lane (g, t) holds rows g + 8 blk at columns c + 4t + e (wide) or
+// c + t + 4e (tall); the DMMA's k slot t is that column.
+template <int RP, typename TG, typename TM, bool TALL, bool ON, bool NEST>
+__device__ __forceinline__ void gram_step_mma(GramAcc<RP>& acc, const TM* Ms, const TG* Gs,
+                                              const double* wrow, TM* Mg, int64_t n, int cs, int c,
+                                              float mu, int g, int t) {
+  using L = GramBulk<RP, TG, TM>;
+  constexpr int NB = TCfg<RP>::NB;
+  float mv[NB][4], gv[NB][4];
+  if constexpr (!TALL) {
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+      El<TM>::ld4(Ms + (g + 8 * blk) * L::PM + cs + 4 * t, mv[blk]);
+      El<TG>::ld4(Gs + (g + 8 * blk) * L::PG + cs + 4 * t, gv[blk]);
+    }
+  } else {
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int o = (cs + t + 4 * e) * RP + g + 8 * blk;
+        mv[blk][e] = El<TM>::ld1(Ms + o);
+        gv[blk][e] = El<TG>::ld1(Gs + o);
+      }
+  }
+  double wd[4], w2d[4];
+  if constexpr (ON) {
+    constexpr int NCOL = L::NCOL;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int o = TALL ? t + 4 * e : 4 * t + e;
+      wd[e] = wrow[o];
+      w2d[e] = wrow[NCOL + o];
+    }
+  }
+  double bx[NB][4];
+#pragma unroll
+  for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float m = momentum_value(mu, mv[blk][e], gv[blk][e], El<TM>::DT);
+      mv[blk][e] = m;
+      bx[blk][e] = NEST ? fma((double)mu, (double)m, (double)gv[blk][e]) : (double)m;
+      acc.er[blk] = fmaf(m, m, acc.er[blk]);
+    }
+  if constexpr (!TALL) {
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) El<TM>::st4(Mg + (int64_t)(g + 8 * blk) * n + c + 4 * t, mv[blk]);
+  } else {
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) El<TM>::st1(Mg + (int64_t)(c + t + 4 * e) * RP + g + 8 * blk, mv[blk][e]);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    double xw[NB], xw2[NB];
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+      xw[blk] = ON ? wd[e] * bx[blk][e] : bx[blk][e];
+      xw2[blk] = ON ? w2d[e] * bx[blk][e] : 0.0;
+    }
+    int ub = 0;
+#pragma unroll
+    for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+      for (int bj = bi; bj < NB; ++bj, ++ub) {
+        dmma(acc.s1[ub][0], acc.s1[ub][1], bx[bi][e], xw[bj]);
+        if constexpr (ON) dmma(acc.s2[ub][0], acc.s2[ub][1], bx[bi][e], xw2[bj]);
+      }
+  }
+}
+
+// Predicated version of gram_step_mma for a step that crosses the stage end.
 template <int RP, typename TG, typename TM>
-__global__ void __launch_bounds__(BT) thin_gram_bulk(const __grid_constant__ ThinParams p) {
+__device__ __noinline__ void gram_step_mma_tail(GramAcc<RP>& acc, const TM* Ms, const TG* Gs,
+                                                const float* Es, TM* Mg, int64_t n, bool tall,
+                                                bool on, int cs, int c, int c1, float mu,
+                                                float inv_mc, float eps, bool nest, int g, int t) {
+  using L = GramBulk<RP, TG, TM>;
+  constexpr int NB = TCfg<RP>::NB;
+  float mv[NB][4], gv[NB][4];
+  bool okc[4];
+  double wd[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int col = tall ? c + t + 4 * e : c + 4 * t + e;
+    okc[e] = col < c1;
+    wd[e] = on ? (okc[e] ? (double)col_weight(Es[col - c + cs], inv_mc, eps) : 0.0) : 1.0;
+  }
+#pragma unroll
+  for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int o = tall ? (cs + t + 4 * e) * RP + g + 8 * blk : (g + 8 * blk) * L::PM + cs + 4 * t + e;
+      const int og = tall ? o : (g + 8 * blk) * L::PG + cs + 4 * t + e;
+      mv[blk][e] = okc[e] ? El<TM>::ld1(Ms + o) : 0.f;
+      gv[blk][e] = okc[e] ? El<TG>::ld1(Gs + og) : 0.f;
+    }
+  double bx[NB][4];
+#pragma unroll
+  for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float m = momentum_value(mu, mv[blk][e], gv[blk][e], El<TM>::DT);
+      mv[blk][e] = m;
+      bx[blk][e] = nest ? fma((double)mu, (double)m, (double)gv[blk][e]) : (double)m;
+      acc.er[blk] = fmaf(m, m, acc.er[blk]);
+      const int col = tall ? c + t + 4 * e : c + 4 * t + e;
+      if (okc[e])
+        El<TM>::st1(Mg + (tall ? (int64_t)col * RP + g + 8 * blk : (int64_t)(g + 8 * blk) * n + col),
+                    m);
+    }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    double xw[NB], xw2[NB];
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+      xw[blk] = wd[e] * bx[blk][e];
+      xw2[blk] = wd[e] * xw[blk];
+    }
+    int ub = 0;
+#pragma unroll
+    for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+      for (int bj = bi; bj < NB; ++bj, ++ub) {
+        dmma(acc.s1[ub][0], acc.s1[ub][1], bx[bi][e], xw[bj]);
+        if (on) dmma(acc.s2[ub][0], acc.s2[ub][1], bx[bi][e], xw2[bj]);
+      }
+  }
+}
+
+// Four long-side columns c .. c + 3 owned by one lane (RP == r <= 4); the
+// stage width is a multiple of 8, so every step is full.
+template <int RP, typename TG, typename TM, bool TALL, bool ON, bool NEST>
+__device__ __forceinline__ void gram_step_small(GramAcc<RP>& acc, const TM* Ms, const TG* Gs,
+                                                const float* Es, TM* Mg, int64_t n, int cs, int c,
+                                                float mu, float inv_mc, float eps) {
+  using L = GramBulk<RP, TG, TM>;
+  float mv[RP][4], gv[RP][4];
+  if constexpr (!TALL) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i) {
+      El<TM>::ld4(Ms + i * L::PM + cs, mv[i]);
+      El<TG>::ld4(Gs + i * L::PG + cs, gv[i]);
+    }
+  } else {
+    float fm[4 * RP], fg[4 * RP];
+#pragma unroll
+    for (int s = 0; s < RP; ++s) {
+      El<TM>::ld4(Ms + cs * RP + 4 * s, &fm[4 * s]);
+      El<TG>::ld4(Gs + cs * RP + 4 * s, &fg[4 * s]);
+    }
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        mv[i][e] = fm[e * RP + i];
+        gv[i][e] = fg[e * RP + i];
+      }
+  }
+  double wd[4];
+  if constexpr (ON) {
+    const float4 e4 = *reinterpret_cast<const float4*>(Es + cs);
+    wd[0] = (double)col_weight(e4.x, inv_mc, eps);
+    wd[1] = (double)col_weight(e4.y, inv_mc, eps);
+    wd[2] = (double)col_weight(e4.z, inv_mc, eps);
+    wd[3] = (double)col_weight(e4.w, inv_mc, eps);
+  }
+  double bx[RP][4];
+#pragma unroll
+  for (int i = 0; i < RP; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float m = momentum_value(mu, mv[i][e], gv[i][e], El<TM>::DT);
+      mv[i][e] = m;
+      bx[i][e] = NEST ? fma((double)mu, (double)m, (double)gv[i][e]) : (double)m;
+      acc.er[i] = fmaf(m, m, acc.er[i]);
+    }
+  if constexpr (!TALL) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i) El<TM>::st4(Mg + (int64_t)i * n + c, mv[i]);
+  } else {
+    float fm[4 * RP];
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) fm[e * RP + i] = mv[i][e];
+#pragma unroll
+    for (int s = 0; s < RP; ++s) El<TM>::st4(Mg + (int64_t)c * RP + 4 * s, &fm[4 * s]);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int k = i; k < RP; ++k) {
+        const double xk = ON ? wd[e] * bx[k][e] : bx[k][e];
+        acc.s1[i][k] = fma(bx[i][e], xk, acc.s1[i][k]);
+        if constexpr (ON) acc.s2[i][k] = fma(bx[i][e], wd[e] * xk, acc.s2[i][k]);
+      }
+  }
+}
+
+template <int RP, typename TG, typename TM>
+__global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>::MINB)
+    thin_gram_bulk(const __grid_constant__ ThinParams p) {
   using L = GramBulk<RP, TG, TM>;
   using Cf = TCfg<RP>;
-  constexpr int CH = L::CH, NS = L::NS;
+  constexpr int CH = L::CH, NS = L::NS, CW = L::CW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
@@ -261,11 +581,15 @@ __global__ void __launch_bounds__(BT) thin_gram_bulk(const __grid_constant__ Thi
   StageInfo* info = reinterpret_cast<StageInfo*>(smem + NS * L::STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(info + NS);
   uint64_t* empty = full + NS;
-  uint64_t* redf = empty + NS;  // consumer warps wrote their partials
-  uint64_t* redr = redf + 1;    // consumer warps read the partials
-  volatile int* abort = reinterpret_cast<volatile int*>(redr + 1);
-  double* red_s = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(redr + 1) + 16);
-  float* red_e = reinterpret_cast<float*>(red_s + CW * 2 * Cf::PART);
+  uint64_t* redf = empty + NS;  // synchronous reduction: consumer warps wrote their partials
+  uint64_t* redr = redf + 1;    // synchronous reduction: consumer warps read the partials
+  uint64_t* done = redr + 1;    // asynchronous reduction: slot summed (one per slot)
+  volatile int* abort = reinterpret_cast<volatile int*>(done + L::NRED);
+  int* cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(done + L::NRED) + 4);  // per slot
+  double* red_s = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(done + L::NRED) + 16 +
+                                            L::NRED * 16);
+  float* red_e = reinterpret_cast<float*>(red_s + L::NRED * CW * 2 * Cf::PART);
+  double* wsm = reinterpret_cast<double*>(red_e + L::NRED * CW * RP);  // CW * RP is even
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -275,28 +599,30 @@ __global__ void __launch_bounds__(BT) thin_gram_bulk(const __grid_constant__ Thi
     }
     mbar_init(redf, CW);
     mbar_init(redr, CW);
+    for (int s = 0; s < L::NRED; ++s) {
+      mbar_init(&done[s], 1);
+      cnt[s] = 0;
+    }
     *abort = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == CW) {
+  if (warp >= CW) {
     produce<RP, CH, NS, TG, TM, TM, 0>(p, stages, L::STAGE_BYTES, L::OFF_G, 0, L::OFF_E, info, full,
-                                       empty, abort, p.counters);
+                                       empty, abort, warp - CW, L::NP);
     return;
   }
 
   // ------------------------------- consumers -------------------------------
   const float mu = p.mu, eps = p.eps;
-  constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH);
-  constexpr int NB = Cf::NB, NUB = Cf::NUB;
-  constexpr int ROWS = Cf::MMA ? NB : RP;
-  double s1[Cf::MMA ? NUB : RP][Cf::MMA ? 2 : RP], s2[Cf::MMA ? NUB : RP][Cf::MMA ? 2 : RP];
-  float er[ROWS];
+  const bool nest = p.nesterov != 0;
+  const int g = lane >> 2, t = lane & 3;
+  GramAcc<RP> acc;
   int stage = 0;
   uint32_t ph = 0, nred = 0;
   for (;;) {
-    if (!mbar_wait_bounded(&full[stage], ph, abort, p.status, WAIT_NS)) break;
+    if (!wait_phase(&full[stage], ph, abort, p.status)) break;
     const StageInfo& si = info[stage];
     const int u = si.u;
     if (u < 0) break;
@@ -313,152 +639,49 @@ __global__ void __launch_bounds__(BT) thin_gram_bulk(const __grid_constant__ Thi
     const float* Es = reinterpret_cast<const float*>(base + L::OFF_E);
     if (first) {
 #pragma unroll
-      for (int a = 0; a < (Cf::MMA ? NUB : RP); ++a)
+      for (int a = 0; a < (Cf::MMA ? Cf::NUB : RP); ++a)
 #pragma unroll
-        for (int b = 0; b < (Cf::MMA ? 2 : RP); ++b) s1[a][b] = s2[a][b] = 0.0;
+        for (int b = 0; b < (Cf::MMA ? 2 : RP); ++b) acc.s1[a][b] = acc.s2[a][b] = 0.0;
 #pragma unroll
-      for (int a = 0; a < ROWS; ++a) er[a] = 0.f;
+      for (int a = 0; a < (Cf::MMA ? Cf::NB : RP); ++a) acc.er[a] = 0.f;
     }
 
     if constexpr (Cf::MMA) {
-      const int g = lane >> 2, t = lane & 3;
-      // 16 columns per warp step: wide lane (g, t) at c + 4t + e, tall c + t + 4e
-      for (int c = c0 + 16 * warp; c < c1; c += 16 * CW) {
+      double* wmine = wsm + warp * 2 * L::NCOL;
+      if (on) stage_weights<16, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
+      int k = 0;
+      for (int c = c0 + 16 * warp; c < c1; c += 16 * CW, ++k) {
         const int cs = c - c0;
-        float mv[NB][4], gv[NB][4], ev[4];
-        bool okc[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = tall ? c + t + 4 * e : c + 4 * t + e;
-          okc[e] = col < c1;
-          ev[e] = (on && okc[e]) ? Es[col - c0] : 0.f;
-        }
-        if (!tall) {
-          const bool ok = c + 4 * t < c1;  // (c1 - c0) is a multiple of 8
-#pragma unroll
-          for (int blk = 0; blk < NB; ++blk) {
-            const int row = g + 8 * blk;
-            if (ok) {
-              El<TM>::ld4(Ms + row * PM + cs + 4 * t, mv[blk]);
-              El<TG>::ld4(Gs + row * PG + cs + 4 * t, gv[blk]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) mv[blk][e] = gv[blk][e] = 0.f;
-            }
+        const double* wrow = wmine + 16 * k;
+        if (c + 16 <= c1) {
+#define DM_GRAM_MMA(TALL_, ON_, NEST_) \
+  gram_step_mma<RP, TG, TM, TALL_, ON_, NEST_>(acc, Ms, Gs, wrow, Mg, n, cs, c, mu, g, t)
+          if (tall) {
+            if (on) { if (nest) DM_GRAM_MMA(true, true, true); else DM_GRAM_MMA(true, true, false); }
+            else { if (nest) DM_GRAM_MMA(true, false, true); else DM_GRAM_MMA(true, false, false); }
+          } else {
+            if (on) { if (nest) DM_GRAM_MMA(false, true, true); else DM_GRAM_MMA(false, true, false); }
+            else { if (nest) DM_GRAM_MMA(false, false, true); else DM_GRAM_MMA(false, false, false); }
           }
+#undef DM_GRAM_MMA
         } else {
-#pragma unroll
-          for (int blk = 0; blk < NB; ++blk)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int o = (cs + t + 4 * e) * RP + g + 8 * blk;
-              mv[blk][e] = okc[e] ? El<TM>::ld1(Ms + o) : 0.f;
-              gv[blk][e] = okc[e] ? El<TG>::ld1(Gs + o) : 0.f;
-            }
-        }
-        double bx[NB][4];
-#pragma unroll
-        for (int blk = 0; blk < NB; ++blk)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float m = momentum_value(mu, mv[blk][e], gv[blk][e], El<TM>::DT);
-            mv[blk][e] = m;
-            bx[blk][e] = p.nesterov ? fma((double)mu, (double)m, (double)gv[blk][e]) : (double)m;
-            er[blk] = fmaf(m, m, er[blk]);
-          }
-        if (!tall) {
-          if (c + 4 * t < c1)
-#pragma unroll
-            for (int blk = 0; blk < NB; ++blk)
-              El<TM>::st4(Mg + (int64_t)(g + 8 * blk) * n + c + 4 * t, mv[blk]);
-        } else {
-#pragma unroll
-          for (int blk = 0; blk < NB; ++blk)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (okc[e]) El<TM>::st1(Mg + (int64_t)(c + t + 4 * e) * RP + g + 8 * blk, mv[blk][e]);
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const double w = on ? (okc[e] ? (double)col_weight(ev[e], inv_mc, eps) : 0.0) : 1.0;
-          double xw[NB], xw2[NB];
-#pragma unroll
-          for (int blk = 0; blk < NB; ++blk) {
-            xw[blk] = w * bx[blk][e];
-            xw2[blk] = w * xw[blk];
-          }
-          int ub = 0;
-#pragma unroll
-          for (int bi = 0; bi < NB; ++bi)
-#pragma unroll
-            for (int bj = bi; bj < NB; ++bj, ++ub) {
-              dmma(s1[ub][0], s1[ub][1], bx[bi][e], xw[bj]);
-              if (on) dmma(s2[ub][0], s2[ub][1], bx[bi][e], xw2[bj]);
-            }
+          gram_step_mma_tail<RP, TG, TM>(acc, Ms, Gs, Es, Mg, n, tall, on, cs, c, c1, mu, inv_mc, eps,
+                                         nest, g, t);
         }
       }
     } else {
-      // RP == r <= 4: lane owns columns c .. c + 3 (c1 - c0 is a multiple of 8)
       for (int c = c0 + 4 * (lane + 32 * warp); c < c1; c += 4 * 32 * CW) {
         const int cs = c - c0;
-        float mv[RP][4], gv[RP][4], ev[4];
-        if (!tall) {
-#pragma unroll
-          for (int i = 0; i < RP; ++i) {
-            El<TM>::ld4(Ms + i * PM + cs, mv[i]);
-            El<TG>::ld4(Gs + i * PG + cs, gv[i]);
-          }
+#define DM_GRAM_SMALL(TALL_, ON_, NEST_) \
+  gram_step_small<RP, TG, TM, TALL_, ON_, NEST_>(acc, Ms, Gs, Es, Mg, n, cs, c, mu, inv_mc, eps)
+        if (tall) {
+          if (on) { if (nest) DM_GRAM_SMALL(true, true, true); else DM_GRAM_SMALL(true, true, false); }
+          else { if (nest) DM_GRAM_SMALL(true, false, true); else DM_GRAM_SMALL(true, false, false); }
         } else {
-          float fm[4 * RP], fg[4 * RP];
-#pragma unroll
-          for (int s = 0; s < RP; ++s) {
-            El<TM>::ld4(Ms + cs * RP + 4 * s, &fm[4 * s]);
-            El<TG>::ld4(Gs + cs * RP + 4 * s, &fg[4 * s]);
-          }
-#pragma unroll
-          for (int i = 0; i < RP; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              mv[i][e] = fm[e * RP + i];
-              gv[i][e] = fg[e * RP + i];
-            }
+          if (on) { if (nest) DM_GRAM_SMALL(false, true, true); else DM_GRAM_SMALL(false, true, false); }
+          else { if (nest) DM_GRAM_SMALL(false, false, true); else DM_GRAM_SMALL(false, false, false); }
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) ev[e] = on ? Es[cs + e] : 0.f;
-        double bx[RP][4];
-#pragma unroll
-        for (int i = 0; i < RP; ++i)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float m = momentum_value(mu, mv[i][e], gv[i][e], El<TM>::DT);
-            mv[i][e] = m;
-            bx[i][e] = p.nesterov ? fma((double)mu, (double)m, (double)gv[i][e]) : (double)m;
-            er[i] = fmaf(m, m, er[i]);
-          }
-        if (!tall) {
-#pragma unroll
-          for (int i = 0; i < RP; ++i) El<TM>::st4(Mg + (int64_t)i * n + c, mv[i]);
-        } else {
-          float fm[4 * RP];
-#pragma unroll
-          for (int i = 0; i < RP; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) fm[e * RP + i] = mv[i][e];
-#pragma unroll
-          for (int s = 0; s < RP; ++s) El<TM>::st4(Mg + (int64_t)c * RP + 4 * s, &fm[4 * s]);
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const double w = on ? (double)col_weight(ev[e], inv_mc, eps) : 1.0;
-#pragma unroll
-          for (int i = 0; i < RP; ++i)
-#pragma unroll
-            for (int k = i; k < RP; ++k) {
-              const double xk = w * bx[k][e];
-              s1[i][k] = fma(bx[i][e], xk, s1[i][k]);
-              if (on) s2[i][k] = fma(bx[i][e], w * xk, s2[i][k]);
-            }
-        }
+#undef DM_GRAM_SMALL
       }
     }
     __syncwarp();
@@ -469,87 +692,379 @@ __global__ void __launch_bounds__(BT) thin_gram_bulk(const __grid_constant__ Thi
     }
 
     if (last) {
-      // slab-end reduction over the consumer warps (mbarrier-synchronised)
-      if (!mbar_wait_bounded(redr, (nred & 1u) ^ 1u, abort, p.status, WAIT_NS)) break;
-      double* mine = red_s + warp * 2 * Cf::PART;
+      // slab-end reduction over the consumer warps
+      const int slot = L::NSLOT > 0 ? (int)(nred % L::NRED) : 0;
+      const uint32_t use = L::NSLOT > 0 ? nred / L::NRED : nred;  // this slot's use count
+      if constexpr (L::NSLOT > 0) {
+        // the slot's previous sum is done before it is overwritten
+        if (use > 0 && !wait_phase(&done[slot], (use - 1) & 1u, abort, p.status)) break;
+      } else {
+        if (!wait_phase(redr, (nred & 1u) ^ 1u, abort, p.status)) break;
+      }
+      double* rs = red_s + (size_t)slot * CW * 2 * Cf::PART;
+      float* re = red_e + slot * CW * RP;
+      double* mine = rs + warp * 2 * Cf::PART;
       if constexpr (Cf::MMA) {
-        const int g = lane >> 2, t = lane & 3;
+        constexpr int NB = Cf::NB, NUB = Cf::NUB;
 #pragma unroll
         for (int ub = 0; ub < NUB; ++ub)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            mine[ub * 64 + g * 8 + 2 * t + h] = s1[ub][h];
-            mine[Cf::PART + ub * 64 + g * 8 + 2 * t + h] = s2[ub][h];
+            mine[ub * 64 + g * 8 + 2 * t + h] = acc.s1[ub][h];
+            mine[Cf::PART + ub * 64 + g * 8 + 2 * t + h] = acc.s2[ub][h];
           }
 #pragma unroll
         for (int blk = 0; blk < NB; ++blk) {
-          float e = er[blk];
+          float e = acc.er[blk];
           e += __shfl_xor_sync(0xffffffffu, e, 1);
           e += __shfl_xor_sync(0xffffffffu, e, 2);
-          if (t == 0) red_e[warp * RP + g + 8 * blk] = e;
+          if (t == 0) re[warp * RP + g + 8 * blk] = e;
         }
       } else {
 #pragma unroll
         for (int i = 0; i < RP; ++i) {
 #pragma unroll
           for (int k = i; k < RP; ++k) {
-            const double a = warp_sum_d(s1[i][k]), b = warp_sum_d(s2[i][k]);
+            const double a = warp_sum_d(acc.s1[i][k]), b = warp_sum_d(acc.s2[i][k]);
             if (lane == 0) {
               mine[i * RP + k] = mine[k * RP + i] = a;
               mine[Cf::PART + i * RP + k] = mine[Cf::PART + k * RP + i] = b;
             }
           }
-          const float e = warp_sum(er[i]);
-          if (lane == 0) red_e[warp * RP + i] = e;
+          const float e = warp_sum(acc.er[i]);
+          if (lane == 0) re[warp * RP + i] = e;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(redf);
-      if (!mbar_wait_bounded(redf, nred & 1u, abort, p.status, WAIT_NS)) break;
       double* dst = p.part + (size_t)u * 2 * Cf::PART;
-      for (int i = tid; i < 2 * Cf::PART; i += 32 * CW) {
-        double s = 0.0;
+      if constexpr (L::NSLOT > 0) {
+        __threadfence_block();
+        __syncwarp();
+        int arrived = 0;
+        if (lane == 0) arrived = atomicAdd(&cnt[slot], 1);
+        arrived = __shfl_sync(0xffffffffu, arrived, 0);
+        if (arrived == CW - 1) {
+          // the last warp of this slab sums the slot in warp order
+          __threadfence_block();
+          for (int i = lane; i < 2 * Cf::PART; i += 32) {
+            double s = 0.0;
 #pragma unroll
-        for (int w = 0; w < CW; ++w) s += red_s[w * 2 * Cf::PART + i];
-        dst[i] = s;
-      }
-      if (cond)
-        for (int i = tid; i < RP; i += 32 * CW) {
-          float s = 0.f;
+            for (int w = 0; w < CW; ++w) s += rs[w * 2 * Cf::PART + i];
+            dst[i] = s;
+          }
+          if (cond)
+            for (int i = lane; i < RP; i += 32) {
+              float s = 0.f;
 #pragma unroll
-          for (int w = 0; w < CW; ++w) s += red_e[w * RP + i];
-          p.rpart[(size_t)u * RP + i] = s;
+              for (int w = 0; w < CW; ++w) s += re[w * RP + i];
+              p.rpart[(size_t)u * RP + i] = s;
+            }
+          __syncwarp();
+          if (lane == 0) {
+            cnt[slot] = 0;
+            __threadfence_block();
+            mbar_arrive(&done[slot]);
+          }
         }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(redr);
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(redf);
+        if (!wait_phase(redf, nred & 1u, abort, p.status)) break;
+        for (int i = tid; i < 2 * Cf::PART; i += 32 * CW) {
+          double s = 0.0;
+#pragma unroll
+          for (int w = 0; w < CW; ++w) s += rs[w * 2 * Cf::PART + i];
+          dst[i] = s;
+        }
+        if (cond)
+          for (int i = tid; i < RP; i += 32 * CW) {
+            float s = 0.f;
+#pragma unroll
+            for (int w = 0; w < CW; ++w) s += re[w * RP + i];
+            p.rpart[(size_t)u * RP + i] = s;
+          }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(redr);
+      }
       ++nred;
     }
   }
 }
 
 // ===========================================================================
-// thin_apply_bulk
+// thin_apply_bulk: O = C^2 T B, W update, long-side energies
 // ===========================================================================
 template <int RP, typename TG, typename TM, typename TW>
 struct ApplyBulk {
-  static constexpr int CH = (RP >= 32 ? 4096 : 2048) / RP;
-  static constexpr int NS = 3;
+  static constexpr int CW = RP == 32 ? 4 : 8;
+  static constexpr int NP = 2;                 // producer warps
+  static constexpr int BT = 32 * (CW + NP);
+  static constexpr int MINB = RP == 8 || RP == 2 ? 2 : 1;  // resident CTAs the registers allow
+  static constexpr int CH = RP <= 4 ? 1024 : RP <= 16 ? 256 : 128;
+  static constexpr int NS = RP == 32 ? 3 : 4;
+  static constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH), PW = pitch_elems<TW>(CH);
   static constexpr int OFF_W = opnd_bytes<TM>(RP, CH);
   static constexpr int OFF_E = OFF_W + opnd_bytes<TW>(RP, CH);
   static constexpr int OFF_G = OFF_E + CH * 4;  // Nesterov only
   static constexpr int BYTES_NO_G = (OFF_G + 127) / 128 * 128;
   static constexpr int BYTES_G = (OFF_G + opnd_bytes<TG>(RP, CH) + 127) / 128 * 128;
   __host__ __device__ static constexpr int stage_bytes(bool nest) { return nest ? BYTES_G : BYTES_NO_G; }
+  static constexpr int NCOL = TCfg<RP>::MMA ? CH / CW : 0;  // columns of one consumer warp per stage
   __host__ __device__ static constexpr int smem(bool nest) {
-    return NS * stage_bytes(nest) + NS * (int)sizeof(StageInfo) + 2 * NS * 8 + 16 + 128;
+    return NS * stage_bytes(nest) + NS * (int)sizeof(StageInfo) + 2 * NS * 8 + 16 + CW * 2 * NCOL * 8 +
+           128;
   }
 };
 
-template <int RP, typename TG, typename TM, typename TW>
-__global__ void __launch_bounds__(BT) thin_apply_bulk(const __grid_constant__ ThinParams p) {
+// 32 long-side columns c .. c + 31 inside the stage (RP >= 8).  Lane (g, t)
+// holds B rows 4 kb + t at column slots c + 4g + e (wide) or c + 8e + g
+// (tall); wide computes D = T B (output rows 8 bo + g, columns c + 8t ..
+// c + 8t + 7), tall D = B^T T^T (output rows 8 bo + 2t, +1 of column
+// c + 8e + g).  FULL = false predicates the columns against c1.
+template <int RP, typename TG, typename TM, typename TW, bool TALL, bool ON, bool COND, bool FULL,
+          bool NEST>
+__device__ __forceinline__ void apply_step_mma(const TM* Ms, const TG* Gs, const TW* Ws,
+                                               const double* wrow, const double* Tg, TW* Wg, float* Ug,
+                                               float* ecg, int64_t n, int cs, int c, int c1, float mu,
+                                               float lr, float decay, float inv_mc, float eps,
+                                               bool zero, int g, int t, int lane) {
   using L = ApplyBulk<RP, TG, TM, TW>;
-  using Cf = TCfg<RP>;
-  constexpr int CH = L::CH, NS = L::NS;
+  constexpr int NB = TCfg<RP>::NB, KB = TCfg<RP>::KB;
+  bool okc[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) okc[e] = FULL || (TALL ? c + 8 * e + g : c + 4 * g + e) < c1;
+  const bool okq = FULL || c + 4 * g < c1;  // wide: this lane's column quad is inside
+  double wd[4];
+  if constexpr (ON) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) wd[e] = wrow[TALL ? 8 * e + g : 4 * g + e];  // zero past c1
+  }
+  double acc[NB][4][2];
+#pragma unroll
+  for (int bo = 0; bo < NB; ++bo)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[bo][e][0] = acc[bo][e][1] = 0.0;
+  float sq[4] = {0.f, 0.f, 0.f, 0.f};
+  // k blocks one at a time: B rows 4 kb + t of this lane's four column slots
+#pragma unroll
+  for (int kb = 0; kb < KB; ++kb) {
+    float mv[4], gv[4];
+    if constexpr (!TALL) {
+      if (okq) {
+        El<TM>::ld4(Ms + (4 * kb + t) * L::PM + cs + 4 * g, mv);
+        if (NEST) El<TG>::ld4(Gs + (4 * kb + t) * L::PG + cs + 4 * g, gv);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mv[e] = gv[e] = 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int o = (cs + 8 * e + g) * RP + 4 * kb + t;
+        mv[e] = okc[e] ? El<TM>::ld1(Ms + o) : 0.f;
+        gv[e] = (NEST && okc[e]) ? El<TG>::ld1(Gs + o) : 0.f;
+      }
+    }
+    double tf[NB];
+#pragma unroll
+    for (int bo = 0; bo < NB; ++bo) tf[bo] = __ldg(Tg + (bo * KB + kb) * 32 + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double m = (double)mv[e];
+      const double bv = NEST ? fma((double)mu, m, (double)gv[e]) : m;
+      const double x = ON ? wd[e] * bv : bv;
+      if constexpr (COND) sq[e] = fmaf(mv[e], mv[e], sq[e]);
+#pragma unroll
+      for (int bo = 0; bo < NB; ++bo) {
+        if constexpr (TALL)
+          dmma(acc[bo][e][0], acc[bo][e][1], x, tf[bo]);
+        else
+          dmma(acc[bo][e][0], acc[bo][e][1], tf[bo], x);
+      }
+    }
+  }
+  float ce[4];
+  if constexpr (COND) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v = sq[e];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      ce[e] = v;
+    }
+  }
+  if constexpr (!TALL) {
+#pragma unroll
+    for (int bo = 0; bo < NB; ++bo)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = 8 * bo + g, cl = cs + 8 * t + 4 * h;
+        if (FULL || c + 8 * t + 4 * h < c1) {
+          float w4[4], o4[4];
+          El<TW>::ld4(Ws + row * L::PW + cl, w4);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o4[e] = zero ? 0.f : (float)acc[bo][e][h];
+            w4[e] = decay * w4[e] - lr * o4[e];
+          }
+          El<TW>::st4(Wg + (int64_t)row * n + c + 8 * t + 4 * h, w4);
+          if (Ug) El<float>::st4(Ug + (int64_t)row * n + c + 8 * t + 4 * h, o4);
+        }
+      }
+  } else {
+#pragma unroll
+    for (int bo = 0; bo < NB; ++bo)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (!okc[e]) continue;
+        const int row0 = 8 * bo + 2 * t;
+        float w0, w1;
+        El<TW>::ld2(Ws + (cs + 8 * e + g) * RP + row0, w0, w1);
+        const float o0 = zero ? 0.f : (float)acc[bo][e][0];
+        const float o1 = zero ? 0.f : (float)acc[bo][e][1];
+        const int64_t go = (int64_t)(c + 8 * e + g) * RP + row0;
+        El<TW>::st2(Wg + go, decay * w0 - lr * o0, decay * w1 - lr * o1);
+        if (Ug) El<float>::st2(Ug + go, o0, o1);
+      }
+  }
+  if constexpr (COND) {
+    if (t == 0) {
+      if constexpr (!TALL) {
+        if (FULL || c + 4 * g < c1) El<float>::st4(ecg + c + 4 * g, ce);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (okc[e]) ecg[c + 8 * e + g] = ce[e];
+      }
+    }
+  }
+}
+
+// Four long-side columns c .. c + 3 owned by one lane (RP == r <= 4).
+template <int RP, typename TG, typename TM, typename TW, bool TALL, bool ON, bool COND, bool NEST>
+__device__ __forceinline__ void apply_step_small(const TM* Ms, const TG* Gs, const TW* Ws,
+                                                 const float* Es, const double* Tg, TW* Wg, float* Ug,
+                                                 float* ecg, int64_t n, int cs, int c, float mu,
+                                                 float lr, float decay, float inv_mc, float eps,
+                                                 bool zero) {
+  using L = ApplyBulk<RP, TG, TM, TW>;
+  float mv[RP][4], gv[RP][4], wv[RP][4];
+  if constexpr (!TALL) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i) {
+      El<TM>::ld4(Ms + i * L::PM + cs, mv[i]);
+      if (NEST) El<TG>::ld4(Gs + i * L::PG + cs, gv[i]);
+      El<TW>::ld4(Ws + i * L::PW + cs, wv[i]);
+    }
+  } else {
+    float fm[4 * RP], fg[4 * RP], fw[4 * RP];
+#pragma unroll
+    for (int s = 0; s < RP; ++s) {
+      El<TM>::ld4(Ms + cs * RP + 4 * s, &fm[4 * s]);
+      if (NEST) El<TG>::ld4(Gs + cs * RP + 4 * s, &fg[4 * s]);
+      El<TW>::ld4(Ws + cs * RP + 4 * s, &fw[4 * s]);
+    }
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        mv[i][e] = fm[e * RP + i];
+        gv[i][e] = NEST ? fg[e * RP + i] : 0.f;
+        wv[i][e] = fw[e * RP + i];
+      }
+  }
+  double wd[4];
+  if constexpr (ON) {
+    const float4 e4 = *reinterpret_cast<const float4*>(Es + cs);
+    wd[0] = (double)col_weight(e4.x, inv_mc, eps);
+    wd[1] = (double)col_weight(e4.y, inv_mc, eps);
+    wd[2] = (double)col_weight(e4.z, inv_mc, eps);
+    wd[3] = (double)col_weight(e4.w, inv_mc, eps);
+  }
+  double tm[RP][RP];
+#pragma unroll
+  for (int i = 0; i < RP; ++i)
+#pragma unroll
+    for (int k = 0; k < RP; ++k) tm[i][k] = __ldg(Tg + i * RP + k);
+  float ov[RP][4], ce[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    double x[RP];
+    float sq = 0.f;
+#pragma unroll
+    for (int k = 0; k < RP; ++k) {
+      const double m = (double)mv[k][e];
+      const double bv = NEST ? fma((double)mu, m, (double)gv[k][e]) : m;
+      x[k] = ON ? wd[e] * bv : bv;
+      if constexpr (COND) sq = fmaf(mv[k][e], mv[k][e], sq);
+    }
+    ce[e] = sq;
+#pragma unroll
+    for (int i = 0; i < RP; ++i) {
+      double y = 0.0;
+#pragma unroll
+      for (int k = 0; k < RP; ++k) y = fma(tm[i][k], x[k], y);
+      ov[i][e] = zero ? 0.f : (float)y;
+      wv[i][e] = decay * wv[i][e] - lr * ov[i][e];
+    }
+  }
+  if constexpr (!TALL) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i) {
+      El<TW>::st4(Wg + (int64_t)i * n + c, wv[i]);
+      if (Ug) El<float>::st4(Ug + (int64_t)i * n + c, ov[i]);
+    }
+  } else {
+    float fw[4 * RP], fo[4 * RP];
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        fw[e * RP + i] = wv[i][e];
+        fo[e * RP + i] = ov[i][e];
+      }
+#pragma unroll
+    for (int s = 0; s < RP; ++s) {
+      El<TW>::st4(Wg + (int64_t)c * RP + 4 * s, &fw[4 * s]);
+      if (Ug) El<float>::st4(Ug + (int64_t)c * RP + 4 * s, &fo[4 * s]);
+    }
+  }
+  if constexpr (COND) El<float>::st4(ecg + c, ce);
+}
+
+template <int RP, typename TG, typename TM, typename TW, bool TALL, bool ON, bool COND, bool NEST>
+__device__ __forceinline__ void apply_stage(const TM* Ms, const TG* Gs, const TW* Ws, const float* Es,
+                                            double* wmine, const double* Tg, TW* Wg, float* Ug,
+                                            float* ecg, int64_t n, int c0, int c1, float mu, float lr,
+                                            float decay, float inv_mc, float eps, bool zero,
+                                            int warp, int lane) {
+  using L = ApplyBulk<RP, TG, TM, TW>;
+  constexpr int CW = L::CW;
+  if constexpr (TCfg<RP>::MMA) {
+    const int g = lane >> 2, t = lane & 3;
+    if (ON) stage_weights<32, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
+    int k = 0;
+    for (int c = c0 + 32 * warp; c < c1; c += 32 * CW, ++k) {
+      if (c + 32 <= c1)
+        apply_step_mma<RP, TG, TM, TW, TALL, ON, COND, true, NEST>(Ms, Gs, Ws, wmine + 32 * k, Tg, Wg, Ug, ecg,
+                                                             n, c - c0, c, c1, mu, lr, decay, inv_mc, eps,
+                                                             zero, g, t, lane);
+      else
+        apply_step_mma<RP, TG, TM, TW, TALL, ON, COND, false, NEST>(Ms, Gs, Ws, wmine + 32 * k, Tg, Wg, Ug,
+                                                              ecg, n, c - c0, c, c1, mu, lr, decay, inv_mc,
+                                                              eps, zero, g, t, lane);
+    }
+  } else {
+    for (int c = c0 + 4 * (lane + 32 * warp); c < c1; c += 4 * 32 * CW)
+      apply_step_small<RP, TG, TM, TW, TALL, ON, COND, NEST>(Ms, Gs, Ws, Es, Tg, Wg, Ug, ecg, n, c - c0, c, mu,
+                                                       lr, decay, inv_mc, eps, zero);
+  }
+}
+
+template <int RP, typename TG, typename TM, typename TW>
+__global__ void __launch_bounds__(ApplyBulk<RP, TG, TM, TW>::BT, ApplyBulk<RP, TG, TM, TW>::MINB)
+    thin_apply_bulk(const __grid_constant__ ThinParams p) {
+  using L = ApplyBulk<RP, TG, TM, TW>;
+  constexpr int CH = L::CH, NS = L::NS, CW = L::CW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
@@ -559,6 +1074,7 @@ __global__ void __launch_bounds__(BT) thin_apply_bulk(const __grid_constant__ Th
   uint64_t* full = reinterpret_cast<uint64_t*>(info + NS);
   uint64_t* empty = full + NS;
   volatile int* abort = reinterpret_cast<volatile int*>(empty + NS);
+  double* wsm = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(empty + NS) + 16);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -571,22 +1087,21 @@ __global__ void __launch_bounds__(BT) thin_apply_bulk(const __grid_constant__ Th
   }
   __syncthreads();
 
-  if (warp == CW) {
+  if (warp >= CW) {
     produce<RP, CH, NS, TG, TM, TW, 1>(p, stages, stage_bytes, L::OFF_G, L::OFF_W, L::OFF_E, info, full,
-                                       empty, abort, p.counters + 1);
+                                       empty, abort, warp - CW, L::NP);
     return;
   }
 
   const float mu = p.mu, lr = p.lr, decay = p.decay, eps = p.eps;
   const bool nest = p.nesterov != 0;
-  constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH), PW = pitch_elems<TW>(CH);
   int stage = 0;
   uint32_t ph = 0;
   for (;;) {
-    if (!mbar_wait_bounded(&full[stage], ph, abort, p.status, WAIT_NS)) break;
+    if (!wait_phase(&full[stage], ph, abort, p.status)) break;
     const StageInfo& si = info[stage];
     if (si.u < 0) break;
-    const int c0 = si.c0, c1 = si.c1, f = si.f;
+    const int c0 = si.c0, c1 = si.c1;
     const bool on = si.on != 0, zero = si.zero != 0;
     const float inv_mc = si.inv_mc;
     const bool tall = si.mt.rows > si.mt.cols;
@@ -600,196 +1115,28 @@ __global__ void __launch_bounds__(BT) thin_apply_bulk(const __grid_constant__ Th
     const TW* Ws = reinterpret_cast<const TW*>(base + L::OFF_W);
     const float* Es = reinterpret_cast<const float*>(base + L::OFF_E);
     const TG* Gs = reinterpret_cast<const TG*>(base + L::OFF_G);
-    const double* Tg = p.T + (size_t)f * RP * RP;
-
-    if constexpr (Cf::MMA) {
-      constexpr int NB = Cf::NB, KB = Cf::KB;
-      const int g = lane >> 2, t = lane & 3;
-      // 32 columns per warp step; see thin_apply for the fragment layout
-      for (int c = c0 + 32 * warp; c < c1; c += 32 * CW) {
-        const int cs = c - c0;
-        float mv[KB][4], gv[KB][4];
-        bool okc[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) okc[e] = (tall ? c + 8 * e + g : c + 4 * g + e) < c1;
-        if (!tall) {
-          const bool ok = c + 4 * g < c1;
-#pragma unroll
-          for (int kb = 0; kb < KB; ++kb) {
-            const int row = 4 * kb + t;
-            if (ok) {
-              El<TM>::ld4(Ms + row * PM + cs + 4 * g, mv[kb]);
-              if (nest) El<TG>::ld4(Gs + row * PG + cs + 4 * g, gv[kb]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) mv[kb][e] = gv[kb][e] = 0.f;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int o = (cs + 8 * e + g) * RP + 4 * kb + t;
-              mv[kb][e] = okc[e] ? El<TM>::ld1(Ms + o) : 0.f;
-              if (nest) gv[kb][e] = okc[e] ? El<TG>::ld1(Gs + o) : 0.f;
-            }
-        }
-        float ce[4];
-        double x[KB][4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = tall ? c + 8 * e + g : c + 4 * g + e;
-          const double w =
-              on ? (okc[e] ? (double)col_weight(Es[col - c0], inv_mc, eps) : 0.0) : 1.0;
-          float sq = 0.f;
-#pragma unroll
-          for (int kb = 0; kb < KB; ++kb) {
-            const double m = (double)mv[kb][e];
-            x[kb][e] = w * (nest ? fma((double)mu, m, (double)gv[kb][e]) : m);
-            sq = fmaf(mv[kb][e], mv[kb][e], sq);
-          }
-          sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-          sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-          ce[e] = sq;
-        }
-        double acc[NB][4][2];
-#pragma unroll
-        for (int bo = 0; bo < NB; ++bo)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[bo][e][0] = acc[bo][e][1] = 0.0;
-#pragma unroll
-        for (int kb = 0; kb < KB; ++kb) {
-          double tf[NB];
-#pragma unroll
-          for (int bo = 0; bo < NB; ++bo) tf[bo] = __ldg(Tg + (bo * KB + kb) * 32 + lane);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-#pragma unroll
-            for (int bo = 0; bo < NB; ++bo) {
-              if (tall)
-                dmma(acc[bo][e][0], acc[bo][e][1], x[kb][e], tf[bo]);
-              else
-                dmma(acc[bo][e][0], acc[bo][e][1], tf[bo], x[kb][e]);
-            }
-        }
-        if (!tall) {
-          // acc[bo][e][h] is column c + 8t + 4h + e of row 8 bo + g
-#pragma unroll
-          for (int bo = 0; bo < NB; ++bo)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int row = 8 * bo + g, col0 = c + 8 * t + 4 * h;
-              if (col0 < c1) {
-                float w4[4], o4[4];
-                El<TW>::ld4(Ws + row * PW + (col0 - c0), w4);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  o4[e] = zero ? 0.f : (float)acc[bo][e][h];
-                  w4[e] = decay * w4[e] - lr * o4[e];
-                }
-                El<TW>::st4(Wg + (int64_t)row * n + col0, w4);
-                if (Ug) El<float>::st4(Ug + (int64_t)row * n + col0, o4);
-              }
-            }
-        } else {
-          // acc[bo][e][h] is row 8 bo + 2t + h of column c + 8e + g
-#pragma unroll
-          for (int bo = 0; bo < NB; ++bo)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (!okc[e]) continue;
-              const int col = c + 8 * e + g, row0 = 8 * bo + 2 * t;
-              float w0, w1;
-              El<TW>::ld2(Ws + (col - c0) * RP + row0, w0, w1);
-              const float o0 = zero ? 0.f : (float)acc[bo][e][0];
-              const float o1 = zero ? 0.f : (float)acc[bo][e][1];
-              El<TW>::st2(Wg + (int64_t)col * RP + row0, decay * w0 - lr * o0, decay * w1 - lr * o1);
-              if (Ug) El<float>::st2(Ug + (int64_t)col * RP + row0, o0, o1);
-            }
-        }
-        if (cond && t == 0)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = tall ? c + 8 * e + g : c + 4 * g + e;
-            if (okc[e]) ecg[col] = ce[e];
-          }
-      }
+    const double* Tg = p.T + (size_t)si.f * RP * RP;
+#define DM_APPLY_STAGE(TALL_, ON_, COND_)                                                              \
+  do {                                                                                                \
+    if (nest)                                                                                         \
+      apply_stage<RP, TG, TM, TW, TALL_, ON_, COND_, true>(Ms, Gs, Ws, Es, wsm + warp * 2 * L::NCOL, \
+                                                           Tg, Wg, Ug, ecg, n, c0, c1, mu, lr, decay, \
+                                                           inv_mc, eps, zero, warp, lane);            \
+    else                                                                                              \
+      apply_stage<RP, TG, TM, TW, TALL_, ON_, COND_, false>(Ms, Gs, Ws, Es, wsm + warp * 2 * L::NCOL, \
+                                                            Tg, Wg, Ug, ecg, n, c0, c1, mu, lr, decay, \
+                                                            inv_mc, eps, zero, warp, lane);           \
+  } while (0)
+    if (tall) {
+      if (on) DM_APPLY_STAGE(true, true, true);
+      else if (cond) DM_APPLY_STAGE(true, false, true);
+      else DM_APPLY_STAGE(true, false, false);
     } else {
-      // RP == r <= 4: lane owns columns c .. c + 3
-      for (int c = c0 + 4 * (lane + 32 * warp); c < c1; c += 4 * 32 * CW) {
-        const int cs = c - c0;
-        float mv[RP][4], gv[RP][4], wv[RP][4];
-        if (!tall) {
-#pragma unroll
-          for (int i = 0; i < RP; ++i) {
-            El<TM>::ld4(Ms + i * PM + cs, mv[i]);
-            if (nest) El<TG>::ld4(Gs + i * PG + cs, gv[i]);
-            El<TW>::ld4(Ws + i * PW + cs, wv[i]);
-          }
-        } else {
-          float fm[4 * RP], fg[4 * RP], fw[4 * RP];
-#pragma unroll
-          for (int s = 0; s < RP; ++s) {
-            El<TM>::ld4(Ms + cs * RP + 4 * s, &fm[4 * s]);
-            if (nest) El<TG>::ld4(Gs + cs * RP + 4 * s, &fg[4 * s]);
-            El<TW>::ld4(Ws + cs * RP + 4 * s, &fw[4 * s]);
-          }
-#pragma unroll
-          for (int i = 0; i < RP; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              mv[i][e] = fm[e * RP + i];
-              gv[i][e] = nest ? fg[e * RP + i] : 0.f;
-              wv[i][e] = fw[e * RP + i];
-            }
-        }
-        float ov[RP][4], ce[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const double w = on ? (double)col_weight(Es[cs + e], inv_mc, eps) : 1.0;
-          double x[RP];
-          float sq = 0.f;
-#pragma unroll
-          for (int k = 0; k < RP; ++k) {
-            const double m = (double)mv[k][e];
-            x[k] = w * (nest ? fma((double)mu, m, (double)gv[k][e]) : m);
-            sq = fmaf(mv[k][e], mv[k][e], sq);
-          }
-          ce[e] = sq;
-#pragma unroll
-          for (int i = 0; i < RP; ++i) {
-            double y = 0.0;
-#pragma unroll
-            for (int k = 0; k < RP; ++k) y = fma(__ldg(Tg + i * RP + k), x[k], y);
-            ov[i][e] = zero ? 0.f : (float)y;
-            wv[i][e] = decay * wv[i][e] - lr * ov[i][e];
-          }
-        }
-        if (!tall) {
-#pragma unroll
-          for (int i = 0; i < RP; ++i) {
-            El<TW>::st4(Wg + (int64_t)i * n + c, wv[i]);
-            if (Ug) El<float>::st4(Ug + (int64_t)i * n + c, ov[i]);
-          }
-        } else {
-          float fw[4 * RP], fo[4 * RP];
-#pragma unroll
-          for (int i = 0; i < RP; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              fw[e * RP + i] = wv[i][e];
-              fo[e * RP + i] = ov[i][e];
-            }
-#pragma unroll
-          for (int s = 0; s < RP; ++s) {
-            El<TW>::st4(Wg + (int64_t)c * RP + 4 * s, &fw[4 * s]);
-            if (Ug) El<float>::st4(Ug + (int64_t)c * RP + 4 * s, &fo[4 * s]);
-          }
-        }
-        if (cond) El<float>::st4(ecg + c, ce);
-      }
+      if (on) DM_APPLY_STAGE(false, true, true);
+      else if (cond) DM_APPLY_STAGE(false, false, true);
+      else DM_APPLY_STAGE(false, false, false);
     }
+#undef DM_APPLY_STAGE
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
     if (++stage == NS) {
@@ -822,21 +1169,28 @@ cudaError_t launch_bulk_rp(ThinParams& p, int nsm, cudaStream_t st) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(thin_apply_bulk<RP, TG, TM, TW>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, LA::smem(true));
+    // shared memory over L1 for the staging rings
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(thin_gram_bulk<RP, TG, TM>,
+                               cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(thin_apply_bulk<RP, TG, TM, TW>,
+                               cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    occ_g = resident(thin_gram_bulk<RP, TG, TM>, BT, LG::SMEM);
-    occ_a[0] = resident(thin_apply_bulk<RP, TG, TM, TW>, BT, LA::smem(false));
-    occ_a[1] = resident(thin_apply_bulk<RP, TG, TM, TW>, BT, LA::smem(true));
+    occ_g = resident(thin_gram_bulk<RP, TG, TM>, LG::BT, LG::SMEM);
+    occ_a[0] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(false));
+    occ_a[1] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(true));
     configured = dev;
   }
   const bool nest = p.nesterov != 0;
   p.grid_gram = std::min(p.units, nsm * occ_g);
   p.grid_apply = std::min(p.units, nsm * occ_a[nest ? 1 : 0]);
-  thin_gram_bulk<RP, TG, TM><<<p.grid_gram, BT, LG::SMEM, st>>>(p);
+  thin_gram_bulk<RP, TG, TM><<<p.grid_gram, LG::BT, LG::SMEM, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_thin_iterate(p, st);
   if (e != cudaSuccess) return e;
-  thin_apply_bulk<RP, TG, TM, TW><<<p.grid_apply, BT, LA::smem(nest), st>>>(p);
+  thin_apply_bulk<RP, TG, TM, TW><<<p.grid_apply, LA::BT, LA::smem(nest), st>>>(p);
   return cudaGetLastError();
 }
 
