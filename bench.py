@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload large_batch|large_batch_quarter|gpt2_small|square1024|
-                               lora_r2|lora_r8|lora_r32]
+                               lora_r2|lora_r8|lora_r32|vec_w1|vec_w2|vec_w8|vec_w32|vec_w128]
 
 One step = one optimizer step (momentum, normalisation, five Newton-Schulz
 iterations, scale, decay, apply) over every matrix of the workload.  The
@@ -55,6 +55,13 @@ def workload_spec(name):
                     lr={2: 0.018, 8: 0.010, 32: 0.010}.get(r, 0.01), wd=0.0, moonshot=False,
                     seed=4, desc=f"224 LoRA projections r={r} (A r x 4096, B 4096 x r), "
                                  "fp32 momentum, bf16 weights, Dimuon")
+    if name.startswith("vec_w"):
+        w = int(name[5:])
+        return dict(shapes=workloads.vector_shapes(w), cond=False, mdt="fp32", lr=0.02, wd=0.0,
+                    moonshot=False, seed=5, nesterov=1, vec_len=workloads.VECTOR_LENGTH,
+                    desc=f"{workloads.VECTOR_COUNT} 1-D parameters of {workloads.VECTOR_LENGTH} "
+                         f"variables at width {w} (zero-padded), fp32 momentum, bf16 weights, "
+                         "Muon with Nesterov")
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -245,7 +252,10 @@ def main():
     torch.manual_seed(spec["seed"] + 1000 + rank)
     G_host, G, W, M, ER, EC = [], [], [], [], [], []
     for (r, c) in shapes:
-        g = torch.from_numpy(rng.standard_normal((r, c), dtype=np.float32)).to(bf)
+        gn = rng.standard_normal((r, c), dtype=np.float32)
+        if spec.get("vec_len"):  # 1-D parameter: zero gradient in the padding cells
+            gn.reshape(-1)[spec["vec_len"]:] = 0.0
+        g = torch.from_numpy(gn).to(bf)
         G_host.append(g.pin_memory())
         G.append(g.to(dev))
         W.append((0.02 * torch.randn((r, c), device=dev, dtype=torch.float32)).to(bf))
@@ -255,7 +265,7 @@ def main():
     mats = [dm.dm_matrix(W[i], G[i], M[i], ER[i], EC[i]) for i in range(len(shapes))]
     hp = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"],
                                scale_mode=dm.DM_SCALE_MOONSHOT if spec["moonshot"]
-                               else dm.DM_SCALE_NONE)
+                               else dm.DM_SCALE_NONE, nesterov=spec.get("nesterov", 0))
     step_fn = dm.dm_dimuon_step if spec["cond"] else dm.dm_muon_step
     ws = torch.empty(dm.dm_workspace_size(mats, hp, int(spec["cond"])), dtype=torch.uint8,
                      device=dev)
@@ -303,7 +313,7 @@ def main():
     # schedule over a 1-step schedule, on the launch stream
     reps = max(2, min(args.steps, 5))
     hp1 = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"], ns_steps=1,
-                                scale_mode=hp.scale_mode)
+                                scale_mode=hp.scale_mode, nesterov=hp.nesterov)
     g1 = capture(hp1)
     g1.replay()
     t5 = timed(graph, reps) / reps

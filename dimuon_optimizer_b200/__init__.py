@@ -227,3 +227,16 @@ def check(status):
     if status != DM_OK:
         raise DimuonError(status)
     return status
+
+
+def vector_matrix_shape(length, width):
+    """Shape (rows, width) of the matrix a 1-D parameter of `length`
+    variables is laid out in ("From PCG to Muon", section 6 "Muon
+    Reshaping"): the variables in order, row-major, the cells past the end
+    zero.  Give the library the padded matrices with zero gradient in the
+    padding: the padded momentum cells then stay zero, and the padded weight
+    cells (which the update does write) are simply not read back."""
+    length, width = int(length), int(width)
+    if length < 1 or width < 1:
+        raise ValueError("length and width must be positive")
+    return (-(-length // width), width)

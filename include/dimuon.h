@@ -191,12 +191,15 @@ dm_status_t dm_read_device_status(const void* workspace, void* stream,
  * every input and output.
  *   - Groups whose dm_workspace_size exceeds DM_NOALLOC_MAX_BYTES are
  *     rejected with DM_ERR_WORKSPACE before any device work.  Thin factors
- *     (short side <= DM_THIN_MAX) need no scratch, so any number of them fits.
+ *     (short side <= DM_THIN_MAX) need a little scratch per 512-2048 long-side
+ *     columns (fp64 Gram partials) and per factor; 448 LoRA factors of rank
+ *     32 and width 4096 need about 22 MB.
  *   - The first call on a device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress); make that first call before
  *     any stream capture.
  *   - Every call shares the one array and leaves its contents behind; the step
- *     zeroes its status word itself and needs nothing else zeroed.  Calls whose
+ *     zeroes its header (status word, slab counters) itself and needs nothing
+ *     else zeroed.  Calls whose
  *     device work overlaps (different streams or threads without ordering)
  *     race on the array: order them on the device.
  *   - device_status_out (nullable, device int32) receives the step's device

@@ -8,5 +8,5 @@ from .dimuon_oracle import (  # noqa: F401
     SCALE_NONE, HParams, StepResult, conditioning, dimuon_step, energies,
     f32, frobenius_normalise, momentum_update, muon_step, newton_schulz,
     optimizer_step, polar_factor_svd, round_bf16, scale_factor, store_round,
-    top_column_share,
+    top_column_share, vector_matrix_shape, vector_step, vector_to_matrix, matrix_to_vector,
 )

@@ -298,6 +298,55 @@ def dimuon_step(W_prev, G, M_prev, e_row_prev, e_col_prev, hp: HParams,
 # ----------------------------------------------------------------------------
 # Reference quantities used by the pins (not part of the step itself).
 # ----------------------------------------------------------------------------
+# Muon on a 1-D variable ([PCG2Muon] section 6, "Muon Reshaping")
+# ----------------------------------------------------------------------------
+def vector_matrix_shape(length: int, width: int) -> tuple[int, int]:
+    """Shape of the matrix a length-`length` vector is laid out in at a given
+    width: rows = ceil(length / width), the variables kept in their order
+    (row-major), the cells past the end zero."""
+    if length < 1 or width < 1:
+        raise ValueError("length and width must be positive")
+    return -(-length // width), width
+
+
+def vector_to_matrix(v, width: int) -> np.ndarray:
+    """The vector in row-major order in a rows x width matrix, zero-padded
+    ([PCG2Muon] section 6: the remaining cells are padded with 0)."""
+    v = np.asarray(v, np.float64).reshape(-1)
+    rows, cols = vector_matrix_shape(v.size, width)
+    X = np.zeros(rows * cols)
+    X[:v.size] = v
+    return X.reshape(rows, cols)
+
+
+def matrix_to_vector(X, length: int) -> np.ndarray:
+    """The first `length` cells in row-major order: the padding is dropped
+    after the update ([PCG2Muon] section 6: restored after the update)."""
+    return np.asarray(X, np.float64).reshape(-1)[:length].copy()
+
+
+def vector_step(w_prev, g, m_prev, width: int, hp: HParams, *, conditioned: bool = False,
+                e_row_prev=None, e_col_prev=None, momentum_dtype: str = "fp32",
+                weight_dtype: str = "fp32") -> StepResult:
+    """One step on a 1-D variable: lay W, G and M out at the given width with
+    zero padding, run optimizer_step on the matrices, return the first
+    len(w) entries of W_t, M_t and O_t.  The padded gradient cells are zero,
+    so the padded momentum cells stay zero; the padded weight cells are
+    dropped.  Dimuon energies (when conditioned) belong to the padded matrix
+    and are returned for it."""
+    w_prev = np.asarray(w_prev, np.float64).reshape(-1)
+    L = w_prev.size
+    res = optimizer_step(vector_to_matrix(w_prev, width), vector_to_matrix(g, width),
+                         vector_to_matrix(m_prev, width), hp, conditioned=conditioned,
+                         e_row_prev=e_row_prev, e_col_prev=e_col_prev,
+                         momentum_dtype=momentum_dtype, weight_dtype=weight_dtype)
+    return StepResult(W=matrix_to_vector(res.W, L), M=matrix_to_vector(res.M, L),
+                      O=matrix_to_vector(res.O, L), e_row=res.e_row, e_col=res.e_col,
+                      nonfinite=res.nonfinite,
+                      extras={"matrix": res, "padded_M": res.M.reshape(-1)[L:].copy()})
+
+
+# ----------------------------------------------------------------------------
 def polar_factor_svd(X) -> np.ndarray:
     """U V^T from a LAPACK SVD: the exact orthogonal polar factor that the
     iteration approximates ([MuonNote], "Newton-Schulz orthogonalisation":

@@ -16,7 +16,7 @@ import torch
 import dimuon_optimizer_b200 as dm
 import oracle as orc
 import workloads
-from gpu_harness import (TOL_BF16, TOL_FP32, Group, rel_fro, run_gpu_step, step_and_compare,
+from gpu_harness import (TOL_BF16, TOL_FP32, Group, oracle_hp, rel_fro, run_gpu_step, step_and_compare,
                          to_dev, to_host)
 
 pytestmark = [pytest.mark.gpu,
@@ -315,3 +315,41 @@ def test_lora_batch_twenty_steps(r):
             er = to_host(grp.er[1])
             assert np.all(er[dead] == 0.0) if t <= 5 else True
     assert rel_fro(to_host(grp.W[1]), free["W"]) < 3e-2
+
+
+# --------------------------------------------------------------------------
+# 1-D parameters laid out at widths 1 .. 128 ("From PCG to Muon", section 6)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("width", [1, 2, 8, 32, 128])
+def test_vector_reshape(width):
+    """Vectors of ragged lengths at each width, Muon with momentum and
+    Nesterov: the first `length` cells of M_t, O_t, W_t match the oracle's
+    vector step (teacher-forced, three steps) and the padded momentum cells
+    stay exactly zero."""
+    lengths = [1000, 4099, 65537]
+    shapes = [dm.vector_matrix_shape(L, width) for L in lengths]
+    grp = Group(shapes, BF, BF, F32, cond=False, seed=31 + width)
+    prec = dm.DM_PREC_FP32  # width 128 takes the fp32 Newton-Schulz kernels
+    hp = hparams(prec, nesterov=1, weight_decay=0.01)
+    h = oracle_hp(hp)
+    rng = np.random.default_rng(width)
+    ws = None
+    for step in range(3):
+        grads = []
+        for (r, c), L in zip(shapes, lengths):
+            g = np.zeros(r * c)
+            g[:L] = rng.standard_normal(L)
+            grads.append(g.reshape(r, c))
+        before = [(to_host(grp.W[i]).reshape(-1)[:L], to_host(grp.M[i]).reshape(-1)[:L])
+                  for i, L in enumerate(lengths)]
+        ws, G = run_gpu_step(grp, grads, hp, ws)
+        for i, L in enumerate(lengths):
+            w0, m0 = before[i]
+            g_host = to_host(G[i]).reshape(-1)[:L]
+            res = orc.vector_step(w0, g_host, m0, width, h, momentum_dtype="fp32",
+                                  weight_dtype="bf16")
+            Mg = to_host(grp.M[i]).reshape(-1)
+            Og = to_host(grp.upd[i]).reshape(-1)[:L]
+            np.testing.assert_array_equal(Mg[:L], res.M)
+            assert np.all(Mg[L:] == 0.0)
+            assert rel_fro(Og, res.O) <= TOL_FP32, (width, L, rel_fro(Og, res.O))

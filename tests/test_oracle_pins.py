@@ -474,3 +474,55 @@ def test_nesterov_without_momentum_is_plain():
     a = orc.muon_step(W, G, Z, orc.HParams(mu=0.0, nesterov=True))
     b = orc.muon_step(W, G, Z, orc.HParams(mu=0.0))
     np.testing.assert_array_equal(a.O, b.O)
+
+
+# --------------------------------------------------------------------------
+# Muon on a 1-D variable (From PCG to Muon, section 6 "Muon Reshaping")
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("width,length", [(1, 37), (2, 37), (8, 37), (32, 37), (128, 37), (5, 40)])
+def test_vector_layout_brute_force(width, length):
+    """Row-major layout with zero padding and the padding dropped after the
+    update, checked against the pure-Python step on a matrix filled by hand;
+    the padded momentum cells stay exactly zero."""
+    rng = np.random.default_rng(width * 100 + length)
+    w = rng.standard_normal(length) * 0.02
+    g = rng.standard_normal(length)
+    m = rng.standard_normal(length)
+    rows = (length + width - 1) // width
+
+    def by_hand(v):
+        return [[float(v[i * width + j]) if i * width + j < length else 0.0 for j in range(width)]
+                for i in range(rows)]
+
+    hp = orc.HParams(mu=0.9, lr=0.05, weight_decay=0.01)
+    h = hp.as_f32()
+    want = brute_force_step(by_hand(w), by_hand(g), by_hand(m), h.mu, h.lr, h.weight_decay,
+                            h.a, h.b, h.c, h.ns_steps, h.cond_eps, h.scale_coef, False)
+    flat = lambda X: np.array(X, np.float64).reshape(-1)[:length]  # noqa: E731
+    got = orc.vector_step(w, g, m, width, hp)
+    np.testing.assert_array_equal(got.M, np.float32(flat(want[1])))
+    np.testing.assert_allclose(got.O, flat(want[2]), rtol=1e-10, atol=1e-13)
+    assert np.all(got.extras["padded_M"] == 0.0)
+    assert got.W.shape == (length,) and got.O.shape == (length,)
+
+
+@pytest.mark.parametrize("width", [1, 4096])
+def test_vector_width_one_closed_form(width, golden):
+    """A width-1 layout (and a single row, width >= length) normalises the whole
+    vector: O = kappa p^5(1) B / ||B|| with B = G + mu M_t under Nesterov
+    (From PCG to Muon, section 6: width 1 normalises the vector; momentum
+    and Nesterov stay in the step)."""
+    g5 = golden("ns5_coefficients.json")
+    rng = np.random.default_rng(41)
+    L = 1000
+    w, g, m = rng.standard_normal(L) * 0.02, rng.standard_normal(L), rng.standard_normal(L)
+    hp = orc.HParams(mu=0.95, lr=0.02, nesterov=True)
+    h = hp.as_f32()
+    got = orc.vector_step(w, g, m, width, hp)
+    Mt = np.float32(h.mu * m + g).astype(np.float64)
+    B = g + h.mu * Mt
+    # the step carries its coefficients through float32 like the library
+    assert (h.a, h.b, h.c) == tuple(float(np.float32(g5[k])) for k in "abc")
+    k = quintic_scalar(1.0, h.a, h.b, h.c, g5["iterations"])
+    np.testing.assert_array_equal(got.M, Mt)
+    np.testing.assert_allclose(got.O, k * B / np.linalg.norm(B), rtol=1e-12, atol=1e-15)

@@ -23,6 +23,10 @@ Recipes (all host-side numpy, float64 draws, then cast by the caller):
   B) are scaled by s_j^2 and drawn fresh N(0,1) each step; for 16 chosen rows
   of each B the gradient is zero for steps 1-5 and scaled by 1e-3 from step 6.
   Seed 4.
+* 1-D parameters ("From PCG to Muon", section 6 "Muon Reshaping"): 64
+  vectors of 262,267 variables (2^18 + 123, so the last row is ragged),
+  each laid out row-major at width 1, 2, 8, 32 or 128 with the cells past the
+  end zero; gradients N(0,1) on the variables and zero in the padding, seed 5.
 * weights: W ~ N(0, 0.02^2) from default_rng(seed + 1000).
 """
 from __future__ import annotations
@@ -31,6 +35,8 @@ import numpy as np
 
 GPT2_LAYERS = 12
 GPT2_WIDTH = 768
+VECTOR_LENGTH = (1 << 18) + 123
+VECTOR_COUNT = 64
 
 
 def toy_lora_factor():
@@ -123,3 +129,22 @@ CONFIGS = {
     "large_batch": "8x4096^2 + 4x4096x14336 + 4x14336x4096 bf16",
     "lora": "224 LoRA projections (A r x 4096, B 4096 x r), Dimuon, 20 steps",
 }
+
+
+def vector_shapes(width, count=VECTOR_COUNT, length=VECTOR_LENGTH):
+    """count vectors of `length` variables, each in a ceil(length / width) x
+    width matrix (row-major, zero-padded)."""
+    return [(-(-length // width), width)] * count
+
+
+def vector_grads(width, count=VECTOR_COUNT, length=VECTOR_LENGTH, seed=5):
+    """N(0,1) gradients on the variables, zero in the padding cells, laid out
+    as vector_shapes(width)."""
+    rng = np.random.default_rng(seed)
+    rows = -(-length // width)
+    out = []
+    for _ in range(count):
+        g = np.zeros(rows * width)
+        g[:length] = rng.standard_normal(length)
+        out.append(g.reshape(rows, width))
+    return out
