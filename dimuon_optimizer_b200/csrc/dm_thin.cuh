@@ -21,7 +21,9 @@ struct TCfg {
   static constexpr int KB = MMA ? RP / 4 : 1;       // 4-wide k steps
   static constexpr int NUB = NB * (NB + 1) / 2;     // upper-triangle 8x8 blocks
   static constexpr int PART = MMA ? NUB * 64 : RP * RP;  // doubles per Gram partial
-  static constexpr int SLD = RP + 1;                // padded r x r row (iteration)
+  // padded r x r row of the iteration's shared matrices: RP + 4 doubles puts
+  // the MMA fragment reads of 16 lanes on 16 distinct 8-byte bank pairs
+  static constexpr int SLD = RP >= 16 ? RP + 4 : RP + 1;
   // long-side columns per slab (work unit of thin_gram / thin_apply)
   static constexpr int SLAB = RP <= 4 ? 2048 : RP <= 16 ? 512 : 1024;
   // the next step's loads are issued before the current step computes

@@ -385,24 +385,42 @@ struct IterSmem {
   double red[32];
 };
 
-// C = A * B for RP x RP fp64 matrices in shared memory (padded rows).
+// Threads of the one-CTA-per-factor iteration (RP = 16, 32).
+constexpr int IT = 256;
+constexpr int IW = IT / 32;
+
+// C = A * B for RP x RP fp64 matrices in shared memory (padded rows); each
+// warp interleaves the k chains of its 8x8 output blocks.
 template <int RP>
 __device__ __forceinline__ void mm(double (*C)[TCfg<RP>::SLD], double (*A)[TCfg<RP>::SLD],
                                    double (*B)[TCfg<RP>::SLD]) {
   if constexpr (TCfg<RP>::MMA) {
-    constexpr int NB = TCfg<RP>::NB;
+    constexpr int NB = TCfg<RP>::NB, NBLK = NB * NB, PER = (NBLK + IW - 1) / IW;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    for (int blk = warp; blk < NB * NB; blk += TW) {
-      const int rb = blk / NB, cb = blk % NB;
-      double d0 = 0.0, d1 = 0.0;
+    double d[PER][2];
 #pragma unroll
-      for (int kb = 0; kb < RP / 4; ++kb)
-        dmma(d0, d1, A[rb * 8 + g][kb * 4 + t], B[kb * 4 + t][cb * 8 + g]);
-      C[rb * 8 + g][cb * 8 + 2 * t] = d0;
-      C[rb * 8 + g][cb * 8 + 2 * t + 1] = d1;
+    for (int q = 0; q < PER; ++q) d[q][0] = d[q][1] = 0.0;
+#pragma unroll
+    for (int kb = 0; kb < RP / 4; ++kb)
+#pragma unroll
+      for (int q = 0; q < PER; ++q) {
+        const int blk = warp + q * IW;
+        if (blk < NBLK) {
+          const int rb = blk / NB, cb = blk % NB;
+          dmma(d[q][0], d[q][1], A[rb * 8 + g][kb * 4 + t], B[kb * 4 + t][cb * 8 + g]);
+        }
+      }
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int blk = warp + q * IW;
+      if (blk < NBLK) {
+        const int rb = blk / NB, cb = blk % NB;
+        C[rb * 8 + g][cb * 8 + 2 * t] = d[q][0];
+        C[rb * 8 + g][cb * 8 + 2 * t + 1] = d[q][1];
+      }
     }
   } else {
-    for (int idx = threadIdx.x; idx < RP * RP; idx += TT) {
+    for (int idx = threadIdx.x; idx < RP * RP; idx += IT) {
       const int i = idx / RP, j = idx % RP;
       double s = 0.0;
 #pragma unroll
@@ -555,7 +573,7 @@ __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ 
 }
 
 template <int RP>
-__global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinParams p) {
+__global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinParams p) {
   using Cf = TCfg<RP>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   IterSmem<RP>& s = *reinterpret_cast<IterSmem<RP>*>(smem_raw);
@@ -567,7 +585,7 @@ __global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinP
   const int u0 = p.starts[f], nu = p.starts[f + 1] - p.starts[f];
 
   // S_1, S_2: slab partials in slab order; lower 8x8 blocks mirror upper ones
-  for (int idx = tid; idx < RP * RP; idx += TT) {
+  for (int idx = tid; idx < RP * RP; idx += IT) {
     const int i = idx / RP, j = idx % RP;
     int src;
     if constexpr (Cf::MMA) {
@@ -604,7 +622,7 @@ __global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinP
   }
   // A_0 = R S_1 R, H = R S_2 R; ||X_0||^2 = tr A_0
   double tr = 0.0;
-  for (int idx = tid; idx < RP * RP; idx += TT) {
+  for (int idx = tid; idx < RP * RP; idx += IT) {
     const int i = idx / RP, j = idx % RP;
     const double rr = s.R[i] * s.R[j];
     s.G[i][j] *= rr;
@@ -615,7 +633,7 @@ __global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinP
   const bool finite = isfinite(s2);
   const bool valid = finite && s2 >= NORM2_FLOOR;  // else the update is zero
   const double inv_s2 = valid ? 1.0 / s2 : 0.0;
-  for (int idx = tid; idx < RP * RP; idx += TT) {
+  for (int idx = tid; idx < RP * RP; idx += IT) {
     const int i = idx / RP, j = idx % RP;
     s.A[i][j] = valid ? s.G[i][j] * inv_s2 : 0.0;
     s.P[i][j] = i == j ? 1.0 : 0.0;
@@ -624,13 +642,13 @@ __global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinP
   const double a = p.a, b = p.b, c = p.c;
   for (int it = 0; it < p.ns_steps; ++it) {
     mm<RP>(s.Q, s.A, s.A);  // Q = A A
-    for (int idx = tid; idx < RP * RP; idx += TT) {
+    for (int idx = tid; idx < RP * RP; idx += IT) {
       const int i = idx / RP, j = idx % RP;
       s.Q[i][j] = c * s.Q[i][j] + b * s.A[i][j] + (i == j ? a : 0.0);
     }
     __syncthreads();
     mm<RP>(s.S, s.Q, s.P);  // P <- Q P
-    for (int idx = tid; idx < RP * RP; idx += TT) s.P[idx / RP][idx % RP] = s.S[idx / RP][idx % RP];
+    for (int idx = tid; idx < RP * RP; idx += IT) s.P[idx / RP][idx % RP] = s.S[idx / RP][idx % RP];
     __syncthreads();
     mm<RP>(s.S, s.Q, s.A);  // A <- Q A Q
     mm<RP>(s.A, s.S, s.Q);
@@ -638,11 +656,11 @@ __global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinP
   // ||X_5||^2 s^2 = tr(P A_0 P^T); ||R X_5 C||^2 s^2 = sum_i R_i^2 (P H P^T)_ii
   mm<RP>(s.S, s.P, s.G);
   double nx = 0.0;
-  for (int idx = tid; idx < RP * RP; idx += TT) nx += s.S[idx / RP][idx % RP] * s.P[idx / RP][idx % RP];
+  for (int idx = tid; idx < RP * RP; idx += IT) nx += s.S[idx / RP][idx % RP] * s.P[idx / RP][idx % RP];
   nx = block_sum_d(nx, s.red);
   mm<RP>(s.Q, s.P, s.H);
   double ny = 0.0;
-  for (int idx = tid; idx < RP * RP; idx += TT) {
+  for (int idx = tid; idx < RP * RP; idx += IT) {
     const int i = idx / RP;
     ny += s.R[i] * s.R[i] * s.Q[i][idx % RP] * s.P[i][idx % RP];
   }
@@ -656,7 +674,7 @@ __global__ void __launch_bounds__(TT) thin_iterate(const __grid_constant__ ThinP
   // T = f R P R; for RP >= 8 in MMA fragment order: T(8 bo + l/4, 4 kb + l%4)
   // at ((bo * KB + kb) * 32 + l)
   double* T = p.T + (size_t)f * RP * RP;
-  for (int idx = tid; idx < RP * RP; idx += TT) {
+  for (int idx = tid; idx < RP * RP; idx += IT) {
     int i, j;
     if constexpr (Cf::MMA) {
       const int l = idx & 31, fr = idx >> 5;
@@ -1034,7 +1052,7 @@ cudaError_t launch_iter_rp(const ThinParams& p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = dev;
   }
-  thin_iterate<RP><<<p.count, TT, iter_bytes, st>>>(p);
+  thin_iterate<RP><<<p.count, IT, iter_bytes, st>>>(p);
   return cudaGetLastError();
 }
 

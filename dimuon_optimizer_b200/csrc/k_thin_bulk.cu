@@ -335,7 +335,7 @@ struct GramBulk {
   static constexpr int CW = RP == 32 ? 4 : 8;  // consumer warps
   static constexpr int NP = 2;                 // producer warps
   static constexpr int BT = 32 * (CW + NP);
-  static constexpr int MINB = RP == 8 || RP == 16 ? 3 : 1;  // resident CTAs the registers allow
+  static constexpr int MINB = RP == 8 || RP == 16 ? 3 : RP == 32 ? 2 : 1;  // resident CTAs
   static constexpr int CH = RP <= 4 ? 1024 : RP == 8 ? 256 : RP == 16 ? 128 : 64;
   static constexpr int NS = 4;
   // reduction at the end of a run of slabs: NSLOT > 0 = asynchronous (each
@@ -798,7 +798,7 @@ struct ApplyBulk {
   static constexpr int CW = RP == 32 ? 4 : 8;
   static constexpr int NP = 2;                 // producer warps
   static constexpr int BT = 32 * (CW + NP);
-  static constexpr int MINB = RP == 8 || RP == 2 ? 2 : 1;  // resident CTAs the registers allow
+  static constexpr int MINB = RP == 8 || RP == 2 || RP == 32 ? 2 : 1;  // resident CTAs
   static constexpr int CH = RP <= 4 ? 1024 : RP <= 16 ? 256 : 128;
   static constexpr int NS = RP == 32 ? 3 : 4;
   static constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH), PW = pitch_elems<TW>(CH);
