@@ -591,9 +591,10 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     for (int k = 1; k <= hp->ns_steps; ++k)
       for (int ph = 0; ph < 3; ++ph)
         for (size_t b = 0; b < big.size(); b += TC_MAX) {
-          // CTA pairs when there are at least two 256 x 256 tiles per pair
           const int pair_tiles = build(b, ph, k, TC2_BM, TC2_BN);
-          bool pair = pair_tiles >= nsm;
+          // CTA pairs (256 x 256 tiles) measured at least as fast as single
+          // CTAs on every workload tried, including one 1024^2 matrix
+          bool pair = true;
           if (hp->debug_flags & DM_DBG_TC_PAIR) pair = true;
           if (hp->debug_flags & DM_DBG_TC_SINGLE) pair = false;
           if (pair) {
