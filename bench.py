@@ -2,7 +2,7 @@
 """Throughput of the B200 Muon / Dimuon step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large_batch|large_batch_quarter|gpt2_small|square1024|
+                    [--workload large_batch|large_batch_dimuon|large_batch_quarter|gpt2_small|square1024|
                                lora_r2|lora_r8|lora_r32|vec_w1|vec_w2|vec_w8|vec_w32|vec_w128]
 
 One step = one optimizer step (momentum, normalisation, five Newton-Schulz
@@ -38,6 +38,10 @@ def workload_spec(name):
         return dict(shapes=workloads.large_batch_shapes(), cond=False, mdt="bf16", lr=0.02,
                     wd=0.0, moonshot=False, seed=3,
                     desc="8x4096^2 + 4x4096x14336 + 4x14336x4096 bf16, Muon, 5 NS5 iterations")
+    if name == "large_batch_dimuon":  # the large batch through the Dimuon path
+        return dict(shapes=[(4096, 4096)] * 8 + [(4096, 14336)] * 4 + [(14336, 4096)] * 4,
+                    cond=True, mdt="bf16", lr=0.02, wd=0.0, moonshot=False, seed=3,
+                    desc="8x4096^2 + 4x4096x14336 + 4x14336x4096 bf16, Dimuon, 5 NS5 iterations")
     if name == "large_batch_quarter":  # same shapes, a quarter of the matrices
         return dict(shapes=[(4096, 4096)] * 2 + [(4096, 14336), (14336, 4096)], cond=False,
                     mdt="bf16", lr=0.02, wd=0.0, moonshot=False, seed=3,
@@ -85,8 +89,8 @@ def step_bytes(spec):
 # DRAM traffic of the tensor-core product per launch (ncu dram__bytes_read.sum +
 # dram__bytes_write.sum), valid only for the kernel build it was taken from:
 # profiles/tc_ns_product_pair_large_batch_quarter.md (quarter batch x 4).
-TRAFFIC_CAPTURED = {"large_batch": 2846e6}
-TRAFFIC_BUILD = "7698eb153da99050"
+TRAFFIC_CAPTURED = {"large_batch": 2842e6}
+TRAFFIC_BUILD = "7a4c787a77da2048"
 TRAFFIC_SOURCES = ["k_ns_tc2.cu", "dm_tc_epilogue.cuh", "dm_sm100.cuh"]
 
 

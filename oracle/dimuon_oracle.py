@@ -51,6 +51,9 @@ the repository's design notes):
     takes the momentum-and-Nesterov combination B_t; its formula is not
     printed, this is the standard look-ahead form).  M_t itself, and the
     energies Dimuon reads, are unchanged.
+  * 1-D variables ([PCG2Muon], section 6 "Muon Reshaping"): the vector keeps
+    its order in a row-major ceil(L/w) x w matrix with the cells past the end
+    zero; "restored after the update" is read as keeping the first L cells.
 
 Parity pins for every function here live in tests/test_oracle_pins.py.
 """
