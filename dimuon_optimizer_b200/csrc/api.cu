@@ -121,8 +121,10 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
     p.n = (int)std::max(p.rows, p.cols);
     p.thin = p.m <= DM_THIN_MAX && !(hp->debug_flags & DM_DBG_NO_THIN);
     if (!p.thin) {
-      p.ldx = (int64_t)round_up((size_t)p.cols, 8);
-      p.ldm = (int64_t)round_up((size_t)p.m, 8);
+      // rows padded to whole 64-element chunks, so a chunked (3-D) operand
+      // map never reads past the end of a row
+      p.ldx = (int64_t)round_up((size_t)p.cols, 64);
+      p.ldm = (int64_t)round_up((size_t)p.m, 64);
       p.k1_rt = (int)ceil_div(p.rows, K1_ROWS);
       p.k1_ct = (int)ceil_div(p.cols, K1_COLS);
       if (L.tc)  // enough (sum x^2, sum y^2) slots for either tensor-core kernel
@@ -211,22 +213,45 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 matrix [outer][inner] with leading dimension ld (elements); 64 x 64
-// boxes with the 128-byte swizzle the UMMA descriptors expect.
-bool make_map(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_t ld) {
+// bf16 matrix [outer][inner] with leading dimension ld (elements); boxes of
+// 64 inner x `rows` outer elements with the 128-byte swizzle the UMMA
+// descriptors expect (64 x 64 for the single-CTA kernel, 64 x 128 for one
+// CTA's K-major operand slab in the pair kernel).
+bool make_map(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_t ld, int rows = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {64, (cuuint32_t)rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same matrix seen as 64-element chunks of its rows: dims (element in
+// chunk, row, chunk), box 64 x 64 rows x 2 chunks.  One copy then fills the
+// 128 x 64 MN-major operand slab of a pair CTA in the layout two 64 x 64
+// boxes give ([chunk][row][64], 8 KB per chunk).  Needs ld >= the chunk count
+// x 64 (rows are padded to whole chunks).  Returns false if the driver does
+// not take the map; the caller then falls back to two 2-D boxes.
+bool make_map3(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || ld < (int64_t)round_up((size_t)inner, 64)) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)outer, (cuuint64_t)ceil_div(inner, 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), 128};
+  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Operand maps of one matrix's buffers (X[0], X[1], A, B): 64 x 64 boxes,
+// 64 x 128 boxes, and chunked 3-D maps (valid when has3).
 struct MatMaps {
-  CUtensorMap X[2], A, B;
+  CUtensorMap m64[4], m128[4], m3[4];
+  bool has3;
 };
 
 std::mutex g_cache_mu;
@@ -260,10 +285,16 @@ bool get_maps(const Layout& L, uint8_t* ws, int dev, std::vector<MatMaps>& out) 
   for (size_t i = 0; i < L.mats.size(); ++i) {
     const MatPlan& p = L.mats[i];
     if (p.thin) continue;
-    for (int b = 0; b < 2; ++b)
-      if (!make_map(&out[i].X[b], ws + p.off_X[b], p.cols, p.rows, p.ldx)) return false;
-    if (!make_map(&out[i].A, ws + p.off_A, p.m, p.m, p.ldm)) return false;
-    if (!make_map(&out[i].B, ws + p.off_B, p.m, p.m, p.ldm)) return false;
+    MatMaps& mm = out[i];
+    mm.has3 = true;
+    for (int b = 0; b < 4; ++b) {
+      uint8_t* base = ws + (b < 2 ? p.off_X[b] : b == 2 ? p.off_A : p.off_B);
+      const int64_t inner = b < 2 ? p.cols : p.m, outer = b < 2 ? p.rows : p.m;
+      const int64_t ld = b < 2 ? p.ldx : p.ldm;
+      if (!make_map(&mm.m64[b], base, inner, outer, ld, 64)) return false;
+      if (!make_map(&mm.m128[b], base, inner, outer, ld, 128)) return false;
+      mm.has3 = mm.has3 && make_map3(&mm.m3[b], base, inner, outer, ld);
+    }
   }
   std::lock_guard<std::mutex> lk(g_cache_mu);
   if (g_map_cache.size() > 64) g_map_cache.clear();
@@ -563,7 +594,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     if (!get_maps(L, ws, dev, maps)) return DM_ERR_CUDA;
     const int nsm = sm_count(dev);
     static thread_local TcParams pt;
-    auto build = [&](size_t b, int ph, int k, int bm, int bn) {
+    auto build = [&](size_t b, int ph, int k, int bm, int bn, bool pair) {
       std::memset(&pt, 0, sizeof(pt));
       pt.status = status;
       pt.lr = hp->lr;
@@ -576,11 +607,20 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
         const OperandSrc src = fill_gemm(tm.g, p, mats[p.idx], hp, ws, ph, k, cond != 0,
                                          kappa_of(hp, p.rows, p.cols), bm, bn);
         const MatMaps& mm = maps[p.idx];
-        auto pick = [&](int buf) -> const CUtensorMap& {
-          return buf < 2 ? mm.X[buf] : (buf == 2 ? mm.A : mm.B);
+        // single-CTA kernel: 64 x 64 boxes; pair kernel: one 64 x 128 box per
+        // K-major slab, one chunked box per MN-major slab (two 64 x 64 boxes
+        // if the driver took no chunked map)
+        auto pick = [&](int buf, bool mn, int box3_flag) -> const CUtensorMap& {
+          if (!pair) return mm.m64[buf];
+          if (!mn) return mm.m128[buf];
+          if (mm.has3) {
+            tm.g.flags |= box3_flag;
+            return mm.m3[buf];
+          }
+          return mm.m64[buf];
         };
-        tm.ta = pick(src.a_buf);
-        tm.tb = pick(src.b_buf);
+        tm.ta = pick(src.a_buf, (tm.g.flags & GF_A_MN) != 0, GF_A_BOX3);
+        tm.tb = pick(src.b_buf, (tm.g.flags & GF_B_MN) != 0, GF_B_BOX3);
         pt.starts[pt.count++] = tiles;
         tiles += gemm_tile_count(tm.g, bm, bn);
       }
@@ -591,7 +631,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     for (int k = 1; k <= hp->ns_steps; ++k)
       for (int ph = 0; ph < 3; ++ph)
         for (size_t b = 0; b < big.size(); b += TC_MAX) {
-          const int pair_tiles = build(b, ph, k, TC2_BM, TC2_BN);
+          const int pair_tiles = build(b, ph, k, TC2_BM, TC2_BN, true);
           // CTA pairs (256 x 256 tiles) measured at least as fast as single
           // CTAs on every workload tried, including one 1024^2 matrix
           bool pair = true;
@@ -600,7 +640,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
           if (pair) {
             DM_CUDA(launch_tc_pair(pt, std::min(pair_tiles, nsm / 2), s));
           } else {
-            const int tiles = build(b, ph, k, TC_BM, TC_BN);
+            const int tiles = build(b, ph, k, TC_BM, TC_BN, false);
             DM_CUDA(launch_tc(pt, std::min(tiles, nsm), s));
           }
           if (k == hp->ns_steps && ph == PH_GEMM)

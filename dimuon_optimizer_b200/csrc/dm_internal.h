@@ -120,7 +120,9 @@ struct GemmMat {
   int wdt;                // weight dtype
   float coef_acc, coef_aux, kappa;
 };
-enum { GF_A_MN = 1, GF_B_MN = 2, GF_SYM = 4, GF_N_FAST = 8 };
+// GF_A_BOX3 / GF_B_BOX3: the pair kernel's MN-major operand map is the
+// chunked 3-D map (one copy per 128 x 64 slab)
+enum { GF_A_MN = 1, GF_B_MN = 2, GF_SYM = 4, GF_N_FAST = 8, GF_A_BOX3 = 16, GF_B_BOX3 = 32 };
 
 // fp32 SIMT products
 constexpr int SIMT_MAX = 120;
@@ -142,7 +144,7 @@ struct SimtParams {
 // tcgen05 products (bf16 operands, fp32 accumulation in TMEM)
 constexpr int TC_BM = 128, TC_BN = 256, TC_BK = 64;
 struct TcMat {
-  CUtensorMap ta;   // A-operand map, box 64 x 64 bf16, 128-byte swizzle
+  CUtensorMap ta;   // A-operand map, bf16, 128-byte swizzle (box per kernel: see the host)
   CUtensorMap tb;   // B-operand map
   GemmMat g;
 };

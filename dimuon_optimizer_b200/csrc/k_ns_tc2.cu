@@ -5,9 +5,11 @@
 // "Muon Optimizer 정리", "Why orthogonalise"), with 256 x 256 output tiles
 // computed by a pair of CTAs (a cluster of 2 on two SMs):
 //   - each CTA loads its own 128 rows of the A operand and its own 128
-//     columns of the B operand (TMA, 64 x 64 boxes, 128-byte swizzle, no
-//     multicast), 32 KB per stage, 6 stages; both CTAs' loads complete on
-//     the leader's "full" barrier;
+//     columns of the B operand (TMA, 128-byte swizzle, no multicast; one
+//     16 KB copy per operand slab: a 64 x 128 box for K-major slabs, a
+//     64 x 64 x 2 box of the chunked 3-D map for MN-major ones), 32 KB per
+//     stage, 6 stages; both CTAs' loads complete on the leader's "full"
+//     barrier;
 //   - one thread of the leader issues tcgen05.mma.cta_group::2 with M = 256,
 //     N = 256: the accumulator's rows 0..127 live in the leader's tensor
 //     memory, rows 128..255 in the peer's; per k-block the MMA reads half of
@@ -41,6 +43,7 @@ constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t TMEM_COLS = 512;              // two 128-lane x 256-column accumulators
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
 constexpr uint64_t FORCED_LIMIT_NS = 20000000ull;   // forced-timeout hook: 20 ms
@@ -125,6 +128,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
         const Tile tl = decode_tile(p, t);
         const TcMat& mt = p.mats[tl.g];
         const int a_mn = mt.g.flags & GF_A_MN, b_mn = mt.g.flags & GF_B_MN;
+        const int a3 = mt.g.flags & GF_A_BOX3, b3 = mt.g.flags & GF_B_BOX3;
         const int m0 = tl.tm * PAIR_BM + (int)rank * HALF;
         const int n0 = tl.tn * PAIR_BN + (int)rank * HALF;
         const int nkb = (mt.g.K + TC_BK - 1) / TC_BK;
@@ -143,17 +147,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
           }
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
           const int k0 = kb * TC_BK;
-#pragma unroll
-          for (int q = 0; q < HALF / 64; ++q) {
-            if (a_mn)
+          // one copy per 128 x 64 slab where the map allows: K-major slabs
+          // take a 64 x 128 box, MN-major ones the chunked 3-D box; the
+          // copy engine's per-copy cost makes 8 KB boxes too slow to feed
+          // the tensor pipe
+          if (!a_mn)
+            tma_load_2d_pair(sa, &mt.ta, bar, k0, m0);
+          else if (a3)
+            tma_load_3d_pair(sa, &mt.ta, bar, 0, k0, m0 / 64);
+          else
+            for (int q = 0; q < HALF / 64; ++q)
               tma_load_2d_pair(sa + q * BOX_BYTES, &mt.ta, bar, m0 + 64 * q, k0);
-            else
-              tma_load_2d_pair(sa + q * BOX_BYTES, &mt.ta, bar, k0, m0 + 64 * q);
-            if (b_mn)
+          if (!b_mn)
+            tma_load_2d_pair(sb, &mt.tb, bar, k0, n0);
+          else if (b3)
+            tma_load_3d_pair(sb, &mt.tb, bar, 0, k0, n0 / 64);
+          else
+            for (int q = 0; q < HALF / 64; ++q)
               tma_load_2d_pair(sb + q * BOX_BYTES, &mt.tb, bar, n0 + 64 * q, k0);
-            else
-              tma_load_2d_pair(sb + q * BOX_BYTES, &mt.tb, bar, k0, n0 + 64 * q);
-          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
