@@ -89,8 +89,8 @@ def step_bytes(spec):
 # DRAM traffic of the tensor-core product per launch (ncu dram__bytes_read.sum +
 # dram__bytes_write.sum), valid only for the kernel build it was taken from:
 # profiles/tc_ns_product_pair_large_batch_quarter.md (quarter batch x 4).
-TRAFFIC_CAPTURED = {"large_batch": 2842e6}
-TRAFFIC_BUILD = "7a4c787a77da2048"
+TRAFFIC_CAPTURED = {"large_batch": 2902e6}
+TRAFFIC_BUILD = "6c1826947c21ad68"
 TRAFFIC_SOURCES = ["k_ns_tc2.cu", "dm_tc_epilogue.cuh", "dm_sm100.cuh"]
 
 

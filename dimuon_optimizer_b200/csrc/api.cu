@@ -230,17 +230,22 @@ bool make_map(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_t
 }
 
 // The same matrix seen as 64-element chunks of its rows: dims (element in
-// chunk, row, chunk), box 64 x 64 rows x 2 chunks.  One copy then fills the
-// 128 x 64 MN-major operand slab of a pair CTA in the layout two 64 x 64
-// boxes give ([chunk][row][64], 8 KB per chunk).  Needs ld >= the chunk count
-// x 64 (rows are padded to whole chunks).  Returns false if the driver does
-// not take the map; the caller then falls back to two 2-D boxes.
-bool make_map3(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_t ld) {
+// chunk, row, chunk), box 64 x `rows` rows x `chunks` chunks, laid out
+// [chunk][row][64] in shared memory (the layout 64-wide 2-D boxes stacked
+// chunk by chunk give).  Used for one CTA's operand slab in one copy:
+// MN-major slabs (2 chunks of 64 output rows/columns x BK k rows) and
+// K-major slabs (BK / 64 chunks of k x 128 rows).  Needs ld >= the chunk
+// count x 64 (rows are padded to whole chunks); the padding is read, so a
+// K-major (chunks along k) map is only built when the inner extent is a
+// multiple of 64.  Returns false if the driver does not take the map; the
+// caller then falls back to 2-D boxes.
+bool make_map3(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_t ld, int rows,
+               int chunks) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || ld < (int64_t)round_up((size_t)inner, 64)) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)outer, (cuuint64_t)ceil_div(inner, 64)};
   cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), 128};
-  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, (cuuint32_t)chunks};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -248,10 +253,11 @@ bool make_map3(CUtensorMap* map, void* ptr, int64_t inner, int64_t outer, int64_
 }
 
 // Operand maps of one matrix's buffers (X[0], X[1], A, B): 64 x 64 boxes,
-// 64 x 128 boxes, and chunked 3-D maps (valid when has3).
+// 64 x 128 boxes, chunked 3-D maps for MN-major slabs (valid when has3) and
+// for K-major slabs of 128 k (valid when hask3[b]).
 struct MatMaps {
-  CUtensorMap m64[4], m128[4], m3[4];
-  bool has3;
+  CUtensorMap m64[4], m128[4], m3[4], k3[4];
+  bool has3, hask3[4];
 };
 
 std::mutex g_cache_mu;
@@ -293,7 +299,9 @@ bool get_maps(const Layout& L, uint8_t* ws, int dev, std::vector<MatMaps>& out) 
       const int64_t ld = b < 2 ? p.ldx : p.ldm;
       if (!make_map(&mm.m64[b], base, inner, outer, ld, 64)) return false;
       if (!make_map(&mm.m128[b], base, inner, outer, ld, 128)) return false;
-      mm.has3 = mm.has3 && make_map3(&mm.m3[b], base, inner, outer, ld);
+      const int bk = tc_pair_bk();
+      mm.has3 = mm.has3 && make_map3(&mm.m3[b], base, inner, outer, ld, bk, 2);
+      mm.hask3[b] = bk == 128 && inner % 64 == 0 && make_map3(&mm.k3[b], base, inner, outer, ld, 128, 2);
     }
   }
   std::lock_guard<std::mutex> lk(g_cache_mu);
@@ -607,12 +615,18 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
         const OperandSrc src = fill_gemm(tm.g, p, mats[p.idx], hp, ws, ph, k, cond != 0,
                                          kappa_of(hp, p.rows, p.cols), bm, bn);
         const MatMaps& mm = maps[p.idx];
-        // single-CTA kernel: 64 x 64 boxes; pair kernel: one 64 x 128 box per
-        // K-major slab, one chunked box per MN-major slab (two 64 x 64 boxes
-        // if the driver took no chunked map)
+        // single-CTA kernel: 64 x 64 boxes; pair kernel: one copy per slab
+        // (chunked maps) where the maps allow, else 64 x 128 boxes (K-major)
+        // or 64 x 64 boxes (MN-major)
         auto pick = [&](int buf, bool mn, int box3_flag) -> const CUtensorMap& {
           if (!pair) return mm.m64[buf];
-          if (!mn) return mm.m128[buf];
+          if (!mn) {
+            if (mm.hask3[buf]) {
+              tm.g.flags |= box3_flag;
+              return mm.k3[buf];
+            }
+            return mm.m128[buf];
+          }
           if (mm.has3) {
             tm.g.flags |= box3_flag;
             return mm.m3[buf];

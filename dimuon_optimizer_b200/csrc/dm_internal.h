@@ -120,8 +120,8 @@ struct GemmMat {
   int wdt;                // weight dtype
   float coef_acc, coef_aux, kappa;
 };
-// GF_A_BOX3 / GF_B_BOX3: the pair kernel's MN-major operand map is the
-// chunked 3-D map (one copy per 128 x 64 slab)
+// GF_A_BOX3 / GF_B_BOX3: the pair kernel's operand map is a chunked 3-D map
+// (one copy per operand slab of a stage)
 enum { GF_A_MN = 1, GF_B_MN = 2, GF_SYM = 4, GF_N_FAST = 8, GF_A_BOX3 = 16, GF_B_BOX3 = 32 };
 
 // fp32 SIMT products
@@ -249,6 +249,7 @@ int tc_smem_bytes();
 constexpr int TC2_BM = 256, TC2_BN = 256;  // CTA-pair output tile
 cudaError_t launch_tc_pair(const TcParams& p, int pairs, cudaStream_t s);
 int tc_pair_smem_bytes();
+int tc_pair_bk();  // k per stage of the pair kernel (box shapes of its maps)
 cudaError_t launch_thin_setup(const ThinSetupParams& p, cudaStream_t s);
 cudaError_t launch_thin(ThinParams& p, int nsm, cudaStream_t s);
 cudaError_t launch_thin_iterate(const ThinParams& p, cudaStream_t s);

@@ -5,11 +5,11 @@
 // "Muon Optimizer 정리", "Why orthogonalise"), with 256 x 256 output tiles
 // computed by a pair of CTAs (a cluster of 2 on two SMs):
 //   - each CTA loads its own 128 rows of the A operand and its own 128
-//     columns of the B operand (TMA, 128-byte swizzle, no multicast; one
-//     16 KB copy per operand slab: a 64 x 128 box for K-major slabs, a
-//     64 x 64 x 2 box of the chunked 3-D map for MN-major ones), 32 KB per
-//     stage, 6 stages; both CTAs' loads complete on the leader's "full"
-//     barrier;
+//     columns of the B operand for k blocks of 128 (TMA, 128-byte swizzle,
+//     no multicast; one 32 KB copy per operand slab through chunked 3-D
+//     maps: 2 chunks of 64 k x 128 rows for K-major slabs, 2 chunks of 64
+//     columns x 128 k for MN-major ones), 64 KB per stage, 3 stages; both
+//     CTAs' loads complete on the leader's "full" barrier;
 //   - one thread of the leader issues tcgen05.mma.cta_group::2 with M = 256,
 //     N = 256: the accumulator's rows 0..127 live in the leader's tensor
 //     memory, rows 128..255 in the peer's; per k-block the MMA reads half of
@@ -34,11 +34,17 @@ using namespace tcepi;
 constexpr int PAIR_BM = 256;                     // output tile rows (both CTAs)
 constexpr int PAIR_BN = 256;                     // output tile columns
 constexpr int HALF = 128;                        // rows (A) / columns (B) per CTA
-constexpr int STAGES = 6;
+// k per stage.  128 (3 stages of 64 KB) measured faster than 64 (6 stages of
+// 32 KB) on every workload tried: one 32 KB copy per operand slab keeps the
+// copy engine well below its per-copy limit (large batch 39.0 -> 35.6 ms per
+// step).  The code also takes BK = 64.
+constexpr int BK = 128;
+constexpr int STAGES = BK == 64 ? 6 : 3;
+constexpr int CHUNK_BYTES = HALF * 64 * 2;       // 128 rows x 64 k (K-major) or 64 k x 64 (MN-major), 16 KB
 constexpr int BOX_BYTES = 64 * 64 * 2;
-constexpr int A_BYTES = HALF * TC_BK * 2;        // 16 KB
-constexpr int B_BYTES = HALF * TC_BK * 2;        // 16 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 KB per CTA
+constexpr int A_BYTES = HALF * BK * 2;
+constexpr int B_BYTES = HALF * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 32 or 64 KB per CTA
 constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t TMEM_COLS = 512;              // two 128-lane x 256-column accumulators
 constexpr int BAR_BYTES = 256;
@@ -59,6 +65,31 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, int t) {
   tl.lt = t - p.starts[tl.g];
   gemm_tile_coord(p.mats[tl.g].g, tl.lt, PAIR_BM, PAIR_BN, tl.tm, tl.tn);
   return tl;
+}
+
+// One CTA's operand slab (128 rows or columns x BK k) of one stage.
+//   K-major, chunked map (box 64 k x 128 rows x 2 k chunks): one copy;
+//   K-major, 2-D map (box 64 x 128): one copy per 64-k chunk;
+//   MN-major, chunked map (box 64 x BK k rows x 2 chunks): one copy;
+//   MN-major, 2-D map (box 64 x 64): one copy per 64 x 64 block.
+__device__ __forceinline__ void load_slab(uint8_t* s, const CUtensorMap* map, uint32_t bar, int mn,
+                                          int chunked, int k0, int r0) {
+  if (!mn) {
+    if (chunked) {
+      tma_load_3d_pair(s, map, bar, 0, r0, k0 / 64);
+    } else {
+#pragma unroll
+      for (int c = 0; c < BK / 64; ++c) tma_load_2d_pair(s + c * CHUNK_BYTES, map, bar, k0 + 64 * c, r0);
+    }
+  } else if (chunked) {
+    tma_load_3d_pair(s, map, bar, 0, k0, r0 / 64);
+  } else {
+#pragma unroll
+    for (int c = 0; c < HALF / 64; ++c)
+#pragma unroll
+      for (int j = 0; j < BK / 64; ++j)
+        tma_load_2d_pair(s + c * (BK * 128) + j * BOX_BYTES, map, bar, r0 + 64 * c, k0 + 64 * j);
+  }
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __grid_constant__ TcParams p) {
@@ -131,7 +162,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
         const int a3 = mt.g.flags & GF_A_BOX3, b3 = mt.g.flags & GF_B_BOX3;
         const int m0 = tl.tm * PAIR_BM + (int)rank * HALF;
         const int n0 = tl.tn * PAIR_BN + (int)rank * HALF;
-        const int nkb = (mt.g.K + TC_BK - 1) / TC_BK;
+        const int nkb = (mt.g.K + BK - 1) / BK;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort, p.status, WAIT_LIMIT_NS)) {
@@ -146,25 +177,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           }
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-          const int k0 = kb * TC_BK;
-          // one copy per 128 x 64 slab where the map allows: K-major slabs
-          // take a 64 x 128 box, MN-major ones the chunked 3-D box; the
-          // copy engine's per-copy cost makes 8 KB boxes too slow to feed
-          // the tensor pipe
-          if (!a_mn)
-            tma_load_2d_pair(sa, &mt.ta, bar, k0, m0);
-          else if (a3)
-            tma_load_3d_pair(sa, &mt.ta, bar, 0, k0, m0 / 64);
-          else
-            for (int q = 0; q < HALF / 64; ++q)
-              tma_load_2d_pair(sa + q * BOX_BYTES, &mt.ta, bar, m0 + 64 * q, k0);
-          if (!b_mn)
-            tma_load_2d_pair(sb, &mt.tb, bar, k0, n0);
-          else if (b3)
-            tma_load_3d_pair(sb, &mt.tb, bar, 0, k0, n0 / 64);
-          else
-            for (int q = 0; q < HALF / 64; ++q)
-              tma_load_2d_pair(sb + q * BOX_BYTES, &mt.tb, bar, n0 + 64 * q, k0);
+          const int k0 = kb * BK;
+          // one copy per operand slab where the map allows (the copy
+          // engine's per-copy cost makes 8 KB boxes too slow to feed the
+          // tensor pipe).  Stage layout per operand: K-major [k chunk][128
+          // rows][64 k]; MN-major [64-wide chunk][BK k rows][64].
+          load_slab(sa, &mt.ta, bar, a_mn, a3, k0, m0);
+          load_slab(sb, &mt.tb, bar, b_mn, b3, k0, n0);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -195,7 +214,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * PAIR_BN);
         const uint32_t idesc = idesc_bf16(PAIR_BM, PAIR_BN, a_mn, b_mn);
-        const int nkb = (g.K + TC_BK - 1) / TC_BK;
+        const int nkb = (g.K + BK - 1) / BK;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort, p.status, WAIT_LIMIT_NS)) {
@@ -206,11 +225,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < TC_BK / 16; ++kk) {
-            const uint64_t ad = a_mn ? smem_desc(sa + kk * 2048, BOX_BYTES, 1024)
-                                     : smem_desc(sa + kk * 32, 16, 1024);
-            const uint64_t bd = b_mn ? smem_desc(sb + kk * 2048, BOX_BYTES, 1024)
-                                     : smem_desc(sb + kk * 32, 16, 1024);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // K-major: k chunk kk / 4, 32 bytes per k step inside it;
+            // MN-major: 16 k rows of 128 bytes per k step, chunks BK rows apart
+            const uint32_t koff = (uint32_t)((kk >> 2) * CHUNK_BYTES + (kk & 3) * 32);
+            const uint64_t ad = a_mn ? smem_desc(sa + kk * 2048, BK * 128, 1024)
+                                     : smem_desc(sa + koff, 16, 1024);
+            const uint64_t bd = b_mn ? smem_desc(sb + kk * 2048, BK * 128, 1024)
+                                     : smem_desc(sb + koff, 16, 1024);
             mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           mma_commit_pair(&empty[stage], PAIR_MASK);  // frees the stage in both CTAs
@@ -280,6 +302,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
 }  // namespace
 
 int tc_pair_smem_bytes() { return SMEM_BYTES; }
+int tc_pair_bk() { return BK; }
 
 cudaError_t launch_tc_pair(const TcParams& p, int pairs, cudaStream_t s) {
   if (p.total_tiles <= 0 || pairs <= 0) return cudaSuccess;
