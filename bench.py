@@ -216,6 +216,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="large_batch")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--debug-flags", type=lambda v: int(v, 0), default=0,
+                    help="library debug_flags (test hooks such as DM_DBG_NO_PDL; none skips work)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
     spec = workload_spec(args.workload)
@@ -269,7 +271,8 @@ def main():
     mats = [dm.dm_matrix(W[i], G[i], M[i], ER[i], EC[i]) for i in range(len(shapes))]
     hp = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"],
                                scale_mode=dm.DM_SCALE_MOONSHOT if spec["moonshot"]
-                               else dm.DM_SCALE_NONE, nesterov=spec.get("nesterov", 0))
+                               else dm.DM_SCALE_NONE, nesterov=spec.get("nesterov", 0),
+                               debug_flags=args.debug_flags)
     step_fn = dm.dm_dimuon_step if spec["cond"] else dm.dm_muon_step
     ws = torch.empty(dm.dm_workspace_size(mats, hp, int(spec["cond"])), dtype=torch.uint8,
                      device=dev)
@@ -317,7 +320,8 @@ def main():
     # schedule over a 1-step schedule, on the launch stream
     reps = max(2, min(args.steps, 5))
     hp1 = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"], ns_steps=1,
-                                scale_mode=hp.scale_mode, nesterov=hp.nesterov)
+                                scale_mode=hp.scale_mode, nesterov=hp.nesterov,
+                                debug_flags=args.debug_flags)
     g1 = capture(hp1)
     g1.replay()
     t5 = timed(graph, reps) / reps
