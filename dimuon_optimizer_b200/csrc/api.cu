@@ -148,8 +148,10 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
     L.mats.push_back(p);
   }
   // thin factors: one launch group per padded short side and path (staged
-  // path for r == pad, long side a multiple of 8, 16-byte aligned buffers and
-  // a supported storage combination; register path otherwise)
+  // path for r == pad, long side a multiple of 8 (any length for tall factors
+  // with r >= 8: each staged row is then whole 16-byte groups), 16-byte
+  // aligned buffers and a supported storage combination; register path
+  // otherwise)
   auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
   std::vector<std::pair<int, int>> pads;
   std::vector<std::vector<int>> members;
@@ -158,7 +160,8 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
     const int pad = thin_pad(p.m);
     const dm_matrix_t& um = mats[p.idx];
     int combo = thin_bulk_combo(um.grad_dtype, um.momentum_dtype, um.weight_dtype);
-    const bool ok = p.m == pad && pad >= 2 && pad != 3 && p.n % 8 == 0 && al16(um.grad) &&
+    const bool ok = p.m == pad && pad >= 2 && pad != 3 && (p.n % 8 == 0 || (p.tall && pad >= 8)) &&
+                    al16(um.grad) &&
                     al16(um.momentum) && al16(um.weight) && al16(um.update_out) &&
                     (!cond || (al16(um.row_energy) && al16(um.col_energy)));
     if (!ok || (hp->debug_flags & DM_DBG_THIN_REGS)) combo = -1;

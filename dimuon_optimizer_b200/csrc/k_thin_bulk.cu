@@ -1,7 +1,8 @@
 // Thin-factor streaming passes with shared-memory staging: the same
 // arithmetic as thin_gram / thin_apply in k_thin.cu (Gram route, see there),
 // for factors whose short side r equals the padded rank RP, whose long side
-// is a multiple of 8 and whose buffers are 16-byte aligned, in one of the
+// is a multiple of 8 (any length for tall factors with r >= 8, whose staged
+// rows are whole 16-byte groups) and whose buffers are 16-byte aligned, in one of the
 // storage combinations (G, M, W) = (bf16, fp32, bf16), (bf16, bf16, bf16),
 // (fp32, fp32, fp32).
 //
@@ -247,7 +248,20 @@ __device__ void produce(const ThinParams& p, uint8_t* stages, int stage_bytes, i
           uint32_t bytes = (uint32_t)(RP * w) * (uint32_t)sizeof(TM);
           if (KIND == 0 || p.nesterov) bytes += (uint32_t)(RP * w) * (uint32_t)sizeof(TG);
           if (KIND == 1) bytes += (uint32_t)(RP * w) * (uint32_t)sizeof(TW);
-          if (cur.on) bytes += (uint32_t)w * 4u;
+          if (cur.on) {
+            // energies: whole 16-byte groups by bulk copy, the last w % 4
+            // values (a ragged tall factor's end) by plain stores, made
+            // visible to the consumers by this arrive's release
+            const int wq = w & ~3;
+            bytes += (uint32_t)wq * 4u;
+            const float* ec = geometry(cur.mt, p.conditioned).e_c;
+            float* es = reinterpret_cast<float*>(stages + (size_t)stage * stage_bytes + offE);
+            if (wq < w) {
+              for (int i = wq; i < w; ++i) es[i] = ec[si.c0 + i];
+              // later bulk copies into this stage come after these writes
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+          }
           mbar_arrive_expect_tx(&full[stage], bytes);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (ph << stage);
@@ -290,8 +304,8 @@ __device__ void produce(const ThinParams& p, uint8_t* stages, int stage_bytes, i
           bulk_load(base + offW, reinterpret_cast<const TW*>(si.mt.W) + g0,
                     (uint32_t)(w * RP * sizeof(TW)), &full[stage]);
       }
-      if (si.on && lane == 1)
-        bulk_load(base + offE, qs.e_c + si.c0, (uint32_t)(w * 4), &full[stage]);
+      if (si.on && lane == 1 && (w & ~3) > 0)
+        bulk_load(base + offE, qs.e_c + si.c0, (uint32_t)((w & ~3) * 4), &full[stage]);
       if (++stage == NS) {
         stage = 0;
         ph ^= 1;
