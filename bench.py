@@ -163,16 +163,17 @@ class ClockSampler:
                 "samples": len(load)}
 
 
-def oracle_sample_time(spec):
+def oracle_sample_time(spec, ns_steps=5):
     """Times the fp64 CPU oracle on one matrix of the workload (the cheapest
-    representative: the first shape) and extrapolates by algorithmic flops."""
+    representative: the first shape) with `ns_steps` Newton-Schulz iterations
+    and extrapolates to the whole 5-iteration step by algorithmic flops."""
     import oracle as orc
     shp = spec["shapes"][0]
     rng = np.random.default_rng(spec["seed"])
     G = rng.standard_normal(shp)
     W = 0.02 * rng.standard_normal(shp)
     M = np.zeros(shp)
-    h = orc.HParams(lr=spec["lr"], weight_decay=spec["wd"],
+    h = orc.HParams(lr=spec["lr"], weight_decay=spec["wd"], ns_steps=ns_steps,
                     scale_mode=orc.SCALE_MOONSHOT if spec["moonshot"] else orc.SCALE_NONE)
     t0 = time.perf_counter()
     if spec["cond"]:
@@ -181,19 +182,23 @@ def oracle_sample_time(spec):
     else:
         orc.muon_step(W, G, M, h, momentum_dtype=spec["mdt"], weight_dtype="bf16")
     dt = time.perf_counter() - t0
-    scale = ns_flops(spec["shapes"]) / ns_flops([shp])
-    return dt, dt * scale, f"one {shp[0]}x{shp[1]} matrix of the workload per step, " \
-                           f"extrapolated to all {len(spec['shapes'])} by algorithmic flops"
+    scale = 5 * ns_flops(spec["shapes"]) / (ns_steps * ns_flops([shp]))
+    what = "" if ns_steps == 5 else f" with {ns_steps} of the 5 Newton-Schulz iterations"
+    return dt, dt * scale, f"one {shp[0]}x{shp[1]} matrix of the workload{what} per step, " \
+                           f"extrapolated to all {len(spec['shapes'])} matrices and 5 iterations " \
+                           f"by algorithmic flops"
 
 
 def run_reference(args, spec, rank):
     if rank != 0:
         return
     threads = os.cpu_count()
-    oracle_sample_time(spec)  # one untimed warm-up step
+    # each step a bounded sample (one matrix, one Newton-Schulz iteration), so
+    # that the default 50 steps end within a few minutes
+    oracle_sample_time(spec, ns_steps=1)  # one untimed warm-up step
     times = []
     for _ in range(args.steps):
-        _, full, sample = oracle_sample_time(spec)
+        _, full, sample = oracle_sample_time(spec, ns_steps=1)
         times.append(full)
     t = float(np.median(times))
     value = len(spec["shapes"]) / t
@@ -211,8 +216,8 @@ def run_reference(args, spec, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="large_batch")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -377,6 +377,44 @@ __global__ void __launch_bounds__(TT) thin_gram(const __grid_constant__ ThinPara
 // ===========================================================================
 // thin_iterate: one CTA per factor
 // ===========================================================================
+// Sums over one factor's nu slab partials, in slab order (the same additions
+// as a plain loop), with the loads of up to 8 slabs issued before their
+// additions so that their L2 latencies overlap instead of adding up.
+// sum_slabs: entries base[v * stride + src] and base[v * stride + off + src].
+__device__ __forceinline__ void sum_slabs(const double* base, size_t stride, int off, int nu, int src,
+                                          double& g1, double& g2) {
+  g1 = 0.0;
+  g2 = 0.0;
+  for (int v0 = 0; v0 < nu; v0 += 8) {
+    double a[8], b[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const bool in = v0 + k < nu;
+      const double* pp = base + (size_t)(v0 + k) * stride;
+      a[k] = in ? pp[src] : 0.0;
+      b[k] = in ? pp[off + src] : 0.0;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      g1 += a[k];
+      g2 += b[k];
+    }
+  }
+}
+
+// sum_slabs for the float entries base[v * stride].
+__device__ __forceinline__ float sum_slabs_f(const float* base, size_t stride, int nu) {
+  float e = 0.f;
+  for (int v0 = 0; v0 < nu; v0 += 8) {
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = v0 + k < nu ? base[(size_t)(v0 + k) * stride] : 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) e += a[k];
+  }
+  return e;
+}
+
 template <int RP>
 struct IterSmem {
   double G[RP][TCfg<RP>::SLD], H[RP][TCfg<RP>::SLD], P[RP][TCfg<RP>::SLD],
@@ -482,12 +520,8 @@ __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ 
     } else {
       src = idx;
     }
-    double g1 = 0.0, g2 = 0.0;
-    for (int v = 0; v < nu; ++v) {
-      const double* pp = p.part + (size_t)(u0 + v) * 2 * Cf::PART;
-      g1 += pp[src];
-      g2 += pp[Cf::PART + src];
-    }
+    double g1, g2;
+    sum_slabs(p.part + (size_t)u0 * 2 * Cf::PART, 2 * Cf::PART, Cf::PART, nu, src, g1, g2);
     s.G[i][j] = g1;
     s.H[i][j] = g2;
   }
@@ -500,9 +534,7 @@ __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ 
   }
   __syncwarp();
   if (q.cond && lane < r) {
-    float e = 0.f;
-    for (int v = 0; v < nu; ++v) e += p.rpart[(size_t)(u0 + v) * RP + lane];
-    q.e_r[lane] = e;
+    q.e_r[lane] = sum_slabs_f(p.rpart + (size_t)u0 * RP + lane, RP, nu);
   }
   double tr = 0.0;
   for (int idx = lane; idx < RP * RP; idx += 32) {
@@ -597,12 +629,8 @@ __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinP
     } else {
       src = idx;
     }
-    double g1 = 0.0, g2 = 0.0;
-    for (int v = 0; v < nu; ++v) {
-      const double* pp = p.part + (size_t)(u0 + v) * 2 * Cf::PART;
-      g1 += pp[src];
-      g2 += pp[Cf::PART + src];
-    }
+    double g1, g2;
+    sum_slabs(p.part + (size_t)u0 * 2 * Cf::PART, 2 * Cf::PART, Cf::PART, nu, src, g1, g2);
     s.G[i][j] = g1;
     s.H[i][j] = g2;
   }
@@ -616,9 +644,7 @@ __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinP
   }
   __syncthreads();
   if (q.cond && tid < r) {
-    float e = 0.f;
-    for (int v = 0; v < nu; ++v) e += p.rpart[(size_t)(u0 + v) * RP + tid];
-    q.e_r[tid] = e;
+    q.e_r[tid] = sum_slabs_f(p.rpart + (size_t)u0 * RP + tid, RP, nu);
   }
   // A_0 = R S_1 R, H = R S_2 R; ||X_0||^2 = tr A_0
   double tr = 0.0;

@@ -352,20 +352,16 @@ struct GramBulk {
   static constexpr int MINB = RP == 8 || RP == 16 ? 3 : RP == 32 ? 2 : 1;  // resident CTAs
   static constexpr int CH = RP <= 4 ? 1024 : RP == 8 ? 256 : RP == 16 ? 128 : 64;
   static constexpr int NS = 4;
-  // reduction at the end of a run of slabs: NSLOT > 0 = asynchronous (each
-  // warp drops its partial into one of NSLOT slots, the last warp to arrive
-  // sums); 0 = all consumer warps meet
-  static constexpr int NSLOT = 0;
-  static constexpr int NRED = NSLOT > 0 ? NSLOT : 1;
   static constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH);
   static constexpr int OFF_G = opnd_bytes<TM>(RP, CH);
   static constexpr int OFF_E = OFF_G + opnd_bytes<TG>(RP, CH);
   static constexpr int STAGE_BYTES = (OFF_E + CH * 4 + 127) / 128 * 128;
-  static constexpr int RED_BYTES = NRED * (CW * 2 * TCfg<RP>::PART * 8 + CW * RP * 4) + NRED * 16;
+  // per-warp Gram and energy partials for the reduction at a run's end
+  static constexpr int RED_BYTES = CW * 2 * TCfg<RP>::PART * 8 + CW * RP * 4;
   static constexpr int NCOL = TCfg<RP>::MMA ? CH / CW : 0;  // columns of one consumer warp per stage
   static constexpr int WS_BYTES = CW * 2 * NCOL * 8;
-  static constexpr int SMEM = NS * STAGE_BYTES + NS * (int)sizeof(StageInfo) +
-                              (2 * NS + 2 + NRED) * 8 + 16 + RED_BYTES + WS_BYTES + 128;
+  static constexpr int SMEM = NS * STAGE_BYTES + NS * (int)sizeof(StageInfo) + (2 * NS + 2) * 8 + 16 +
+                              RED_BYTES + WS_BYTES + 128;
 };
 
 // Accumulators of one consumer lane for one slab.
@@ -595,15 +591,12 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
   StageInfo* info = reinterpret_cast<StageInfo*>(smem + NS * L::STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(info + NS);
   uint64_t* empty = full + NS;
-  uint64_t* redf = empty + NS;  // synchronous reduction: consumer warps wrote their partials
-  uint64_t* redr = redf + 1;    // synchronous reduction: consumer warps read the partials
-  uint64_t* done = redr + 1;    // asynchronous reduction: slot summed (one per slot)
-  volatile int* abort = reinterpret_cast<volatile int*>(done + L::NRED);
-  int* cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(done + L::NRED) + 4);  // per slot
-  double* red_s = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(done + L::NRED) + 16 +
-                                            L::NRED * 16);
-  float* red_e = reinterpret_cast<float*>(red_s + L::NRED * CW * 2 * Cf::PART);
-  double* wsm = reinterpret_cast<double*>(red_e + L::NRED * CW * RP);  // CW * RP is even
+  uint64_t* redf = empty + NS;  // run-end reduction: consumer warps wrote their partials
+  uint64_t* redr = redf + 1;    // run-end reduction: consumer warps read the partials
+  volatile int* abort = reinterpret_cast<volatile int*>(redr + 1);
+  double* red_s = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(redr + 1) + 16);
+  float* red_e = reinterpret_cast<float*>(red_s + CW * 2 * Cf::PART);
+  double* wsm = reinterpret_cast<double*>(red_e + CW * RP);  // CW * RP is even
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -613,10 +606,6 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
     }
     mbar_init(redf, CW);
     mbar_init(redr, CW);
-    for (int s = 0; s < L::NRED; ++s) {
-      mbar_init(&done[s], 1);
-      cnt[s] = 0;
-    }
     *abort = 0;
     fence_mbar_init();
   }
@@ -706,18 +695,11 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
     }
 
     if (last) {
-      // slab-end reduction over the consumer warps
-      const int slot = L::NSLOT > 0 ? (int)(nred % L::NRED) : 0;
-      const uint32_t use = L::NSLOT > 0 ? nred / L::NRED : nred;  // this slot's use count
-      if constexpr (L::NSLOT > 0) {
-        // the slot's previous sum is done before it is overwritten
-        if (use > 0 && !wait_phase(&done[slot], (use - 1) & 1u, abort, p.status)) break;
-      } else {
-        if (!wait_phase(redr, (nred & 1u) ^ 1u, abort, p.status)) break;
-      }
-      double* rs = red_s + (size_t)slot * CW * 2 * Cf::PART;
-      float* re = red_e + slot * CW * RP;
-      double* mine = rs + warp * 2 * Cf::PART;
+      // run-end reduction over the consumer warps: each writes its partials,
+      // all meet on redf, the sums go to the run's last slab, all meet on
+      // redr before the partial buffers are written again
+      if (!wait_phase(redr, (nred & 1u) ^ 1u, abort, p.status)) break;
+      double* mine = red_s + warp * 2 * Cf::PART;
       if constexpr (Cf::MMA) {
         constexpr int NB = Cf::NB, NUB = Cf::NUB;
 #pragma unroll
@@ -732,7 +714,7 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
           float e = acc.er[blk];
           e += __shfl_xor_sync(0xffffffffu, e, 1);
           e += __shfl_xor_sync(0xffffffffu, e, 2);
-          if (t == 0) re[warp * RP + g + 8 * blk] = e;
+          if (t == 0) red_e[warp * RP + g + 8 * blk] = e;
         }
       } else {
 #pragma unroll
@@ -746,59 +728,28 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
             }
           }
           const float e = warp_sum(acc.er[i]);
-          if (lane == 0) re[warp * RP + i] = e;
+          if (lane == 0) red_e[warp * RP + i] = e;
         }
       }
       double* dst = p.part + (size_t)u * 2 * Cf::PART;
-      if constexpr (L::NSLOT > 0) {
-        __threadfence_block();
-        __syncwarp();
-        int arrived = 0;
-        if (lane == 0) arrived = atomicAdd(&cnt[slot], 1);
-        arrived = __shfl_sync(0xffffffffu, arrived, 0);
-        if (arrived == CW - 1) {
-          // the last warp of this slab sums the slot in warp order
-          __threadfence_block();
-          for (int i = lane; i < 2 * Cf::PART; i += 32) {
-            double s = 0.0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(redf);
+      if (!wait_phase(redf, nred & 1u, abort, p.status)) break;
+      for (int i = tid; i < 2 * Cf::PART; i += 32 * CW) {
+        double s = 0.0;
 #pragma unroll
-            for (int w = 0; w < CW; ++w) s += rs[w * 2 * Cf::PART + i];
-            dst[i] = s;
-          }
-          if (cond)
-            for (int i = lane; i < RP; i += 32) {
-              float s = 0.f;
-#pragma unroll
-              for (int w = 0; w < CW; ++w) s += re[w * RP + i];
-              p.rpart[(size_t)u * RP + i] = s;
-            }
-          __syncwarp();
-          if (lane == 0) {
-            cnt[slot] = 0;
-            __threadfence_block();
-            mbar_arrive(&done[slot]);
-          }
-        }
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(redf);
-        if (!wait_phase(redf, nred & 1u, abort, p.status)) break;
-        for (int i = tid; i < 2 * Cf::PART; i += 32 * CW) {
-          double s = 0.0;
-#pragma unroll
-          for (int w = 0; w < CW; ++w) s += rs[w * 2 * Cf::PART + i];
-          dst[i] = s;
-        }
-        if (cond)
-          for (int i = tid; i < RP; i += 32 * CW) {
-            float s = 0.f;
-#pragma unroll
-            for (int w = 0; w < CW; ++w) s += re[w * RP + i];
-            p.rpart[(size_t)u * RP + i] = s;
-          }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(redr);
+        for (int w = 0; w < CW; ++w) s += red_s[w * 2 * Cf::PART + i];
+        dst[i] = s;
       }
+      if (cond)
+        for (int i = tid; i < RP; i += 32 * CW) {
+          float s = 0.f;
+#pragma unroll
+          for (int w = 0; w < CW; ++w) s += red_e[w * RP + i];
+          p.rpart[(size_t)u * RP + i] = s;
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(redr);
       ++nred;
     }
   }
