@@ -139,28 +139,35 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        rows = []
-        for ln in out.strip().splitlines():
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 10:
-                continue
-            try:
-                rows.append(dict(sm=float(f[1]), smax=float(f[2]), util=float(f[4]),
-                                 hw=f[6], hwt=f[7], swt=f[8], pcap=f[9]))
-            except ValueError:
-                continue
-        load = [r for r in rows if r["util"] >= 50] or rows
-        if not load:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        reasons = set()
-        for r in load:
-            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                            ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[k].lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": float(np.median([r["sm"] for r in load])),
-                "sm_max_mhz": max(r["smax"] for r in load), "reasons": sorted(reasons),
-                "samples": len(load)}
+        return parse_clock_log(out)
+
+
+def parse_clock_log(text):
+    """Summary of nvidia-smi samples (the ClockSampler query, csv, no header,
+    no units): median SM clock and the throttle reasons seen while the GPU
+    was busy (utilisation >= 50 %; all samples if none was)."""
+    rows = []
+    for ln in text.strip().splitlines():
+        f = [x.strip() for x in ln.split(",")]
+        if len(f) < 10:
+            continue
+        try:
+            rows.append(dict(sm=float(f[1]), smax=float(f[2]), util=float(f[4]),
+                             hw=f[6], hwt=f[7], swt=f[8], pcap=f[9]))
+        except ValueError:
+            continue
+    load = [r for r in rows if r["util"] >= 50] or rows
+    if not load:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    reasons = set()
+    for r in load:
+        for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                        ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+            if r[k].lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": float(np.median([r["sm"] for r in load])),
+            "sm_max_mhz": max(r["smax"] for r in load), "reasons": sorted(reasons),
+            "samples": len(load)}
 
 
 def oracle_sample_time(spec, ns_steps=5):

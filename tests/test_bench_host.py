@@ -1,0 +1,100 @@
+"""Host logic of bench.py (no GPU): the algorithmic flop count against the
+figures the workload definitions quote, the workload table, the clock-log
+summary that accepts or rejects a timed run, and the reference arm's JSON
+line (the fp64 oracle timed on the host cores)."""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+bench = _bench()
+
+
+@pytest.mark.parametrize("name,total", [
+    # five-iteration algorithmic totals quoted for the workloads (3 m^2 n + m^3
+    # per matrix per iteration, symmetric products counted once)
+    ("square1024", 2.15e10),
+    ("gpt2_small", 1.14e12),
+    ("large_batch", 4.26e13),
+])
+def test_ns_flops_matches_quoted_totals(name, total):
+    shapes = bench.workload_spec(name)["shapes"]
+    assert 5 * bench.ns_flops(shapes) == pytest.approx(total, rel=5e-3)
+
+
+def test_ns_flops_uses_the_short_side():
+    assert bench.ns_flops([(4096, 14336)]) == bench.ns_flops([(14336, 4096)])
+    # a square matrix: 3 m^3 + m^3
+    assert bench.ns_flops([(64, 64)]) == 4 * 64 ** 3
+
+
+@pytest.mark.parametrize("name,count", [
+    ("large_batch", 16), ("large_batch_dimuon", 16), ("large_batch_quarter", 4),
+    ("gpt2_small", 72), ("square1024", 1), ("lora_r2", 448), ("lora_r8", 448),
+    ("lora_r32", 448), ("vec_w1", 64), ("vec_w32", 64), ("vec_w128", 64)])
+def test_workload_table(name, count):
+    spec = bench.workload_spec(name)
+    assert len(spec["shapes"]) == count
+    assert spec["desc"]
+    assert spec["mdt"] in ("bf16", "fp32")
+
+
+def test_unknown_workload_exits():
+    with pytest.raises(SystemExit):
+        bench.workload_spec("no_such_workload")
+
+
+def _row(sm, util, pcap="Not Active", hw="Not Active", hwt="Not Active", swt="Not Active"):
+    return f"2026/12/02 10:00:00.000, {sm}, 1965, 900.0, {util}, 0x0, {hw}, {hwt}, {swt}, {pcap}"
+
+
+def test_clock_log_busy_samples_only():
+    text = "\n".join([_row(1965, 0), _row(1300, 100, pcap="Active"), _row(1310, 99, pcap="Active"),
+                      _row(1290, 98), _row(1965, 3)])
+    out = bench.parse_clock_log(text)
+    assert out["samples"] == 3
+    assert out["sm_mhz"] == 1300.0
+    assert out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_log_reports_slowdowns():
+    text = "\n".join([_row(900, 100, hw="Active"), _row(950, 100, hwt="Active", swt="Active")])
+    out = bench.parse_clock_log(text)
+    assert out["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+
+
+def test_clock_log_without_samples():
+    assert bench.parse_clock_log("garbage\n\n")["reasons"] == ["no samples"]
+    # all idle: the summary falls back to every sample
+    assert bench.parse_clock_log(_row(1965, 0))["samples"] == 1
+
+
+def test_reference_arm_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--workload", "square1024"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    assert d["metric"] == bench.METRIC
+    assert d["unit"] == "matrices/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["value"] == d["cpu_baseline"]["value"] == d["e2e"]["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == bench.workload_spec("square1024")["desc"]
