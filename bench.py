@@ -201,12 +201,23 @@ def run_reference(args, spec, rank):
         return
     threads = os.cpu_count()
     # each step a bounded sample (one matrix, one Newton-Schulz iteration), so
-    # that the default 50 steps end within a few minutes
-    oracle_sample_time(spec, ns_steps=1)  # one untimed warm-up step
+    # that the default 50 steps end within a few minutes; it is scaled to the
+    # five-iteration step by the time ratio of the two on the same matrix,
+    # measured once beforehand (untimed), so the per-matrix work outside the
+    # iterations is not multiplied by the iteration count
+    t5, _, _ = oracle_sample_time(spec, ns_steps=5)
+    t1, _, _ = oracle_sample_time(spec, ns_steps=1)
+    ratio = t5 / t1
+    shp = spec["shapes"][0]
+    to_all = ns_flops(spec["shapes"]) / ns_flops([shp])
     times = []
     for _ in range(args.steps):
-        _, full, sample = oracle_sample_time(spec, ns_steps=1)
-        times.append(full)
+        dt, _, _ = oracle_sample_time(spec, ns_steps=1)
+        times.append(dt * ratio * to_all)
+    sample = (f"one {shp[0]}x{shp[1]} matrix of the workload with 1 of the 5 Newton-Schulz "
+              f"iterations per step, scaled by that matrix's measured 5- to 1-iteration time "
+              f"ratio ({ratio:.2f}, calibrated once, untimed) and extrapolated to all "
+              f"{len(spec['shapes'])} matrices by algorithmic flops")
     t = float(np.median(times))
     value = len(spec["shapes"]) / t
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "matrices/s",
