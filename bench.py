@@ -374,18 +374,43 @@ def main():
                               "algorithmic bytes of the whole step over the step time",
                     "peak_kind": f"{peak_kind} HBM copy"}
 
-    # end to end through the public API: pinned host gradients in, status out
+    # end to end through the public API: every step's gradients copied in from
+    # pinned host memory, its status word read back.  Two device gradient sets:
+    # step t + 1's host-to-device copy runs on its own stream while step t
+    # computes; a step waits for its copy, and a copy waits until the step that
+    # last read its buffer has finished.
     h2d = sum(g.numel() * g.element_size() for g in G_host)
+    G2 = [torch.empty_like(g) for g in G]
+    bufs = [G, G2]
+    mats_buf = [mats, [dm.dm_matrix(W[i], G2[i], M[i], ER[i], EC[i]) for i in range(len(shapes))]]
+    cstream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    consumed = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def h2d_copy(t):
+        b = t % 2
+        with torch.cuda.stream(cstream):
+            if t >= 2:
+                cstream.wait_event(consumed[b])
+            for gd, gh in zip(bufs[b], G_host):
+                gd.copy_(gh, non_blocking=True)
+            copied[b].record(cstream)
+
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(args.steps):
-            for gd, gh in zip(G, G_host):
-                gd.copy_(gh, non_blocking=True)
-            dm.check(step_fn(mats, hp, ws, stream=stream))
+        cstream.wait_event(e0)
+        h2d_copy(0)
+        for t in range(args.steps):
+            b = t % 2
+            stream.wait_event(copied[b])
+            dm.check(step_fn(mats_buf[b], hp, ws, stream=stream))
+            consumed[b].record(stream)
+            if t + 1 < args.steps:
+                h2d_copy(t + 1)
             st = dm.dm_read_device_status(ws, stream=stream)
             assert st == dm.DM_OK, dm.dm_status_string(st)
         e1.record(stream)
@@ -393,7 +418,9 @@ def main():
     barrier()
     t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     e2e = {"value": world * n_mat * args.steps / t_e2e, "unit": "matrices/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4,
+           "h2d_overlap": "step t+1's copy overlaps step t (two device gradient sets)"}
+    del G2, mats_buf
     del graph
     if world > 1:
         dist.destroy_process_group()
