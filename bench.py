@@ -279,18 +279,28 @@ def main():
     mdt = torch.float32 if spec["mdt"] == "fp32" else bf
     rng = np.random.default_rng(spec["seed"] + 17 * rank)
     torch.manual_seed(spec["seed"] + 1000 + rank)
-    G_host, G, W, M, ER, EC = [], [], [], [], [], []
+    # gradients: views into one flat buffer on each side (each matrix starts on
+    # a 128-byte boundary), so a step's host-to-device copy is a single copy
+    offs, tot = [], 0
     for (r, c) in shapes:
+        offs.append(tot)
+        tot += (r * c + 63) // 64 * 64
+    G_host_flat = torch.zeros(tot, dtype=bf).pin_memory()
+    G_flat = torch.empty(tot, dtype=bf, device=dev)
+    G_host, G, W, M, ER, EC = [], [], [], [], [], []
+    for (r, c), o in zip(shapes, offs):
         gn = rng.standard_normal((r, c), dtype=np.float32)
         if spec.get("vec_len"):  # 1-D parameter: zero gradient in the padding cells
             gn.reshape(-1)[spec["vec_len"]:] = 0.0
-        g = torch.from_numpy(gn).to(bf)
-        G_host.append(g.pin_memory())
-        G.append(g.to(dev))
+        gh = G_host_flat[o:o + r * c].view(r, c)
+        gh.copy_(torch.from_numpy(gn).to(bf))
+        G_host.append(gh)
+        G.append(G_flat[o:o + r * c].view(r, c))
         W.append((0.02 * torch.randn((r, c), device=dev, dtype=torch.float32)).to(bf))
         M.append(torch.zeros((r, c), device=dev, dtype=mdt))
         ER.append(torch.zeros(r, device=dev, dtype=torch.float32) if spec["cond"] else None)
         EC.append(torch.zeros(c, device=dev, dtype=torch.float32) if spec["cond"] else None)
+    G_flat.copy_(G_host_flat)
     mats = [dm.dm_matrix(W[i], G[i], M[i], ER[i], EC[i]) for i in range(len(shapes))]
     hp = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"],
                                scale_mode=dm.DM_SCALE_MOONSHOT if spec["moonshot"]
@@ -379,9 +389,10 @@ def main():
     # step t + 1's host-to-device copy runs on its own stream while step t
     # computes; a step waits for its copy, and a copy waits until the step that
     # last read its buffer has finished.
-    h2d = sum(g.numel() * g.element_size() for g in G_host)
-    G2 = [torch.empty_like(g) for g in G]
-    bufs = [G, G2]
+    h2d = G_host_flat.numel() * G_host_flat.element_size()
+    G2_flat = torch.empty_like(G_flat)
+    G2 = [G2_flat[o:o + r * c].view(r, c) for (r, c), o in zip(shapes, offs)]
+    bufs = [G_flat, G2_flat]
     mats_buf = [mats, [dm.dm_matrix(W[i], G2[i], M[i], ER[i], EC[i]) for i in range(len(shapes))]]
     cstream = torch.cuda.Stream(dev)
     copied = [torch.cuda.Event(), torch.cuda.Event()]
@@ -392,8 +403,7 @@ def main():
         with torch.cuda.stream(cstream):
             if t >= 2:
                 cstream.wait_event(consumed[b])
-            for gd, gh in zip(bufs[b], G_host):
-                gd.copy_(gh, non_blocking=True)
+            bufs[b].copy_(G_host_flat, non_blocking=True)
             copied[b].record(cstream)
 
     e0 = torch.cuda.Event(enable_timing=True)
@@ -420,7 +430,7 @@ def main():
     e2e = {"value": world * n_mat * args.steps / t_e2e, "unit": "matrices/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4,
            "h2d_overlap": "step t+1's copy overlaps step t (two device gradient sets)"}
-    del G2, mats_buf
+    del G2, G2_flat, mats_buf
     del graph
     if world > 1:
         dist.destroy_process_group()
