@@ -4,6 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload large_batch|large_batch_dimuon|large_batch_quarter|gpt2_small|square1024|
                                lora_r2|lora_r8|lora_r32|vec_w1|vec_w2|vec_w8|vec_w32|vec_w128]
+                    [--no-cpu-baseline] [--debug-flags BITS]
+
+Defaults: 50 timed steps after 10 warm-ups, the large batch, one GPU.
 
 One step = one optimizer step (momentum, normalisation, five Newton-Schulz
 iterations, scale, decay, apply) over every matrix of the workload.  The
@@ -287,14 +290,12 @@ def main():
         tot += (r * c + 63) // 64 * 64
     G_host_flat = torch.zeros(tot, dtype=bf).pin_memory()
     G_flat = torch.empty(tot, dtype=bf, device=dev)
-    G_host, G, W, M, ER, EC = [], [], [], [], [], []
+    G, W, M, ER, EC = [], [], [], [], []
     for (r, c), o in zip(shapes, offs):
         gn = rng.standard_normal((r, c), dtype=np.float32)
         if spec.get("vec_len"):  # 1-D parameter: zero gradient in the padding cells
             gn.reshape(-1)[spec["vec_len"]:] = 0.0
-        gh = G_host_flat[o:o + r * c].view(r, c)
-        gh.copy_(torch.from_numpy(gn).to(bf))
-        G_host.append(gh)
+        G_host_flat[o:o + r * c].view(r, c).copy_(torch.from_numpy(gn).to(bf))
         G.append(G_flat[o:o + r * c].view(r, c))
         W.append((0.02 * torch.randn((r, c), device=dev, dtype=torch.float32)).to(bf))
         M.append(torch.zeros((r, c), device=dev, dtype=mdt))
