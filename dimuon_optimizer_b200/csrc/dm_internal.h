@@ -186,8 +186,9 @@ struct K3Params {
 // side, thin_setup copies the factor descriptors into the workspace (up to
 // THIN_MAX per launch) and sums the previous energies; thin_gram,
 // thin_iterate and thin_apply then cover every factor of that padded side,
-// the streaming two in slabs of thin_slab(pad) long-side columns handed out
-// by a device counter.
+// the streaming two in slabs of thin_slab(pad) long-side columns (handed out
+// by a device counter in the register kernels, as contiguous per-CTA ranges
+// in the staged ones).
 struct ThinMat {           // 64 bytes
   const void* G;
   void* M;

@@ -6,19 +6,20 @@
 // storage combinations (G, M, W) = (bf16, fp32, bf16), (bf16, bf16, bf16),
 // (fp32, fp32, fp32).
 //
-// One producer warp per CTA takes slabs from the device counter and streams
-// each slab through a ring of shared-memory stages with 1-D bulk async copies
-// (cp.async.bulk, completion on an mbarrier): the copies of the next stages
-// are in flight while the consumer warps (8, or 4 for r = 32) work on the
-// current one, so the loads need neither registers nor per-lane address
-// arithmetic.  Full steps run branch-free code specialised on the layout
-// (wide / tall), on whether Dimuon conditioning is on and on whether
-// energies are written; partial steps at a factor's end take a predicated
-// version.  Consumers
-// write their results (M_t, W, O, energies) straight to global memory.  Every
-// wait is bounded; the slab-end reduction of the Gram partials synchronises
-// the consumer warps through mbarriers, so a timeout can never leave a warp
-// stuck at a hardware barrier.
+// Each CTA owns a contiguous range of slabs (balanced to within one slab).
+// Two producer warps stream it through a ring of shared-memory stages, taking
+// alternate stages, with 1-D bulk async copies (cp.async.bulk, completion on
+// an mbarrier): the copies of the next stages are in flight while the
+// consumer warps (8, or 4 for r = 32) work on the current one, so the loads
+// need neither registers nor per-lane address arithmetic.  Full steps run
+// branch-free code specialised on the layout (wide / tall), on whether Dimuon
+// conditioning is on and on whether energies are written; partial steps at a
+// factor's end take a predicated version.  Consumers write their results
+// (M_t, W, O, energies) straight to global memory.  The Gram accumulators
+// live across a run of consecutive slabs of one factor and are reduced once
+// per run.  Every wait is bounded; the run-end reduction synchronises the
+// consumer warps through mbarriers, so a timeout can never leave a warp stuck
+// at a hardware barrier.
 #include <algorithm>
 
 #include "dm_common.cuh"
