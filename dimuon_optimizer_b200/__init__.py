@@ -43,6 +43,7 @@ DM_DBG_TC_SINGLE = 0x2
 DM_DBG_TC_PAIR = 0x4
 DM_DBG_FORCE_TIMEOUT = 0x8
 DM_DBG_THIN_REGS = 0x10
+DM_DBG_THIN_STAGED = 0x20
 
 DM_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 

@@ -496,7 +496,17 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     tp.T = reinterpret_cast<double*>(ws + tl.off_T);
     tp.fsc = fsc;
     tp.counters = reinterpret_cast<int*>(ws + THIN_CTR_OFFSET) + 2 * gi;
-    if (tl.combo >= 0)
+    // r = 2 on the staged layout whose momentum (and Nesterov gradient) fits
+    // one CTA's shared memory: the single-pass kernel
+    int64_t max_n = 0;
+    for (int i : tl.idx) max_n = std::max<int64_t>(max_n, L.mats[i].n);
+    const size_t fused_smem = thin_fused_smem(tl.pad, max_n, hp->nesterov != 0);
+    const bool fused = tl.combo >= 0 && tl.pad == 2 &&
+                       fused_smem <= THIN_FUSED_MAX_SMEM &&
+                       !(hp->debug_flags & DM_DBG_THIN_STAGED);
+    if (fused)
+      DM_CUDA(launch_thin_fused(tp, fused_smem, s));
+    else if (tl.combo >= 0)
       DM_CUDA(launch_thin_bulk(tp, tl.combo, sm_count(dev), s));
     else
       DM_CUDA(launch_thin(tp, sm_count(dev), s));

@@ -236,6 +236,11 @@ struct ThinParams {
 static_assert(sizeof(ThinMat) == 64, "ThinMat packing");
 static_assert(sizeof(ThinSetupParams) <= 32764, "kernel parameter space");
 int thin_part_doubles(int pad);
+// Single-pass thin step (one CTA per factor, r = pad = 2, the factor's
+// momentum and, under Nesterov, gradient kept in shared memory).
+constexpr size_t THIN_FUSED_MAX_SMEM = 96 * 1024;
+size_t thin_fused_smem(int pad, int64_t n, bool nesterov);
+cudaError_t launch_thin_fused(const ThinParams& p, size_t smem, cudaStream_t s);
 int thin_slab(int pad);
 
 // ------------------------------ launches ----------------------------------

@@ -499,32 +499,17 @@ __device__ __forceinline__ void mm_warp(double (*C)[RP + 1], double (*A)[RP + 1]
   __syncwarp();
 }
 
+// The r x r iteration of factor f by one warp.  On entry s.G and s.H hold
+// S_1 and S_2; the previous short-side energies are read here for R (before
+// the caller replaces them).  On return s.R holds R, s.P holds P_5 and the
+// result is the update factor kappa / ||X_0|| (times ||X_5|| / ||R X_5 C||
+// when conditioning is on), 0 for a degenerate norm; *on_out tells whether
+// conditioning was on.
 template <int RP>
-__global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ ThinParams p) {
-  using Cf = TCfg<RP>;
-  __shared__ WarpIterSmem<RP> sm[TW];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int f = blockIdx.x * TW + warp;
-  if (f >= p.count) return;  // the whole warp leaves; no block-wide barrier follows
-  WarpIterSmem<RP>& s = sm[warp];
-  const ThinMat mt = p.mats[f];
-  const Geo q = geometry(mt, p.conditioned);
+__device__ double iterate_factor_warp(const ThinParams& p, int f, const ThinMat& mt, const Geo& q,
+                                      WarpIterSmem<RP>& s, bool* on_out) {
+  const int lane = threadIdx.x & 31;
   const int r = q.r;
-  const int u0 = p.starts[f], nu = p.starts[f + 1] - p.starts[f];
-
-  for (int idx = lane; idx < RP * RP; idx += 32) {
-    const int i = idx / RP, j = idx % RP;
-    int src;
-    if constexpr (Cf::MMA) {
-      src = (i & 7) * 8 + (j & 7);  // one 8x8 block
-    } else {
-      src = idx;
-    }
-    double g1, g2;
-    sum_slabs(p.part + (size_t)u0 * 2 * Cf::PART, 2 * Cf::PART, Cf::PART, nu, src, g1, g2);
-    s.G[i][j] = g1;
-    s.H[i][j] = g2;
-  }
   const double sc = p.fsc[4 * f], sr = p.fsc[4 * f + 1];
   const bool on = q.cond && sr > 0.0 && sc > 0.0;
   if (lane < RP) {
@@ -533,9 +518,6 @@ __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ 
     s.R[lane] = rv;
   }
   __syncwarp();
-  if (q.cond && lane < r) {
-    q.e_r[lane] = sum_slabs_f(p.rpart + (size_t)u0 * RP + lane, RP, nu);
-  }
   double tr = 0.0;
   for (int idx = lane; idx < RP * RP; idx += 32) {
     const int i = idx / RP, j = idx % RP;
@@ -585,6 +567,41 @@ __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ 
     if (on) factor = ny > 0.0 ? factor * sqrt(nx / ny) : 0.0;
   }
   if (!finite && lane == 0) raise_status(p.status, ST_NONFINITE);
+  *on_out = on;
+  return factor;
+}
+
+template <int RP>
+__global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ ThinParams p) {
+  using Cf = TCfg<RP>;
+  __shared__ WarpIterSmem<RP> sm[TW];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = blockIdx.x * TW + warp;
+  if (f >= p.count) return;  // the whole warp leaves; no block-wide barrier follows
+  WarpIterSmem<RP>& s = sm[warp];
+  const ThinMat mt = p.mats[f];
+  const Geo q = geometry(mt, p.conditioned);
+  const int r = q.r;
+  const int u0 = p.starts[f], nu = p.starts[f + 1] - p.starts[f];
+
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP, j = idx % RP;
+    int src;
+    if constexpr (Cf::MMA) {
+      src = (i & 7) * 8 + (j & 7);  // one 8x8 block
+    } else {
+      src = idx;
+    }
+    double g1, g2;
+    sum_slabs(p.part + (size_t)u0 * 2 * Cf::PART, 2 * Cf::PART, Cf::PART, nu, src, g1, g2);
+    s.G[i][j] = g1;
+    s.H[i][j] = g2;
+  }
+  __syncwarp();
+  bool on;
+  const double factor = iterate_factor_warp<RP>(p, f, mt, q, s, &on);
+  // new short-side energies (R has been taken from the previous ones)
+  if (q.cond && lane < r) q.e_r[lane] = sum_slabs_f(p.rpart + (size_t)u0 * RP + lane, RP, nu);
   double* T = p.T + (size_t)f * RP * RP;
   for (int idx = lane; idx < RP * RP; idx += 32) {
     int i, j;
@@ -1054,6 +1071,253 @@ __global__ void __launch_bounds__(TT) thin_apply(const __grid_constant__ ThinPar
   }
 }
 
+// ===========================================================================
+// thin_fused: the whole step of one factor in one CTA, for r = RP = 2 when
+// the factor's momentum (and, under Nesterov, its gradient) fits in shared
+// memory.  Pass 1 streams G and M_{t-1} once: M_t (stored, and kept in
+// shared memory), the Gram sums S_1, S_2 and the short-side energies; the
+// block-reduced sums go through the r x r iteration on one warp; pass 2
+// applies O = T (C^2 B) to the kept momentum and streams W once, writing the
+// new long-side energies.  Per element the arithmetic is that of thin_gram /
+// thin_apply (fp64 momentum with one rounding, fp64 Gram sums and products);
+// the HBM traffic is the algorithmic one (G 2, M 4 + 4, W 2 + 2 bytes per
+// element with fp32 momentum), without the two-pass path's second read of
+// M_t, and one launch replaces three.
+// ===========================================================================
+constexpr int FT = 128;  // threads of thin_fused (four CTAs per SM: 448 factors in one wave)
+constexpr int FW = FT / 32;
+
+// Four long-side columns c .. c + 3 of all RP rows, as v[row][column].
+template <int RP>
+__device__ __forceinline__ void load_cols(const void* base, int dt, const Geo& q, int64_t c,
+                                          float v[RP][4]) {
+  if (!q.tall) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i) ld4(base, (int64_t)i * q.n + c, dt, v[i]);
+  } else {
+    float t[4 * RP];
+#pragma unroll
+    for (int k = 0; k < RP; ++k) ld4(base, c * RP + 4 * k, dt, &t[4 * k]);
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[i][e] = t[e * RP + i];
+  }
+}
+
+template <int RP>
+__device__ __forceinline__ void store_cols(void* base, int dt, const Geo& q, int64_t c,
+                                           const float v[RP][4]) {
+  if (!q.tall) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i) st4(base, (int64_t)i * q.n + c, dt, v[i]);
+  } else {
+    float t[4 * RP];
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) t[e * RP + i] = v[i][e];
+#pragma unroll
+    for (int k = 0; k < RP; ++k) st4(base, c * RP + 4 * k, dt, &t[4 * k]);
+  }
+}
+
+template <int RP>
+__global__ void __launch_bounds__(FT, 4) thin_fused(const __grid_constant__ ThinParams p) {
+  extern __shared__ __align__(16) uint8_t fused_raw[];
+  __shared__ WarpIterSmem<RP> it;
+  __shared__ double red[FW][2][RP][RP];
+  __shared__ float rede[FW][RP];
+  __shared__ double Tsm[RP][RP];
+  __shared__ int zsh;
+  const int f = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const ThinMat mt = p.mats[f];
+  const Geo q = geometry(mt, p.conditioned);
+  const int64_t n = q.n;
+  const bool nest = p.nesterov != 0;
+  float* Ms = reinterpret_cast<float*>(fused_raw);  // M_t, [n][RP]
+  float* Gs = Ms + (size_t)n * RP;                  // G under Nesterov, [n][RP]
+  const double sc = p.fsc[4 * f], sr = p.fsc[4 * f + 1];
+  const bool on = q.cond && sc > 0.0 && sr > 0.0;
+  const float inv_mc = on ? (float)((double)n / sc) : 0.f;
+  const float mu = p.mu, eps = p.eps;
+
+  // ---- pass 1: momentum, Gram sums, short-side energies -------------------
+  double s1[RP][RP], s2[RP][RP];
+  float er[RP];
+#pragma unroll
+  for (int i = 0; i < RP; ++i) {
+    er[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < RP; ++k) s1[i][k] = s2[i][k] = 0.0;
+  }
+  // each thread's next group of four columns is loaded before the current
+  // one is processed (two groups of loads in flight per thread)
+  float mv[RP][4], gv[RP][4];
+  if (4 * (int64_t)tid < n) {
+    load_cols<RP>(mt.M, mt.mdt, q, 4 * (int64_t)tid, mv);
+    load_cols<RP>(mt.G, mt.gdt, q, 4 * (int64_t)tid, gv);
+  }
+  for (int64_t c = 4 * (int64_t)tid; c < n; c += 4 * FT) {
+    float mn[RP][4], gn[RP][4];
+    const bool more = c + 4 * FT < n;
+    if (more) {
+      load_cols<RP>(mt.M, mt.mdt, q, c + 4 * FT, mn);
+      load_cols<RP>(mt.G, mt.gdt, q, c + 4 * FT, gn);
+    }
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float m = momentum_value(mu, mv[i][e], gv[i][e], mt.mdt);
+        mv[i][e] = m;
+        er[i] = fmaf(m, m, er[i]);
+      }
+    store_cols<RP>(mt.M, mt.mdt, q, c, mv);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+      for (int i = 0; i < RP; ++i) {
+        Ms[(c + e) * RP + i] = mv[i][e];
+        if (nest) Gs[(c + e) * RP + i] = gv[i][e];
+      }
+    double wd[4] = {1.0, 1.0, 1.0, 1.0};
+    if (on) {
+      const float4 e4 = *reinterpret_cast<const float4*>(q.e_c + c);
+      wd[0] = (double)col_weight(e4.x, inv_mc, eps);
+      wd[1] = (double)col_weight(e4.y, inv_mc, eps);
+      wd[2] = (double)col_weight(e4.z, inv_mc, eps);
+      wd[3] = (double)col_weight(e4.w, inv_mc, eps);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      double bx[RP];
+#pragma unroll
+      for (int k = 0; k < RP; ++k)
+        bx[k] = nest ? fma((double)mu, (double)mv[k][e], (double)gv[k][e]) : (double)mv[k][e];
+#pragma unroll
+      for (int i = 0; i < RP; ++i)
+#pragma unroll
+        for (int k = i; k < RP; ++k) {
+          const double xk = on ? wd[e] * bx[k] : bx[k];
+          s1[i][k] = fma(bx[i], xk, s1[i][k]);
+          if (on) s2[i][k] = fma(bx[i], wd[e] * xk, s2[i][k]);
+        }
+    }
+    if (more) {
+#pragma unroll
+      for (int i = 0; i < RP; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          mv[i][e] = mn[i][e];
+          gv[i][e] = gn[i][e];
+        }
+    }
+  }
+
+  // ---- block reduction (warps in order), then the r x r iteration ----------
+#pragma unroll
+  for (int i = 0; i < RP; ++i) {
+#pragma unroll
+    for (int k = i; k < RP; ++k) {
+      const double a = warp_sum_d(s1[i][k]), b = warp_sum_d(s2[i][k]);
+      if (lane == 0) {
+        red[warp][0][i][k] = a;
+        red[warp][1][i][k] = b;
+      }
+    }
+    const float e = warp_sum(er[i]);
+    if (lane == 0) rede[warp][i] = e;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    for (int idx = lane; idx < RP * RP; idx += 32) {
+      const int i = idx / RP, j = idx % RP;
+      const int lo = i <= j ? i : j, hi = i <= j ? j : i;
+      double g1 = 0.0, g2 = 0.0;
+#pragma unroll
+      for (int w = 0; w < FW; ++w) {
+        g1 += red[w][0][lo][hi];
+        g2 += red[w][1][lo][hi];
+      }
+      it.G[i][j] = g1;
+      it.H[i][j] = g2;
+    }
+    __syncwarp();
+    bool on_it;
+    const double factor = iterate_factor_warp<RP>(p, f, mt, q, it, &on_it);
+    // new short-side energies (R has been taken from the previous ones)
+    if (q.cond && lane < q.r) {
+      float e = 0.f;
+#pragma unroll
+      for (int w = 0; w < FW; ++w) e += rede[w][lane];
+      q.e_r[lane] = e;
+    }
+    for (int idx = lane; idx < RP * RP; idx += 32) {
+      const int i = idx / RP, j = idx % RP;
+      Tsm[i][j] = factor * it.R[i] * it.P[i][j] * it.R[j];
+    }
+    if (lane == 0) zsh = factor == 0.0 ? 1 : 0;
+  }
+  __syncthreads();
+
+  // ---- pass 2: O = T (C^2 B), W update, long-side energies -----------------
+  double tm[RP][RP];
+#pragma unroll
+  for (int i = 0; i < RP; ++i)
+#pragma unroll
+    for (int k = 0; k < RP; ++k) tm[i][k] = Tsm[i][k];
+  const bool zero = zsh != 0;
+  const float lr = p.lr, decay = p.decay;
+  float wv[RP][4];
+  if (4 * (int64_t)tid < n) load_cols<RP>(mt.W, mt.wdt, q, 4 * (int64_t)tid, wv);
+  for (int64_t c = 4 * (int64_t)tid; c < n; c += 4 * FT) {
+    float wn[RP][4], ov[RP][4];
+    const bool more = c + 4 * FT < n;
+    if (more) load_cols<RP>(mt.W, mt.wdt, q, c + 4 * FT, wn);
+    double wd[4] = {1.0, 1.0, 1.0, 1.0};
+    if (on) {
+      const float4 e4 = *reinterpret_cast<const float4*>(q.e_c + c);
+      wd[0] = (double)col_weight(e4.x, inv_mc, eps);
+      wd[1] = (double)col_weight(e4.y, inv_mc, eps);
+      wd[2] = (double)col_weight(e4.z, inv_mc, eps);
+      wd[3] = (double)col_weight(e4.w, inv_mc, eps);
+    }
+    float ce[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      double x[RP];
+      float sq = 0.f;
+#pragma unroll
+      for (int k = 0; k < RP; ++k) {
+        const float m = Ms[(c + e) * RP + k];
+        const double bv = nest ? fma((double)mu, (double)m, (double)Gs[(c + e) * RP + k]) : (double)m;
+        x[k] = on ? wd[e] * bv : bv;
+        sq = fmaf(m, m, sq);
+      }
+      ce[e] = sq;
+#pragma unroll
+      for (int i = 0; i < RP; ++i) {
+        double y = 0.0;
+#pragma unroll
+        for (int k = 0; k < RP; ++k) y = fma(tm[i][k], x[k], y);
+        ov[i][e] = zero ? 0.f : (float)y;
+        wv[i][e] = decay * wv[i][e] - lr * ov[i][e];
+      }
+    }
+    store_cols<RP>(mt.W, mt.wdt, q, c, wv);
+    if (mt.upd) store_cols<RP>(mt.upd, DT_FP32, q, c, ov);
+    if (q.cond) *reinterpret_cast<float4*>(q.e_c + c) = make_float4(ce[0], ce[1], ce[2], ce[3]);
+    if (more) {
+#pragma unroll
+      for (int i = 0; i < RP; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wv[i][e] = wn[i][e];
+    }
+  }
+}
+
 template <typename K>
 int resident_ctas(K kernel, int smem) {
   int occ = 0;
@@ -1140,6 +1404,34 @@ cudaError_t launch_thin_iterate(const ThinParams& p, cudaStream_t s) {
     case 16: return launch_iter_rp<16>(p, s);
     default: return launch_iter_rp<32>(p, s);
   }
+}
+
+namespace {
+template <int RP>
+cudaError_t launch_fused_rp(const ThinParams& p, size_t smem, cudaStream_t st) {
+  static int configured = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured != dev) {
+    cudaError_t e = cudaFuncSetAttribute(thin_fused<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)THIN_FUSED_MAX_SMEM);
+    if (e != cudaSuccess) return e;
+    configured = dev;
+  }
+  thin_fused<RP><<<p.count, FT, smem, st>>>(p);
+  return cudaGetLastError();
+}
+}  // namespace
+
+size_t thin_fused_smem(int pad, int64_t n, bool nesterov) {
+  return (size_t)n * (size_t)pad * sizeof(float) * (nesterov ? 2 : 1);
+}
+
+cudaError_t launch_thin_fused(const ThinParams& p, size_t smem, cudaStream_t s) {
+  if (p.count <= 0) return cudaSuccess;
+  if (smem > THIN_FUSED_MAX_SMEM) return cudaErrorInvalidValue;
+  if (p.pad != 2) return cudaErrorInvalidValue;
+  return launch_fused_rp<2>(p, smem, s);
 }
 
 cudaError_t launch_thin_setup(const ThinSetupParams& p, cudaStream_t s) {

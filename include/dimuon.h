@@ -135,6 +135,9 @@ typedef struct {
                                      (256 x 256 tiles) only                */
 #define DM_DBG_THIN_REGS 0x10u    /* thin factors always take the register
                                      path (no shared-memory staging)       */
+#define DM_DBG_THIN_STAGED 0x20u  /* thin factors of r = 2 take the
+                                     two-pass staged kernels instead of the
+                                     single-pass one (one CTA per factor)  */
 #define DM_DBG_FORCE_TIMEOUT 0x8u /* failure-detection hook: each
                                      tensor-core product launch makes one
                                      bounded wait run out (20 ms, on a

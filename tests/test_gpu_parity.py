@@ -103,16 +103,18 @@ def test_ns_step_counts(ns_steps):
 # --------------------------------------------------------------------------
 # thin factors (Gram route).  Shapes with r in {2, 4, 8, 16, 32} and a long
 # side divisible by 8 (any long side for tall factors with r >= 8) take the
-# shared-memory staged kernels, the rest (and everything under
-# DM_DBG_THIN_REGS) the register kernels.  The ragged tall ones end their
-# last stage on a partial group of four energies.
+# shared-memory staged kernels (r = 2: the single-pass kernel unless
+# DM_DBG_THIN_STAGED), the rest (and everything under DM_DBG_THIN_REGS) the
+# register kernels.  The ragged tall ones end their last stage on a partial
+# group of four energies.
 # --------------------------------------------------------------------------
 THIN_SHAPES = [(4, 16), (2, 100), (8, 4096), (4096, 8), (17, 333), (32, 4096), (4096, 32),
                (1, 50), (50, 1), (31, 31), (16, 1000), (2, 2056), (3000, 4), (8, 24),
                (1001, 8), (4099, 16), (777, 32), (13, 8)]
 
 
-@pytest.mark.parametrize("path", [0, dm.DM_DBG_THIN_REGS], ids=["staged", "regs"])
+@pytest.mark.parametrize("path", [0, dm.DM_DBG_THIN_STAGED, dm.DM_DBG_THIN_REGS],
+                         ids=["default", "staged", "regs"])
 @pytest.mark.parametrize("cond", [False, True])
 @pytest.mark.parametrize("mdt", [F32, BF])
 def test_thin_path(cond, mdt, path):
