@@ -381,8 +381,9 @@ def main():
         peak = peaks.get("hbm_gbs", 6650.0)
         roofline = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                     "frac": gbs / peak, "traffic": None,
-                    "kernel": "thin path (thin_setup + thin_gram + thin_iterate + thin_apply), "
-                              "algorithmic bytes of the whole step over the step time",
+                    "kernel": "thin path (thin_setup, then thin_gram + thin_iterate + thin_apply, "
+                              "or thin_fused for r = 2), algorithmic bytes of the whole step over "
+                              "the step time",
                     "peak_kind": f"{peak_kind} HBM copy"}
 
     # end to end through the public API: every step's gradients copied in from
@@ -443,14 +444,21 @@ def main():
     launches = 0
     if thin:
         # per padded short side: thin_setup (448 factors per launch), then the
-        # Gram, r x r iteration and apply launches
+        # Gram, r x r iteration and apply launches, or for r = 2 on the staged
+        # layout with the momentum fitting 96 KB of shared memory the one
+        # single-pass launch
         pads = {}
         for s in shapes:
             r = min(s)
             if r <= dm.DM_THIN_MAX:
                 pad = r if r <= 4 else 8 if r <= 8 else 16 if r <= 16 else 32
-                pads[pad] = pads.get(pad, 0) + 1
-        launches += sum(math.ceil(cnt / 448) + 3 for cnt in pads.values())
+                pads.setdefault(pad, []).append(s)
+        nest = 2 if hp.nesterov else 1
+        for pad, group in pads.items():
+            fused = (pad == 2 and not (args.debug_flags & dm.DM_DBG_THIN_STAGED) and
+                     all(min(s) == 2 and max(s) % 8 == 0 and max(s) * 2 * 4 * nest <= 96 * 1024
+                         for s in group))
+            launches += math.ceil(len(group) / 448) + (1 if fused else 3)
     if big:
         launches += 2 + 3 * hp.ns_steps + (3 if spec["cond"] else 0)
     cpu = None
