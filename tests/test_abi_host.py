@@ -109,3 +109,21 @@ def test_muon_ignores_missing_energies():
     assert dm.dm_workspace_size([m], hp, 0) > 0
     with pytest.raises(dm.DimuonError):
         dm.dm_workspace_size([m], hp, 1)
+
+
+def test_header_constants_match_binding():
+    """Every integer #define and enumerator of the header has the same value in
+    the binding (a flag added on one side only would silently do nothing)."""
+    text = open(HEADER).read()
+    consts = {}
+    for name, val in re.findall(r"^#define (DM_\w+) (0x[0-9a-fA-F]+|\d+)u?\b", text, flags=re.M):
+        consts[name] = int(val, 0)
+    for name, val in re.findall(r"\b(DM_[A-Z0-9_]+) = (\d+)", text):
+        consts[name] = int(val)
+    assert "DM_DBG_THIN_STAGED" in consts and "DM_ERR_NONFINITE" in consts
+    for name, val in consts.items():
+        assert hasattr(dm, name), f"binding lacks {name}"
+        assert getattr(dm, name) == val, (name, getattr(dm, name), val)
+    # debug flags are distinct bits
+    bits = [v for k, v in consts.items() if k.startswith("DM_DBG_")]
+    assert all(b & (b - 1) == 0 for b in bits) and len(set(bits)) == len(bits)
