@@ -37,6 +37,8 @@ DM_PREC_FP32 = 0
 DM_PREC_BF16_TC = 1
 DM_SCALE_NONE = 0
 DM_SCALE_MOONSHOT = 1
+DM_SCALE_JORDAN = 2
+DM_SCALE_BERNSTEIN = 3
 DM_THIN_MAX = 32
 DM_DBG_NO_THIN = 0x1
 DM_DBG_TC_SINGLE = 0x2

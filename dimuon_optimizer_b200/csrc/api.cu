@@ -77,7 +77,9 @@ dm_status_t validate(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int
   if (n < 0 || (n > 0 && !mats) || !hp) return DM_ERR_INVALID_ARG;
   if (hp->ns_steps < 1 || hp->ns_steps > 64) return DM_ERR_INVALID_ARG;
   if (hp->precision != DM_PREC_FP32 && hp->precision != DM_PREC_BF16_TC) return DM_ERR_INVALID_ARG;
-  if (hp->scale_mode != DM_SCALE_NONE && hp->scale_mode != DM_SCALE_MOONSHOT) return DM_ERR_INVALID_ARG;
+  if (hp->scale_mode != DM_SCALE_NONE && hp->scale_mode != DM_SCALE_MOONSHOT &&
+      hp->scale_mode != DM_SCALE_JORDAN && hp->scale_mode != DM_SCALE_BERNSTEIN)
+    return DM_ERR_INVALID_ARG;
   const float scalars[] = {hp->mu, hp->lr, hp->weight_decay, hp->a, hp->b, hp->c, hp->cond_eps,
                            hp->scale_coef};
   for (float v : scalars)
@@ -405,10 +407,18 @@ OperandSrc fill_gemm(GemmMat& g, const MatPlan& p, const dm_matrix_t& um, const 
   return src;
 }
 
+// Per-matrix update scale (dm_scale_t), rows x cols in the caller's orientation.
 float kappa_of(const dm_hparams_t* hp, int64_t rows, int64_t cols) {
-  if (hp->scale_mode == DM_SCALE_MOONSHOT)
-    return (float)((double)hp->scale_coef * std::sqrt((double)std::max(rows, cols)));
-  return 1.f;
+  switch (hp->scale_mode) {
+    case DM_SCALE_MOONSHOT:
+      return (float)((double)hp->scale_coef * std::sqrt((double)std::max(rows, cols)));
+    case DM_SCALE_JORDAN:
+      return (float)std::sqrt(std::max(1.0, (double)rows / (double)cols));
+    case DM_SCALE_BERNSTEIN:
+      return (float)std::sqrt((double)rows / (double)cols);
+    default:
+      return 1.f;
+  }
 }
 
 #define DM_CUDA(x)                          \

@@ -23,7 +23,8 @@
  *      afterwards", Dimuon page, Problem 4 (c)).  Muon: Y = X.
  *   5. O = kappa Y, kappa = 1 (DM_SCALE_NONE) or
  *      scale_coef * sqrt(max(rows, cols)) (DM_SCALE_MOONSHOT, RMS matched to
- *      AdamW: sitech.ge, "From speedrun to real training").
+ *      AdamW: sitech.ge, "From speedrun to real training"), or one of the
+ *      two other rules that section names without formulas (dm_scale_t).
  *   6. W_t = (1 - lr * weight_decay) W_{t-1} - lr O   (decoupled decay:
  *      "Muon Optimizer 정리", "Scaling up"; eq. (3)).
  *
@@ -81,7 +82,19 @@ typedef enum {
                            accumulation in tensor memory                      */
 } dm_precision_t;
 
-typedef enum { DM_SCALE_NONE = 0, DM_SCALE_MOONSHOT = 1 } dm_scale_t;
+/* Per-matrix update scale kappa; rows x cols is the matrix as the caller
+ * stores it (rows = output features of an (out, in) weight).  The sitech.ge
+ * post ("From speedrun to real training") names Jordan's, Moonshot's and
+ * Bernstein's rules as different without printing the first and the last;
+ * DM_SCALE_JORDAN and DM_SCALE_BERNSTEIN follow those authors' published
+ * rules (Jordan's Muon: sqrt(max(1, out / in)); Bernstein's spectral
+ * scaling: sqrt(out / in)).  scale_coef is used by DM_SCALE_MOONSHOT only. */
+typedef enum {
+  DM_SCALE_NONE = 0,      /* kappa = 1                                   */
+  DM_SCALE_MOONSHOT = 1,  /* kappa = scale_coef * sqrt(max(rows, cols))  */
+  DM_SCALE_JORDAN = 2,    /* kappa = sqrt(max(1, rows / cols))           */
+  DM_SCALE_BERNSTEIN = 3  /* kappa = sqrt(rows / cols)                   */
+} dm_scale_t;
 
 #define DM_THIN_MAX 32
 

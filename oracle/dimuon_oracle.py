@@ -76,6 +76,8 @@ NORM_FLOOR = 1e-15      # ||X_0||_F below this: zero update (see module docstrin
 
 SCALE_NONE = 0
 SCALE_MOONSHOT = 1
+SCALE_JORDAN = 2
+SCALE_BERNSTEIN = 3
 
 
 def f32(x: float) -> float:
@@ -197,12 +199,21 @@ def newton_schulz(X, steps: int = NS_STEPS, a: float = NS_A, b: float = NS_B,
 
 
 def scale_factor(mode: int, coef: float, rows: int, cols: int) -> float:
-    """Per-matrix update scale kappa ([Sitech], "From speedrun to real
-    training": RMS matched to AdamW)."""
+    """Per-matrix update scale kappa, rows x cols as the caller stores the
+    matrix (rows = output features).  MOONSHOT: RMS matched to AdamW
+    ([Sitech], "From speedrun to real training").  That section names
+    Jordan's and Bernstein's rules as different ones without formulas; they
+    are read as those authors' published rules: Jordan's Muon scales by
+    sqrt(max(1, rows / cols)), Bernstein's spectral scaling by
+    sqrt(rows / cols).  Parity of these two is unpinned to the pages."""
     if mode == SCALE_NONE:
         return 1.0
     if mode == SCALE_MOONSHOT:
         return coef * math.sqrt(max(rows, cols))
+    if mode == SCALE_JORDAN:
+        return math.sqrt(max(1.0, rows / cols))
+    if mode == SCALE_BERNSTEIN:
+        return math.sqrt(rows / cols)
     raise ValueError(f"unknown scale mode {mode}")
 
 

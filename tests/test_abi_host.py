@@ -83,6 +83,7 @@ def test_workspace_size_host_only():
     (lambda m, h: setattr(h, "ns_steps", 0), dm.DM_ERR_INVALID_ARG),
     (lambda m, h: setattr(h, "precision", 5), dm.DM_ERR_INVALID_ARG),
     (lambda m, h: setattr(h, "scale_mode", 9), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(h, "scale_mode", 4), dm.DM_ERR_INVALID_ARG),
     (lambda m, h: setattr(h, "lr", float("nan")), dm.DM_ERR_INVALID_ARG),
     (lambda m, h: setattr(m, "row_energy", None), dm.DM_ERR_INVALID_ARG),
 ])
@@ -92,6 +93,17 @@ def test_argument_errors_are_synchronous(mutate, code):
     mutate(m, hp)
     # validated before any device call: these return without touching a GPU
     assert dm.dm_dimuon_step([m], hp, (0x100000, 1 << 30), stream=0) == code
+
+
+@pytest.mark.parametrize("mode", [dm.DM_SCALE_NONE, dm.DM_SCALE_MOONSHOT, dm.DM_SCALE_JORDAN,
+                                  dm.DM_SCALE_BERNSTEIN])
+def test_every_scale_mode_is_accepted(mode):
+    """Argument validation passes (the call then stops at the missing
+    workspace, before any device work)."""
+    m = fake_matrix(64, 96)
+    hp = dm.dm_default_hparams(scale_mode=mode)
+    assert dm.dm_muon_step([m], hp, (0, 0), stream=0) == dm.DM_ERR_WORKSPACE
+    assert dm.dm_workspace_size([m], hp, 0) > 0
 
 
 def test_workspace_errors():

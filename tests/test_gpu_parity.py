@@ -165,6 +165,19 @@ def test_nesterov(prec, tol, cond):
                                  max(thin_tol), ws=ws)
 
 
+@pytest.mark.parametrize("prec,tol", [(dm.DM_PREC_FP32, TOL_FP32), (dm.DM_PREC_BF16_TC, TOL_BF16)])
+@pytest.mark.parametrize("mode", [dm.DM_SCALE_JORDAN, dm.DM_SCALE_BERNSTEIN])
+def test_scale_rules(mode, prec, tol):
+    """Jordan's and Bernstein's per-matrix scale on every path (Newton-Schulz
+    wide and tall, thin wide and tall)."""
+    shapes = [(200, 330), (330, 200), (8, 600), (600, 16)]
+    grp = Group(shapes, BF, BF, F32, cond=False, seed=23)
+    hp = hparams(prec, scale_mode=mode, weight_decay=0.02)
+    ws = None
+    for t in range(2):
+        _, ws = step_and_compare(grp, gaussian(shapes, 950 + t, scale_cols=True), hp, tol, ws=ws)
+
+
 # --------------------------------------------------------------------------
 # invariants and edge cases
 # --------------------------------------------------------------------------

@@ -526,3 +526,34 @@ def test_vector_width_one_closed_form(width, golden):
     k = quintic_scalar(1.0, h.a, h.b, h.c, g5["iterations"])
     np.testing.assert_array_equal(got.M, Mt)
     np.testing.assert_allclose(got.O, k * B / np.linalg.norm(B), rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Jordan / Bernstein scale rules (named, not printed, by [Sitech] "From
+# speedrun to real training"; read as those authors' published rules).
+# Parity of the two formulas is unpinned to the pages; what is pinned is how
+# the scale enters the step: O is exactly kappa times the unscaled update,
+# and the orientation (rows = output features) decides which side counts.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(96, 40), (40, 96), (64, 64)])
+def test_scale_rules_closed_forms(shape):
+    r, c = shape
+    assert orc.scale_factor(orc.SCALE_JORDAN, 0.2, r, c) == pytest.approx(max(1.0, r / c) ** 0.5)
+    assert orc.scale_factor(orc.SCALE_BERNSTEIN, 0.2, r, c) == pytest.approx((r / c) ** 0.5)
+    # Jordan's rule never shrinks the update; Bernstein's shrinks it for wide matrices
+    assert orc.scale_factor(orc.SCALE_JORDAN, 0.2, r, c) >= 1.0
+    assert (orc.scale_factor(orc.SCALE_BERNSTEIN, 0.2, r, c) < 1.0) == (r < c)
+
+
+@pytest.mark.parametrize("mode", [orc.SCALE_JORDAN, orc.SCALE_BERNSTEIN])
+@pytest.mark.parametrize("shape", [(48, 20), (20, 48)])
+def test_scale_rules_scale_the_update_only(mode, shape):
+    rng = np.random.default_rng(77)
+    W = 0.02 * rng.standard_normal(shape)
+    G = rng.standard_normal(shape)
+    M = rng.standard_normal(shape)
+    base = orc.muon_step(W, G, M, orc.HParams(weight_decay=0.01))
+    got = orc.muon_step(W, G, M, orc.HParams(weight_decay=0.01, scale_mode=mode))
+    kappa = orc.scale_factor(mode, orc.MOONSHOT_COEF, *shape)
+    np.testing.assert_array_equal(got.M, base.M)
+    np.testing.assert_allclose(got.O, kappa * base.O, rtol=1e-12, atol=1e-15)
