@@ -1,6 +1,7 @@
 """The sharded step's GPU leg at one rank: the library updates the owned
 matrices in place inside the flat weight buffer; with a single rank this must
-equal the ordinary step on separately allocated buffers, bit for bit."""
+equal the ordinary step on separately allocated buffers, bit for bit, with
+the gradients given as separate tensors or in the flat gradient layout."""
 import numpy as np
 import pytest
 import torch
@@ -13,8 +14,9 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 
+@pytest.mark.parametrize("flat_grads", [False, True], ids=["grad_list", "grad_flat"])
 @pytest.mark.parametrize("cond", [False, True])
-def test_sharded_single_rank_matches_plain_step(cond):
+def test_sharded_single_rank_matches_plain_step(cond, flat_grads):
     shapes = workloads.gpt2_small_shapes(layers=1) + workloads.lora_shapes(8, projections=3)
     plan = sharded.plan_shards(shapes, 1)
     sw = sharded.ShardedWeights(plan, dtype=torch.bfloat16, device="cuda")
@@ -36,8 +38,13 @@ def test_sharded_single_rank_matches_plain_step(cond):
     mats = [dm.dm_matrix(Wp[i], G[i], M2[i], er2[i] if cond else None, ec2[i] if cond else None)
             for i in range(len(shapes))]
     ws2 = torch.empty(dm.dm_workspace_size(mats, hp, int(cond)), dtype=torch.uint8, device="cuda")
+    grads = G
+    if flat_grads:
+        grads = sharded.ShardedGrads(plan, dtype=torch.bfloat16, device="cuda")
+        for v, g in zip(grads.views, G):
+            v.copy_(g)
     for _ in range(2):
-        sharded.sharded_step(sw, 0, G, M1, hp, ws1, conditioned=cond, row_energy=er1,
+        sharded.sharded_step(sw, 0, grads, M1, hp, ws1, conditioned=cond, row_energy=er1,
                              col_energy=ec1)
         dm.check((dm.dm_dimuon_step if cond else dm.dm_muon_step)(mats, hp, ws2))
     torch.cuda.synchronize()

@@ -127,3 +127,79 @@ def test_single_rank_gather_is_noop():
     sw.views[0].fill_(3.0)
     sw.gather(0)
     assert float(sw.views[0][0, 0]) == 3.0
+
+
+def _rank_main_dp(rank, world, port, errq):
+    """Data-parallel flavour: every rank holds its own local gradients in the
+    flat layout; one reduce-scatter gives each owner the mean over ranks, the
+    owner steps (the oracle stands in for the GPU step), the weights are
+    all-gathered, and every rank must end with the single-process step on
+    the mean gradient."""
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        plan = sharded.plan_shards(SHAPES, world)
+        sw = sharded.ShardedWeights(plan, dtype=torch.float64, device="cpu")
+        sg = sharded.ShardedGrads(plan, dtype=torch.float64, device="cpu")
+        W, _, M = _inputs()
+        local = _local_grads(world)
+        for i in range(len(SHAPES)):
+            sw.views[i].copy_(torch.from_numpy(W[i]))
+            sg.views[i].copy_(torch.from_numpy(local[rank][i]))
+        sg.reduce(rank)
+        h = orc.HParams(mu=0.9, lr=0.05, weight_decay=0.01)
+        mean = [sum(local[q][i] for q in range(world)) / world for i in range(len(SHAPES))]
+        for i in plan.owned(rank):
+            np.testing.assert_allclose(sg.views[i].numpy(), mean[i], rtol=1e-13, atol=1e-14)
+            sw.views[i].copy_(torch.from_numpy(
+                orc.muon_step(W[i], sg.views[i].numpy(), M[i], h).W))
+        sw.gather(rank)
+        for i in range(len(SHAPES)):
+            want = orc.muon_step(W[i], mean[i], M[i], h).W
+            np.testing.assert_allclose(sw.views[i].numpy(), want, rtol=1e-10, atol=1e-12)
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as e:  # reported to the parent
+        errq.put(f"rank {rank}: {type(e).__name__}: {e}")
+        raise
+
+
+def _local_grads(world):
+    rng = np.random.default_rng(321)
+    return [[rng.standard_normal(s) for s in SHAPES] for _ in range(world)]
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_grad_reduce_scatter_gloo(world):
+    ctx = mp.get_context("spawn")
+    errq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_dp, args=(r, world, port, errq)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    errors = []
+    while not errq.empty():
+        errors.append(errq.get())
+    assert not errors, errors
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+
+
+def test_grads_layout_matches_weights():
+    plan = sharded.plan_shards(SHAPES, 3)
+    sw = sharded.ShardedWeights(plan, dtype=torch.float32, device="cpu")
+    sg = sharded.ShardedGrads(plan, dtype=torch.float32, device="cpu")
+    assert sg.flat.numel() == sw.flat.numel()
+    for a, b in zip(sg.views, sw.views):
+        assert a.shape == b.shape
+        assert a.storage_offset() == b.storage_offset()
+    # one rank: nothing to reduce, no process group needed
+    one = sharded.ShardedGrads(sharded.plan_shards(SHAPES, 1), dtype=torch.float32, device="cpu")
+    one.views[0].fill_(2.0)
+    one.reduce(0)
+    assert float(one.views[0][0, 0]) == 2.0
