@@ -2,8 +2,9 @@
 """Throughput of the B200 Muon / Dimuon step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large_batch|large_batch_dimuon|large_batch_quarter|gpt2_small|square1024|
-                               lora_r2|lora_r8|lora_r32|vec_w1|vec_w2|vec_w8|vec_w32|vec_w128]
+                    [--workload large_batch|large_batch_dimuon|large_batch_quarter|gpt2_small|
+                               square1024|square4096|lora_r2|lora_r8|lora_r32|
+                               vec_w1|vec_w2|vec_w8|vec_w32|vec_w128]
                     [--no-cpu-baseline] [--debug-flags BITS]
 
 Defaults: 50 timed steps after 10 warm-ups, the large batch, one GPU.
@@ -17,6 +18,11 @@ Muon mode, bf16 tensor-core products with fp32 accumulation.
 Each rank runs its own copy of the workload on its own GPU (independent
 problems, no collective on the data path): weak scaling; `value` counts the
 matrices of all ranks.  Rank 0 prints one JSON line.
+
+Workloads whose buffers fit a few times in L2 (126 MB) are timed step by
+step with a 512 MB buffer written between the steps (outside the timed
+events), so every step starts with a cold L2; the large ones run back to
+back (their inputs are larger than L2).
 """
 import argparse
 import json
@@ -56,6 +62,10 @@ def workload_spec(name):
     if name == "square1024":
         return dict(shapes=workloads.single_square_shapes(), cond=False, mdt="bf16", lr=0.02,
                     wd=0.0, moonshot=False, seed=1, desc="one 1024x1024 bf16 matrix, Muon")
+    if name == "square4096":
+        return dict(shapes=workloads.single_square_shapes(4096), cond=False, mdt="bf16",
+                    lr=0.02, wd=0.0, moonshot=False, seed=1,
+                    desc="one 4096x4096 bf16 matrix, Muon, 5 NS5 iterations")
     if name.startswith("lora_r"):
         r = int(name[6:])
         return dict(shapes=workloads.lora_shapes(r), cond=True, mdt="fp32",
@@ -90,8 +100,8 @@ def step_bytes(spec):
 
 
 # DRAM traffic of the tensor-core product per launch (ncu dram__bytes_read.sum +
-# dram__bytes_write.sum), valid only for the kernel build it was taken from:
-# profiles/tc_ns_product_pair_large_batch_quarter.md (quarter batch x 4).
+# dram__bytes_write.sum of the quarter batch, same shapes, scaled by 4), valid
+# only for the kernel build the ncu capture was taken from.
 TRAFFIC_CAPTURED = {"large_batch": 2902e6}
 TRAFFIC_BUILD = "6c1826947c21ad68"
 TRAFFIC_SOURCES = ["k_ns_tc2.cu", "dm_tc_epilogue.cuh", "dm_sm100.cuh"]
@@ -173,17 +183,54 @@ def parse_clock_log(text):
             "samples": len(load)}
 
 
-def oracle_sample_time(spec, ns_steps=5):
-    """Times the fp64 CPU oracle on one matrix of the workload (the cheapest
-    representative: the first shape) with `ns_steps` Newton-Schulz iterations
-    and extrapolates to the whole 5-iteration step by algorithmic flops."""
+L2_BYTES = 126 * 2 ** 20
+FLUSH_BYTES = 512 * 2 ** 20
+
+
+def resident_bytes(spec):
+    """Bytes of the buffers one step touches: G, M, W and the fp32 update
+    each once (the workspace is extra)."""
+    mb = 4 if spec["mdt"] == "fp32" else 2
+    return sum(r * c for r, c in spec["shapes"]) * (2 + mb + 2)
+
+
+def l2_flushed(spec):
+    return resident_bytes(spec) < 3 * L2_BYTES
+
+
+def config_of(spec, world):
+    """The workload description both arms print."""
+    return {"workload": spec["desc"], "matrices": len(spec["shapes"]),
+            "parallelism": f"replica per GPU x{world}",
+            "l2": ("512 MB written between timed steps (per-step CUDA events)" if l2_flushed(spec)
+                   else "inputs larger than L2 (no flush)")}
+
+
+def interleaved_order(shapes):
+    """Matrix indices with the shape classes interleaved (a, b, c, a, b, c,
+    ...), so that any run of consecutive steps samples every class."""
+    classes = {}
+    for i, s in enumerate(shapes):
+        classes.setdefault(s, []).append(i)
+    order, lists = [], list(classes.values())
+    while any(lists):
+        for lst in lists:
+            if lst:
+                order.append(lst.pop(0))
+    return order
+
+
+def oracle_run(spec, idx, ns_steps=5):
+    """Seconds the fp64 CPU oracle takes for one step of matrix `idx` of the
+    workload (input draws excluded)."""
     import oracle as orc
-    shp = spec["shapes"][0]
-    rng = np.random.default_rng(spec["seed"])
+    shp = spec["shapes"][idx]
+    rng = np.random.default_rng(spec["seed"] + idx)
     G = rng.standard_normal(shp)
     W = 0.02 * rng.standard_normal(shp)
     M = np.zeros(shp)
     h = orc.HParams(lr=spec["lr"], weight_decay=spec["wd"], ns_steps=ns_steps,
+                    nesterov=bool(spec.get("nesterov", 0)),
                     scale_mode=orc.SCALE_MOONSHOT if spec["moonshot"] else orc.SCALE_NONE)
     t0 = time.perf_counter()
     if spec["cond"]:
@@ -191,42 +238,64 @@ def oracle_sample_time(spec, ns_steps=5):
                         momentum_dtype=spec["mdt"], weight_dtype="bf16")
     else:
         orc.muon_step(W, G, M, h, momentum_dtype=spec["mdt"], weight_dtype="bf16")
-    dt = time.perf_counter() - t0
-    scale = 5 * ns_flops(spec["shapes"]) / (ns_steps * ns_flops([shp]))
-    what = "" if ns_steps == 5 else f" with {ns_steps} of the 5 Newton-Schulz iterations"
-    return dt, dt * scale, f"one {shp[0]}x{shp[1]} matrix of the workload{what} per step, " \
-                           f"extrapolated to all {len(spec['shapes'])} matrices and 5 iterations " \
-                           f"by algorithmic flops"
+    return time.perf_counter() - t0
 
 
-def run_reference(args, spec, rank):
+def cpu_baseline(spec):
+    """The oracle's time for one whole step of the workload, measured per
+    shape class: one matrix of each (short side, long side) class is run
+    through the full 5-iteration step (a tall matrix is the transposed wide
+    one for the oracle) and the step time is the sum over the workload's
+    matrices of their class's time."""
+    classes = {}
+    for i, (r, c) in enumerate(spec["shapes"]):
+        classes.setdefault((min(r, c), max(r, c)), []).append(i)
+    total = 0.0
+    for key, members in classes.items():
+        total += len(members) * oracle_run(spec, members[0])
+    names = ", ".join(f"{len(m)} x {k[0]}x{k[1]}" for k, m in classes.items())
+    return total, (f"one matrix of each shape class ({names}) timed through the whole "
+                   f"5-iteration step; the step time is the sum over all "
+                   f"{len(spec['shapes'])} matrices of their class's time")
+
+
+def reference_budget(spec):
+    """Matrices per reference step: as many consecutive matrices (in the
+    interleaved order) as make about 2e12 algorithmic flops, at least one."""
+    per = 5 * ns_flops(spec["shapes"]) / len(spec["shapes"])
+    return max(1, int(2e12 // max(per, 1.0)))
+
+
+def run_reference(args, spec, rank, world):
+    """The fp64 oracle as it stands, on the host cores, rank 0 only: each step
+    runs the next few matrices of the workload (interleaved shape classes,
+    cyclically) through the whole step; value = matrices processed / time."""
     if rank != 0:
         return
     threads = os.cpu_count()
-    # each step a bounded sample (one matrix, one Newton-Schulz iteration), so
-    # that the default 50 steps end within a few minutes; it is scaled to the
-    # five-iteration step by the time ratio of the two on the same matrix,
-    # measured once beforehand (untimed), so the per-matrix work outside the
-    # iterations is not multiplied by the iteration count
-    t5, _, _ = oracle_sample_time(spec, ns_steps=5)
-    t1, _, _ = oracle_sample_time(spec, ns_steps=1)
-    ratio = t5 / t1
-    shp = spec["shapes"][0]
-    to_all = ns_flops(spec["shapes"]) / ns_flops([shp])
-    times = []
-    for _ in range(args.steps):
-        dt, _, _ = oracle_sample_time(spec, ns_steps=1)
-        times.append(dt * ratio * to_all)
-    sample = (f"one {shp[0]}x{shp[1]} matrix of the workload with 1 of the 5 Newton-Schulz "
-              f"iterations per step, scaled by that matrix's measured 5- to 1-iteration time "
-              f"ratio ({ratio:.2f}, calibrated once, untimed) and extrapolated to all "
-              f"{len(spec['shapes'])} matrices by algorithmic flops")
-    t = float(np.median(times))
-    value = len(spec["shapes"]) / t
+    order = interleaved_order(spec["shapes"])
+    per_step = min(reference_budget(spec), len(order))
+    pos = 0
+
+    def one_step():
+        nonlocal pos
+        dt = 0.0
+        for _ in range(per_step):
+            dt += oracle_run(spec, order[pos % len(order)])
+            pos += 1
+        return dt
+
+    for _ in range(args.warmup):
+        one_step()
+    t = sum(one_step() for _ in range(args.steps))
+    value = per_step * args.steps / t
+    sample = (f"{per_step} matrix(es) of the workload per step, taken in turn with the shape "
+              f"classes interleaved, each through the whole 5-iteration step (fp64 oracle)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "matrices/s",
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": 1, "ms_per_step": t * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": spec["desc"]},
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(spec, world),
             "cpu_baseline": {"value": value, "unit": "matrices/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "matrices/s", "h2d_bytes_per_step": 0,
@@ -243,15 +312,16 @@ def main():
     ap.add_argument("--workload", default="large_batch")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--debug-flags", type=lambda v: int(v, 0), default=0,
-                    help="library debug_flags (test hooks such as DM_DBG_NO_PDL; none skips work)")
+                    help="library debug_flags (test hooks such as DM_DBG_TC_SINGLE; none skips "
+                         "work)")
     args = ap.parse_args()
-    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+    args.warmup = max(args.warmup, 3)
     spec = workload_spec(args.workload)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        run_reference(args, spec, rank)
+        run_reference(args, spec, rank, world)
         return
 
     import torch
@@ -324,19 +394,37 @@ def main():
     torch.cuda.synchronize(dev)
     graph = capture(hp)
 
+    flush = l2_flushed(spec)
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
     def timed(g, reps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
+        """Device seconds of `reps` replays on the launch stream: one event
+        pair around all of them, or (small workloads) one pair per replay with
+        L2 flushed before each, outside the events."""
         barrier()
         torch.cuda.synchronize(dev)
+        if not flush:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier()
+            return e0.elapsed_time(e1) / 1e3
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(reps):
+            for a, b in evs:
+                flush_buf.fill_(1)
+                a.record(stream)
                 g.replay()
-            e1.record(stream)
+                b.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        return e0.elapsed_time(e1) / 1e3
+        return sum(a.elapsed_time(b) for a, b in evs) / 1e3
 
     for _ in range(args.warmup):
         graph.replay()
@@ -463,17 +551,15 @@ def main():
         launches += 2 + 3 * hp.ns_steps + (3 if spec["cond"] else 0)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        _, full, sample = oracle_sample_time(spec)
+        full, sample = cpu_baseline(spec)
         cpu = {"value": n_mat / full, "unit": "matrices/s", "cores": os.cpu_count(),
                "kind": "oracle", "sample": sample}
     line = {"metric": METRIC, "value": value, "unit": "matrices/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) gradients, N(0,0.02^2) weights)",
-            "config": {"workload": spec["desc"], "matrices": n_mat, "parallelism":
-                       f"replica per GPU x{world}", "l2": "inputs larger than L2 (no flush)",
-                       "cuda_graph": True, "ns_tflops_step": ns_flops(shapes) * hp.ns_steps
-                       / (ms_step / 1e3) / 1e12},
+            "config": config_of(spec, world), "cuda_graph": True,
+            "ns_tflops_step": ns_flops(shapes) * hp.ns_steps / (ms_step / 1e3) / 1e12,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": launches * args.steps}
     print(json.dumps(line), flush=True)

@@ -40,6 +40,7 @@ DM_SCALE_MOONSHOT = 1
 DM_SCALE_JORDAN = 2
 DM_SCALE_BERNSTEIN = 3
 DM_THIN_MAX = 32
+DM_MAX_NS_STEPS = 64
 DM_DBG_NO_THIN = 0x1
 DM_DBG_TC_SINGLE = 0x2
 DM_DBG_TC_PAIR = 0x4
@@ -65,7 +66,7 @@ class dm_hparams_t(ctypes.Structure):
                 ("ns_steps", c_int32), ("a", c_float), ("b", c_float), ("c", c_float),
                 ("cond_eps", c_float), ("scale_mode", c_int32), ("scale_coef", c_float),
                 ("precision", c_int32), ("debug_flags", c_uint32), ("nesterov", c_int32),
-                ("reserved", c_int32 * 3)]
+                ("reserved", c_int32 * 3), ("ns_coeffs", ctypes.POINTER(c_float))]
 
 
 class DimuonError(RuntimeError):
@@ -171,10 +172,34 @@ def _ws(workspace):
 # the C ABI, by name
 # ----------------------------------------------------------------------------
 def dm_default_hparams(**overrides):
+    """dm_hparams_t with the library's defaults and the given fields set.
+    `ns_coeffs` takes a sequence of (a_k, b_k, c_k) triples, one per
+    Newton-Schulz iteration (it also sets ns_steps to its length)."""
     hp = dm_hparams_t()
     _lib.dm_default_hparams(ctypes.byref(hp))
+    coeffs = overrides.pop("ns_coeffs", None)
     for k, v in overrides.items():
         setattr(hp, k, v)
+    if coeffs is not None:
+        set_ns_coeffs(hp, coeffs)
+    return hp
+
+
+def set_ns_coeffs(hp, coeffs):
+    """Points hp.ns_coeffs at a host float array holding the triples (kept
+    alive on the struct) and sets hp.ns_steps to their count; None restores
+    the fixed (a, b, c)."""
+    if coeffs is None:
+        hp.ns_coeffs = None
+        hp._ns_coeffs_keep = None
+        return hp
+    flat = [float(v) for triple in coeffs for v in triple]
+    if len(flat) == 0 or len(flat) % 3:
+        raise ValueError("ns_coeffs must be a non-empty sequence of (a, b, c) triples")
+    arr = (c_float * len(flat))(*flat)
+    hp._ns_coeffs_keep = arr
+    hp.ns_coeffs = ctypes.cast(arr, ctypes.POINTER(c_float))
+    hp.ns_steps = len(flat) // 3
     return hp
 
 

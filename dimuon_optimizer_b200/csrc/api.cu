@@ -9,7 +9,7 @@
 //     K0   (Dimuon) R, C from the previous momentum's energies
 //     K1   momentum, X_0 = R M_t C, partial norms / energies
 //     K1b  energies of M_t, ||X_0||_F scalars
-//     ns_steps x { A = X X^T ; B = bA + cA^2 ; X <- aX + BX }  (tensor cores
+//     ns_steps x { A = X X^T ; B = b_k A + c_k A^2 ; X <- a_k X + BX }  (tensor cores
 //          in DM_PREC_BF16_TC, fp32 SIMT in DM_PREC_FP32); the last product
 //          applies the Muon update or emits X_5
 //     K3a, K3 (Dimuon) renormalise Y = R X_5 C, scale, decay, apply
@@ -75,7 +75,12 @@ struct Layout {
 
 dm_status_t validate(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int cond) {
   if (n < 0 || (n > 0 && !mats) || !hp) return DM_ERR_INVALID_ARG;
-  if (hp->ns_steps < 1 || hp->ns_steps > 64) return DM_ERR_INVALID_ARG;
+  if (hp->ns_steps < 1 || hp->ns_steps > DM_MAX_NS_STEPS) return DM_ERR_INVALID_ARG;
+  if (hp->ns_coeffs)
+    for (int i = 0; i < 3 * hp->ns_steps; ++i) {
+      const float v = hp->ns_coeffs[i];
+      if (!(v == v) || v > 3.0e38f || v < -3.0e38f) return DM_ERR_INVALID_ARG;
+    }
   if (hp->precision != DM_PREC_FP32 && hp->precision != DM_PREC_BF16_TC) return DM_ERR_INVALID_ARG;
   if (hp->scale_mode != DM_SCALE_NONE && hp->scale_mode != DM_SCALE_MOONSHOT &&
       hp->scale_mode != DM_SCALE_JORDAN && hp->scale_mode != DM_SCALE_BERNSTEIN)
@@ -331,6 +336,17 @@ int sm_count(int dev) {
 // ---------------------------- product plans -------------------------------
 enum Phase { PH_SYRK = 0, PH_POLY = 1, PH_GEMM = 2 };
 
+// (a, b, c) of Newton-Schulz iteration k (1-based): the caller's schedule
+// when it gave one, else the fixed quintic.
+struct Coef {
+  float a, b, c;
+};
+Coef coef_of(const dm_hparams_t* hp, int k) {
+  if (!hp->ns_coeffs) return {hp->a, hp->b, hp->c};
+  const float* q = hp->ns_coeffs + 3 * (k - 1);
+  return {q[0], q[1], q[2]};
+}
+
 // Fills the epilogue / shape part of one product; operand sources are set by
 // the caller (tensor maps or pointers).  Returns operand-source descriptors.
 struct OperandSrc {
@@ -364,8 +380,8 @@ OperandSrc fill_gemm(GemmMat& g, const MatPlan& p, const dm_matrix_t& um, const 
     g.aux = ws + p.off_A;
     g.ldaux = (int)p.ldm;
     g.epi = EPI_POLY;
-    g.coef_acc = hp->c;
-    g.coef_aux = hp->b;
+    g.coef_acc = coef_of(hp, k).c;
+    g.coef_aux = coef_of(hp, k).b;
     src = {2, 2};
   } else {
     g.M = (int)p.rows;
@@ -380,7 +396,7 @@ OperandSrc fill_gemm(GemmMat& g, const MatPlan& p, const dm_matrix_t& um, const 
     }
     g.aux = ws + p.off_X[xin];
     g.ldaux = (int)p.ldx;
-    g.coef_aux = hp->a;
+    g.coef_aux = coef_of(hp, k).a;
     if (k == 1) g.scal_idx = SC_INV_S;
     if (k < ns) {
       g.epi = EPI_GEMM;
@@ -493,9 +509,12 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     tp.mu = hp->mu;
     tp.lr = hp->lr;
     tp.decay = decay;
-    tp.a = hp->a;
-    tp.b = hp->b;
-    tp.c = hp->c;
+    for (int k = 1; k <= hp->ns_steps; ++k) {
+      const Coef q = coef_of(hp, k);
+      tp.coef[k - 1][0] = q.a;
+      tp.coef[k - 1][1] = q.b;
+      tp.coef[k - 1][2] = q.c;
+    }
     tp.eps = hp->cond_eps;
     tp.status = status;
     tp.mats = mats_dev;
@@ -560,6 +579,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
       std::memset(&p1, 0, sizeof(p1));
       p1.mu = hp->mu;
       p1.nesterov = hp->nesterov;
+      p1.status = status;
       int tiles = 0;
       for (size_t q = b; q < std::min(big.size(), b + K1_MAX); ++q) {
         const MatPlan& p = *big[q];
@@ -696,6 +716,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
           std::memset(&ps, 0, sizeof(ps));
           ps.lr = hp->lr;
           ps.decay = decay;
+          ps.status = status;
           int tiles = 0;
           for (size_t q = b; q < std::min(big.size(), b + SIMT_MAX); ++q) {
             const MatPlan& p = *big[q];
@@ -725,6 +746,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
       std::memset(&p3, 0, sizeof(p3));
       p3.lr = hp->lr;
       p3.decay = decay;
+      p3.status = status;
       int tiles = 0;
       for (size_t q = b; q < std::min(big.size(), b + K3_MAX); ++q) {
         const MatPlan& p = *big[q];
@@ -780,6 +802,7 @@ void dm_default_hparams(dm_hparams_t* hp) {
   hp->debug_flags = 0;
   hp->nesterov = 0;
   hp->reserved[0] = hp->reserved[1] = hp->reserved[2] = 0;
+  hp->ns_coeffs = nullptr;
 }
 
 dm_status_t dm_workspace_size(const dm_matrix_t* mats, int n, const dm_hparams_t* hp,
@@ -837,6 +860,6 @@ const char* dm_status_string(int32_t status) {
   }
 }
 
-const char* dm_version(void) { return "0.1.0"; }
+const char* dm_version(void) { return "0.2.0"; }
 
 }  // extern "C"

@@ -14,6 +14,7 @@
 // word) and fully writes every other region before reading it.  Calls whose
 // device work overlaps (two streams, two host threads without ordering)
 // race on the array and must not be issued.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -26,21 +27,49 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[DM_NOALLOC_MAX_
 
 constexpr int MAX_DEVICES = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[MAX_DEVICES] = {};
+struct ScratchSlot {
+  CUcontext ctx;  // context the address belongs to
+  void* ptr;
+};
+ScratchSlot g_scratch[MAX_DEVICES] = {};
 
-// Device address of the array on the current device; looked up once per
-// device with that device current.  The host-side symbol itself is only a
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The calling thread's current driver context (null if it has none).
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
+
+// Device address of the array on the current device.  It is looked up once
+// per device with that device current, and again whenever the device's
+// context has changed since (after cudaDeviceReset the array belongs to a new
+// module load, at a new address).  The host-side symbol itself is only a
 // stand-in and must never reach a kernel.
 dm_status_t scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return DM_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  ScratchSlot& slot = g_scratch[dev];
+  if (!slot.ptr || slot.ctx != current_context()) {
     void* p = nullptr;
+    // (the look-up makes the device's primary context current if no
+    // context was, so the context is read after it)
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DM_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx = current_context();
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return DM_OK;
 }
 

@@ -124,6 +124,20 @@ __device__ __forceinline__ void raise_status(int* status, int code) {
   if (status) atomicMax(status, code);
 }
 
+// A bounded wait that gave up also sets the abort word (the int32 after the
+// status word).  Every later launch of the step reads it at its start and
+// returns without writing, so no weight is updated from buffers that a
+// timed-out launch left half written.
+__device__ __forceinline__ void raise_timeout(int* status) {
+  if (!status) return;
+  atomicMax(status, ST_TIMEOUT);
+  atomicExch(status + STATUS_ABORT_WORD, 1);
+}
+
+__device__ __forceinline__ bool step_aborted(const int* status) {
+  return status && *reinterpret_cast<const volatile int*>(status + STATUS_ABORT_WORD) != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

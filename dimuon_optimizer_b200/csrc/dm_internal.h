@@ -6,7 +6,29 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace dm {
+
+// One-time set-up of a launcher (kernel attributes, occupancy queries), run
+// once per device with that device current, safe under concurrent callers.
+// Each launcher keeps its own static DeviceOnce; a failed set-up is
+// remembered and returned on every later call on that device.
+constexpr int MAX_DEVICES = 64;
+struct DeviceOnce {
+  std::once_flag flag[MAX_DEVICES];
+  cudaError_t err[MAX_DEVICES] = {};
+};
+template <class F>
+inline cudaError_t device_once(DeviceOnce& once, int* dev_out, F&& init) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
+  std::call_once(once.flag[dev], [&] { once.err[dev] = init(dev); });
+  if (dev_out) *dev_out = dev;
+  return once.err[dev];
+}
 
 enum { DT_BF16 = 0, DT_FP32 = 1 };
 
@@ -22,6 +44,9 @@ enum {
 
 // Device status codes (mirror dm_status_t).
 enum { ST_OK = 0, ST_TIMEOUT = 5, ST_NONFINITE = 6 };
+// int32 index, after the status word, of the step's abort word (set with
+// ST_TIMEOUT; both live in the workspace header that each step clears).
+constexpr int STATUS_ABORT_WORD = 1;
 
 // debug_flags bit read inside the tensor-core kernels (mirrors the public
 // DM_DBG_FORCE_TIMEOUT).
@@ -65,6 +90,7 @@ constexpr int K1_MAX = 200;
 struct K1Params {
   int count;
   float mu;
+  int* status;
   int nesterov;           // X_0 from B_t = G + mu M_t instead of M_t
   int starts[K1_MAX + 1];
   K1Mat mats[K1_MAX];
@@ -137,6 +163,7 @@ struct SimtMat {
 struct SimtParams {
   int count;
   float lr, decay;
+  int* status;
   int starts[SIMT_MAX + 1];
   SimtMat mats[SIMT_MAX];
 };
@@ -177,6 +204,7 @@ constexpr int K3_MAX = 200;
 struct K3Params {
   int count;
   float lr, decay;
+  int* status;
   int starts[K3_MAX + 1];
   K3Mat mats[K3_MAX];
 };
@@ -221,7 +249,8 @@ struct ThinParams {
   int conditioned;
   int nesterov;
   int ns_steps;
-  float mu, lr, decay, a, b, c, eps;
+  float mu, lr, decay, eps;
+  float coef[64][3];      // (a_k, b_k, c_k) of Newton-Schulz iteration k < ns_steps
   int* status;
   const ThinMat* mats;    // [count]
   const int* starts;      // [count + 1]: first slab of each factor

@@ -63,7 +63,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
-        raise_status(status, ST_TIMEOUT);
+        raise_timeout(status);
         return false;
       }
     }

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(256) k0_conditioning(const __grid_constant__ K
 // covers columns [c0 + 8l, c0 + 8l + 8), warp w covers rows w, w+8, ...
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k1_momentum(const __grid_constant__ K1Params p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   __shared__ float col_acc[8][K1_COLS];
   __shared__ float red[32];
   const int tile = blockIdx.x;
@@ -133,6 +134,7 @@ __global__ void __launch_bounds__(256) k1_momentum(const __grid_constant__ K1Par
 // each produce K1B_THREADS energies (rows first, then columns).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(K1B_THREADS) k1b_reduce(const __grid_constant__ K1bParams p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   __shared__ double red[32];
   const int g = find_group(p.starts, p.count, blockIdx.x);
   const K1bMat& mt = p.mats[g];
@@ -174,6 +176,7 @@ __global__ void __launch_bounds__(K1B_THREADS) k1b_reduce(const __grid_constant_
 // the epilogue of the last Newton-Schulz product.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k3a_factor(const __grid_constant__ K3Params p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   __shared__ double red[32];
   const K3Mat& mt = p.mats[blockIdx.x];
   double sx = 0.0, sy = 0.0;
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(256) k3a_factor(const __grid_constant__ K3Para
 // K3: same tiling as K1.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k3_apply(const __grid_constant__ K3Params p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   const int tile = blockIdx.x;
   const int g = find_group(p.starts, p.count, tile);
   const K3Mat& mt = p.mats[g];

@@ -43,6 +43,7 @@ __device__ __forceinline__ void sym_store_f32(const GemmMat& g, int r, int c, fl
 }
 
 __global__ void __launch_bounds__(256) simt_ns_product(const __grid_constant__ SimtParams p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   __shared__ __align__(16) float As[SK][SB];
   __shared__ __align__(16) float Bs[SK][SB];
   __shared__ float red[2][8];

@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
     }
     mbar_init(drain, 1);
     mbar_init(never, 1);
-    *abort = 0;
+    // an earlier launch of this step gave up on a wait: leave without writing
+    *abort = step_aborted(p.status) ? 1 : 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -256,15 +257,12 @@ int tc_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s) {
   if (p.total_tiles <= 0 || grid <= 0) return cudaSuccess;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(tc_ns_product, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static DeviceOnce once;
+  const cudaError_t e = device_once(once, nullptr, [](int) {
+    return cudaFuncSetAttribute(tc_ns_product, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES);
+  });
+  if (e != cudaSuccess) return e;
   tc_ns_product<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }

@@ -120,7 +120,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
     }
     mbar_init(drain, 1);
     mbar_init(never, 1);
-    *abort = 0;
+    // An earlier launch of this step gave up on a wait: leave without
+    // writing.  Both CTAs of the pair read the abort word at their start; it
+    // only changes when some wait of this launch has run for its full limit,
+    // long after both have read it.  (Were they ever to disagree, the CTA
+    // that goes on ends in its own bounded waits.)
+    *abort = step_aborted(p.status) ? 1 : 0;
     fence_mbar_init();
   }
   if (warp == 1) {  // the same warp of both CTAs allocates collectively
@@ -306,15 +311,12 @@ int tc_pair_bk() { return BK; }
 
 cudaError_t launch_tc_pair(const TcParams& p, int pairs, cudaStream_t s) {
   if (p.total_tiles <= 0 || pairs <= 0) return cudaSuccess;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(tc_ns_product_pair,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static DeviceOnce once;
+  const cudaError_t e = device_once(once, nullptr, [](int) {
+    return cudaFuncSetAttribute(tc_ns_product_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES);
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);

@@ -129,6 +129,7 @@ struct GramFrag {
 
 template <int RP>
 __global__ void __launch_bounds__(TT) thin_gram(const __grid_constant__ ThinParams p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   using Cf = TCfg<RP>;
   using Frag = GramFrag<RP>;
   __shared__ double red_s[TW][2][Cf::PART];
@@ -536,8 +537,8 @@ __device__ double iterate_factor_warp(const ThinParams& p, int f, const ThinMat&
     s.P[i][j] = i == j ? 1.0 : 0.0;
   }
   __syncwarp();
-  const double a = p.a, b = p.b, c = p.c;
   for (int it = 0; it < p.ns_steps; ++it) {
+    const double a = p.coef[it][0], b = p.coef[it][1], c = p.coef[it][2];
     mm_warp<RP>(s.Q, s.A, s.A);
     for (int idx = lane; idx < RP * RP; idx += 32) {
       const int i = idx / RP, j = idx % RP;
@@ -573,6 +574,7 @@ __device__ double iterate_factor_warp(const ThinParams& p, int f, const ThinMat&
 
 template <int RP>
 __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ ThinParams p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   using Cf = TCfg<RP>;
   __shared__ WarpIterSmem<RP> sm[TW];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -623,6 +625,7 @@ __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ 
 
 template <int RP>
 __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinParams p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   using Cf = TCfg<RP>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   IterSmem<RP>& s = *reinterpret_cast<IterSmem<RP>*>(smem_raw);
@@ -682,8 +685,8 @@ __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinP
     s.P[i][j] = i == j ? 1.0 : 0.0;
   }
   __syncthreads();
-  const double a = p.a, b = p.b, c = p.c;
   for (int it = 0; it < p.ns_steps; ++it) {
+    const double a = p.coef[it][0], b = p.coef[it][1], c = p.coef[it][2];
     mm<RP>(s.Q, s.A, s.A);  // Q = A A
     for (int idx = tid; idx < RP * RP; idx += IT) {
       const int i = idx / RP, j = idx % RP;
@@ -751,6 +754,7 @@ struct ApplyFrag {
 
 template <int RP>
 __global__ void __launch_bounds__(TT) thin_apply(const __grid_constant__ ThinParams p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   using Cf = TCfg<RP>;
   using Frag = ApplyFrag<RP>;
   __shared__ double Ts[RP * RP];
@@ -1124,6 +1128,7 @@ __device__ __forceinline__ void store_cols(void* base, int dt, const Geo& q, int
 
 template <int RP>
 __global__ void __launch_bounds__(FT, 4) thin_fused(const __grid_constant__ ThinParams p) {
+  if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   extern __shared__ __align__(16) uint8_t fused_raw[];
   __shared__ WarpIterSmem<RP> it;
   __shared__ double red[FW][2][RP][RP];
@@ -1333,34 +1338,31 @@ cudaError_t launch_iter_rp(const ThinParams& p, cudaStream_t st) {
     return cudaGetLastError();
   }
   const int iter_bytes = (int)sizeof(IterSmem<RP>);
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(thin_iterate<RP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, iter_bytes);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  static DeviceOnce once;
+  const cudaError_t e = device_once(once, nullptr, [&](int) {
+    return cudaFuncSetAttribute(thin_iterate<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                iter_bytes);
+  });
+  if (e != cudaSuccess) return e;
   thin_iterate<RP><<<p.count, IT, iter_bytes, st>>>(p);
   return cudaGetLastError();
 }
 
 template <int RP>
 cudaError_t launch_rp(ThinParams& p, int nsm, cudaStream_t st) {
-  static int configured = -1;
-  static int occ_gram = 1, occ_apply = 1;
+  static DeviceOnce once;
+  static int occ_gram[MAX_DEVICES], occ_apply[MAX_DEVICES];
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    occ_gram = resident_ctas(thin_gram<RP>, 0);
-    occ_apply = resident_ctas(thin_apply<RP>, 0);
-    configured = dev;
-  }
-  p.grid_gram = std::min(p.units, nsm * occ_gram);
-  p.grid_apply = std::min(p.units, nsm * occ_apply);
+  cudaError_t e = device_once(once, &dev, [](int d) {
+    occ_gram[d] = resident_ctas(thin_gram<RP>, 0);
+    occ_apply[d] = resident_ctas(thin_apply<RP>, 0);
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
+  p.grid_gram = std::min(p.units, nsm * occ_gram[dev]);
+  p.grid_apply = std::min(p.units, nsm * occ_apply[dev]);
   thin_gram<RP><<<p.grid_gram, TT, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_iter_rp<RP>(p, st);
   if (e != cudaSuccess) return e;
@@ -1409,15 +1411,12 @@ cudaError_t launch_thin_iterate(const ThinParams& p, cudaStream_t s) {
 namespace {
 template <int RP>
 cudaError_t launch_fused_rp(const ThinParams& p, size_t smem, cudaStream_t st) {
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(thin_fused<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)THIN_FUSED_MAX_SMEM);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  static DeviceOnce once;
+  const cudaError_t e = device_once(once, nullptr, [](int) {
+    return cudaFuncSetAttribute(thin_fused<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)THIN_FUSED_MAX_SMEM);
+  });
+  if (e != cudaSuccess) return e;
   thin_fused<RP><<<p.count, FT, smem, st>>>(p);
   return cudaGetLastError();
 }

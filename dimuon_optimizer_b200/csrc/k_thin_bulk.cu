@@ -63,7 +63,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volat
     if (*abort) return false;
     if (globaltimer_ns() - t0 > WAIT_NS) {
       *abort = 1;
-      raise_status(status, ST_TIMEOUT);
+      raise_timeout(status);
       return false;
     }
   }
@@ -607,10 +607,11 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
     }
     mbar_init(redf, CW);
     mbar_init(redr, CW);
-    *abort = 0;
+    *abort = step_aborted(p.status) ? 1 : 0;
     fence_mbar_init();
   }
   __syncthreads();
+  if (*abort) return;  // an earlier launch of this step timed out
 
   if (warp >= CW) {
     produce<RP, CH, NS, TG, TM, TM, 0>(p, stages, L::STAGE_BYTES, L::OFF_G, 0, L::OFF_E, info, full,
@@ -1048,10 +1049,11 @@ __global__ void __launch_bounds__(ApplyBulk<RP, TG, TM, TW>::BT, ApplyBulk<RP, T
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], CW);
     }
-    *abort = 0;
+    *abort = step_aborted(p.status) ? 1 : 0;
     fence_mbar_init();
   }
   __syncthreads();
+  if (*abort) return;  // an earlier launch of this step timed out
 
   if (warp >= CW) {
     produce<RP, CH, NS, TG, TM, TW, 1>(p, stages, stage_bytes, L::OFF_G, L::OFF_W, L::OFF_E, info, full,
@@ -1125,11 +1127,10 @@ template <int RP, typename TG, typename TM, typename TW>
 cudaError_t launch_bulk_rp(ThinParams& p, int nsm, cudaStream_t st) {
   using LG = GramBulk<RP, TG, TM>;
   using LA = ApplyBulk<RP, TG, TM, TW>;
-  static int configured = -1;
-  static int occ_g = 1, occ_a[2] = {1, 1};
+  static DeviceOnce once;
+  static int occ_g[MAX_DEVICES], occ_a[MAX_DEVICES][2];
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
+  cudaError_t e = device_once(once, &dev, [](int d) {
     cudaError_t e = cudaFuncSetAttribute(thin_gram_bulk<RP, TG, TM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, LG::SMEM);
     if (e == cudaSuccess)
@@ -1143,16 +1144,17 @@ cudaError_t launch_bulk_rp(ThinParams& p, int nsm, cudaStream_t st) {
       e = cudaFuncSetAttribute(thin_apply_bulk<RP, TG, TM, TW>,
                                cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    occ_g = resident(thin_gram_bulk<RP, TG, TM>, LG::BT, LG::SMEM);
-    occ_a[0] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(false));
-    occ_a[1] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(true));
-    configured = dev;
-  }
+    occ_g[d] = resident(thin_gram_bulk<RP, TG, TM>, LG::BT, LG::SMEM);
+    occ_a[d][0] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(false));
+    occ_a[d][1] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(true));
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
   const bool nest = p.nesterov != 0;
-  p.grid_gram = std::min(p.units, nsm * occ_g);
-  p.grid_apply = std::min(p.units, nsm * occ_a[nest ? 1 : 0]);
+  p.grid_gram = std::min(p.units, nsm * occ_g[dev]);
+  p.grid_apply = std::min(p.units, nsm * occ_a[dev][nest ? 1 : 0]);
   thin_gram_bulk<RP, TG, TM><<<p.grid_gram, LG::BT, LG::SMEM, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_thin_iterate(p, st);
   if (e != cudaSuccess) return e;

@@ -19,6 +19,10 @@
  *      on the short side of the matrix (tall matrices are handled transposed).
  *        sitech.ge Muon post, "Instead of SVD - Newton-Schulz";
  *        "Muon Optimizer 정리", "Why orthogonalise".
+ *      Optionally iteration k uses its own (a_k, b_k, c_k) (hp.ns_coeffs): the
+ *      Dimuon page's toy orthogonalises with Polar Express, an iteration of
+ *      this form whose quintic changes from one iteration to the next
+ *      ("16 columns with input size 0.1 to 10").
  *   4. Dimuon only: Y = R X C rescaled to ||X||_F ("the norm is fixed
  *      afterwards", Dimuon page, Problem 4 (c)).  Muon: Y = X.
  *   5. O = kappa Y, kappa = 1 (DM_SCALE_NONE) or
@@ -43,6 +47,13 @@
  *     wait that ran out) are written to a status word inside the workspace;
  *     dm_read_device_status synchronises the stream and reads it.  Each step
  *     clears the word at its start.
+ *   - After a bounded wait has run out (DM_ERR_DEVICE_TIMEOUT), every later
+ *     launch of the same step returns without writing: the weights, updates,
+ *     momenta and energies those launches cover keep their values, so no
+ *     weight is updated from intermediate buffers that the timed-out launch
+ *     left half written.  Only the launch that timed out may have written
+ *     part of its own outputs (in Muon mode, the last Newton-Schulz product
+ *     writes W).
  *   - Calls are re-entrant for distinct workspaces.  Two steps that share a
  *     workspace must be ordered on the device (same stream, or events).
  *   - The enqueued work contains no host synchronisation and no allocation,
@@ -97,6 +108,7 @@ typedef enum {
 } dm_scale_t;
 
 #define DM_THIN_MAX 32
+#define DM_MAX_NS_STEPS 64   /* largest accepted hp.ns_steps */
 
 /* One matrix of the group.  Orientation: rows x cols as stored by the caller.
  *   weight      in/out  rows x cols, weight_dtype
@@ -137,6 +149,16 @@ typedef struct {
                            M_t ("From PCG to Muon", section 3: the
                            momentum-and-Nesterov combination)           */
   int32_t reserved[3];  /* must be zero                                 */
+  const float* ns_coeffs; /* NULL: (a, b, c) above in every iteration.
+                           Else a HOST array of 3 * ns_steps floats:
+                           iteration k (0-based) uses (a_k, b_k, c_k) =
+                           ns_coeffs[3k], ns_coeffs[3k + 1],
+                           ns_coeffs[3k + 2], and a, b, c are ignored.
+                           Read during the call only: the values are
+                           copied into the enqueued launches (a captured
+                           graph keeps them), so the array may be
+                           released when the call returns.  Non-finite
+                           entries are rejected with DM_ERR_INVALID_ARG. */
 } dm_hparams_t;
 
 /* debug_flags bits (test hooks; none of them changes the arithmetic) */
@@ -158,12 +180,17 @@ typedef struct {
                                      issues any copy or product; the launch
                                      then leaves without writing and the
                                      device status reads
-                                     DM_ERR_DEVICE_TIMEOUT.  The step's
-                                     outputs are then meaningless.         */
+                                     DM_ERR_DEVICE_TIMEOUT.  Every later
+                                     launch of the step then returns at
+                                     once, so W and update_out of the
+                                     Newton-Schulz matrices stay as they
+                                     were (their momenta, written before
+                                     the first product, are updated).      */
 
 /* Fills *hp with the defaults: mu 0.95, lr 0.02, wd 0, ns_steps 5,
  * (a,b,c) = (3.4445, -4.7750, 2.0315), cond_eps 1e-4, DM_SCALE_NONE,
- * scale_coef 0.2, DM_PREC_BF16_TC, debug_flags 0, nesterov 0. */
+ * scale_coef 0.2, DM_PREC_BF16_TC, debug_flags 0, nesterov 0,
+ * ns_coeffs NULL. */
 void dm_default_hparams(dm_hparams_t* hp);
 
 /* Bytes of device workspace a step over `mats[0..n)` needs with these

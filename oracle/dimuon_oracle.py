@@ -99,15 +99,22 @@ class HParams:
     scale_mode: int = SCALE_NONE
     scale_coef: float = MOONSHOT_COEF
     nesterov: bool = False
+    # Per-iteration (a_k, b_k, c_k), one triple per Newton-Schulz iteration;
+    # None: the fixed (a, b, c) every iteration (see newton_schulz).
+    ns_coeffs: tuple | None = None
 
     def as_f32(self) -> "HParams":
+        coeffs = None
+        if self.ns_coeffs is not None:
+            coeffs = tuple((f32(a), f32(b), f32(c)) for (a, b, c) in self.ns_coeffs)
         return HParams(mu=f32(self.mu), lr=f32(self.lr),
                        weight_decay=f32(self.weight_decay),
                        ns_steps=int(self.ns_steps), a=f32(self.a),
                        b=f32(self.b), c=f32(self.c),
                        cond_eps=f32(self.cond_eps),
                        scale_mode=int(self.scale_mode),
-                       scale_coef=f32(self.scale_coef), nesterov=bool(self.nesterov))
+                       scale_coef=f32(self.scale_coef), nesterov=bool(self.nesterov),
+                       ns_coeffs=coeffs)
 
 
 # ----------------------------------------------------------------------------
@@ -183,18 +190,28 @@ def frobenius_normalise(X):
 
 
 def newton_schulz(X, steps: int = NS_STEPS, a: float = NS_A, b: float = NS_B,
-                  c: float = NS_C) -> np.ndarray:
+                  c: float = NS_C, coeffs=None) -> np.ndarray:
     """Quintic Newton-Schulz iteration on an already normalised X.
 
     Each step: A = X X^T; B = b A + c A A; X <- a X + B X, i.e.
     X <- aX + b(XX^T)X + c(XX^T)^2 X ([Sitech], "Instead of SVD -
     Newton-Schulz"; coefficients from [MuonNote], "Why orthogonalise").
+
+    `coeffs`, when given, is a schedule: one (a_k, b_k, c_k) per iteration,
+    `steps` of them, used in place of the fixed (a, b, c).  The Dimuon
+    page's toy orthogonalises with Polar Express ([Dimuon], "16 columns with
+    input size 0.1 to 10"), an iteration of this same form whose quintic
+    changes from one iteration to the next; the page prints no
+    coefficients, so only the mechanism is restated here.
     """
     X = np.asarray(X, np.float64)
-    for _ in range(steps):
+    if coeffs is not None and len(coeffs) != steps:
+        raise ValueError("one (a, b, c) triple per iteration")
+    for k in range(steps):
+        ak, bk, ck = (a, b, c) if coeffs is None else coeffs[k]
         A = X @ X.T
-        B = b * A + c * (A @ A)
-        X = a * X + B @ X
+        B = bk * A + ck * (A @ A)
+        X = ak * X + B @ X
     return X
 
 
@@ -274,7 +291,7 @@ def optimizer_step(W_prev, G, M_prev, hp: HParams, *, conditioned: bool,
     if nonfinite or nrm < NORM_FLOOR:
         Y = np.zeros_like(X0)
     else:
-        X5 = newton_schulz(X, hp.ns_steps, hp.a, hp.b, hp.c)
+        X5 = newton_schulz(X, hp.ns_steps, hp.a, hp.b, hp.c, hp.ns_coeffs)
         if R is None:
             Y = X5
         else:

@@ -29,10 +29,11 @@ def test_every_declared_symbol_is_exported():
 
 def test_struct_layouts():
     assert ctypes.sizeof(dm.dm_matrix_t) == 80
-    assert ctypes.sizeof(dm.dm_hparams_t) == 64
+    assert ctypes.sizeof(dm.dm_hparams_t) == 72
     assert dm.dm_matrix_t.update_out.offset == 72
     assert dm.dm_hparams_t.debug_flags.offset == 44
     assert dm.dm_hparams_t.nesterov.offset == 48
+    assert dm.dm_hparams_t.ns_coeffs.offset == 64
 
 
 def test_defaults_and_strings():
@@ -86,6 +87,10 @@ def test_workspace_size_host_only():
     (lambda m, h: setattr(h, "scale_mode", 4), dm.DM_ERR_INVALID_ARG),
     (lambda m, h: setattr(h, "lr", float("nan")), dm.DM_ERR_INVALID_ARG),
     (lambda m, h: setattr(m, "row_energy", None), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: setattr(h, "ns_steps", dm.DM_MAX_NS_STEPS + 1), dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: dm.set_ns_coeffs(h, [(3.0, -4.0, 2.0), (1.0, float("inf"), 0.0)]),
+     dm.DM_ERR_INVALID_ARG),
+    (lambda m, h: dm.set_ns_coeffs(h, [(3.0, float("nan"), 2.0)]), dm.DM_ERR_INVALID_ARG),
 ])
 def test_argument_errors_are_synchronous(mutate, code):
     m = fake_matrix(64, 96)
@@ -104,6 +109,17 @@ def test_every_scale_mode_is_accepted(mode):
     hp = dm.dm_default_hparams(scale_mode=mode)
     assert dm.dm_muon_step([m], hp, (0, 0), stream=0) == dm.DM_ERR_WORKSPACE
     assert dm.dm_workspace_size([m], hp, 0) > 0
+
+
+def test_coefficient_schedule_is_accepted():
+    """A finite per-iteration schedule passes validation (the call then stops
+    at the missing workspace); its length sets ns_steps; the default has none."""
+    m = fake_matrix(64, 96)
+    assert not dm.dm_default_hparams().ns_coeffs
+    hp = dm.dm_default_hparams(ns_coeffs=[(3.4445, -4.775, 2.0315)] * 3 + [(1.875, -1.25, 0.375)])
+    assert hp.ns_steps == 4 and abs(hp.ns_coeffs[9] - 1.875) < 1e-7
+    assert dm.dm_muon_step([m], hp, (0, 0), stream=0) == dm.DM_ERR_WORKSPACE
+    assert dm.dm_workspace_size([m], hp, 0) == dm.dm_workspace_size([m], dm.dm_default_hparams(), 0)
 
 
 def test_workspace_errors():

@@ -43,7 +43,7 @@ def test_ns_flops_uses_the_short_side():
 
 @pytest.mark.parametrize("name,count", [
     ("large_batch", 16), ("large_batch_dimuon", 16), ("large_batch_quarter", 4),
-    ("gpt2_small", 72), ("square1024", 1), ("lora_r2", 448), ("lora_r8", 448),
+    ("gpt2_small", 72), ("square1024", 1), ("square4096", 1), ("lora_r2", 448), ("lora_r8", 448),
     ("lora_r32", 448), ("vec_w1", 64), ("vec_w32", 64), ("vec_w128", 64)])
 def test_workload_table(name, count):
     spec = bench.workload_spec(name)
@@ -85,7 +85,7 @@ def test_clock_log_without_samples():
 
 def test_reference_arm_json_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                          "--steps", "1", "--workload", "square1024"],
+                          "--steps", "2", "--warmup", "3", "--workload", "square1024"],
                          capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
@@ -97,4 +97,31 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["value"] == d["cpu_baseline"]["value"] == d["e2e"]["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"] == bench.workload_spec("square1024")["desc"]
+    # the same workload description, steps and warm-ups as the GPU arm prints
+    assert d["config"] == bench.config_of(bench.workload_spec("square1024"), 1)
+    assert d["steps"] == 2 and d["warmup"] == 3
+    assert d["ms_per_step"] > 0
+
+
+def test_interleaved_order_samples_every_class():
+    shapes = bench.workload_spec("large_batch")["shapes"]
+    order = bench.interleaved_order(shapes)
+    assert sorted(order) == list(range(len(shapes)))
+    first = [shapes[i] for i in order[:3]]
+    assert sorted(first) == sorted({(4096, 4096), (4096, 14336), (14336, 4096)})
+
+
+def test_reference_sample_is_bounded():
+    # about 2e12 algorithmic flops per reference step, at least one matrix
+    assert bench.reference_budget(bench.workload_spec("large_batch")) == 1
+    lora = bench.workload_spec("lora_r8")
+    k = bench.reference_budget(lora)
+    assert k >= len(lora["shapes"])
+
+
+def test_l2_policy():
+    # small workloads are timed with L2 flushed between steps
+    assert bench.l2_flushed(bench.workload_spec("square1024"))
+    assert bench.l2_flushed(bench.workload_spec("lora_r2"))
+    assert not bench.l2_flushed(bench.workload_spec("large_batch"))
+    assert "no flush" in bench.config_of(bench.workload_spec("large_batch"), 1)["l2"]

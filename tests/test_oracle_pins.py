@@ -41,9 +41,10 @@ def bf_transpose(A):
 
 
 def brute_force_step(W, G, M, mu, lr, wd, a, b, c, steps, eps, kappa_coef,
-                     moonshot, e_row=None, e_col=None, nesterov=False):
+                     moonshot, e_row=None, e_col=None, nesterov=False, coeffs=None):
     """Pure-Python restatement of one step on a tiny matrix (lists of floats).
-    Orientation is handled by transposing when rows > cols."""
+    Orientation is handled by transposing when rows > cols.  `coeffs`: one
+    (a, b, c) per iteration in place of the fixed triple."""
     rows, cols = len(G), len(G[0])
     # the stored momentum (fp32 storage) is what the rest of the step reads
     Mt = [[float(np.float32(mu * M[i][j] + G[i][j])) for j in range(cols)]
@@ -63,7 +64,9 @@ def brute_force_step(W, G, M, mu, lr, wd, a, b, c, steps, eps, kappa_coef,
         X0 = bf_transpose(X0)
     nrm = math.sqrt(sum(v * v for r in X0 for v in r))
     X = [[v / nrm for v in r] for r in X0]
-    for _ in range(steps):
+    for it in range(steps):
+        if coeffs is not None:
+            a, b, c = coeffs[it]
         A = bf_matmul(X, bf_transpose(X))
         AA = bf_matmul(A, A)
         Bm = [[b * A[i][j] + c * AA[i][j] for j in range(len(A))]
@@ -557,3 +560,142 @@ def test_scale_rules_scale_the_update_only(mode, shape):
     kappa = orc.scale_factor(mode, orc.MOONSHOT_COEF, *shape)
     np.testing.assert_array_equal(got.M, base.M)
     np.testing.assert_allclose(got.O, kappa * base.O, rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Per-iteration coefficient schedules.  The Dimuon page's toy ("16 columns
+# with input size 0.1 to 10") orthogonalises with Polar Express, whose
+# quintic changes from iteration to iteration; the page prints none of its
+# coefficients, so what is pinned is the mechanism: iteration k applies its
+# own odd quintic p_k to the singular values.
+# ---------------------------------------------------------------------------
+# five distinct quintics; their composition maps [0, 1] into [0, 1]
+SCHEDULE = ((3.4445, -4.7750, 2.0315), (3.0, -3.2, 1.2), (2.5, -2.2, 0.7),
+            (1.875, -1.25, 0.375), (1.5, -0.5, 0.0))
+
+
+@pytest.mark.parametrize("shape", [(5, 9), (9, 9), (16, 40), (3, 70)])
+def test_schedule_equals_composed_spectral_closed_form(shape):
+    """NS with a schedule = U (p_K o ... o p_1)(Sigma / ||X||_F) V^T, each p_k
+    the scalar quintic of its own triple (LAPACK SVD on the other side)."""
+    rng = np.random.default_rng(sum(shape) + 5)
+    X = rng.standard_normal(shape) * np.logspace(-2, 0, shape[1])[None, :]
+    Xn, _ = orc.frobenius_normalise(X)
+    got = orc.newton_schulz(Xn, len(SCHEDULE), coeffs=SCHEDULE)
+    U, S, Vt = np.linalg.svd(X, full_matrices=False)
+    s = S / np.linalg.norm(X)
+    for (a, b, c) in SCHEDULE:
+        s = quintic_scalar(s, a, b, c, 1)
+    np.testing.assert_allclose(got, U @ np.diag(s) @ Vt, atol=1e-12, rtol=0)
+    # the order of the iterations matters: the reversed schedule differs
+    rev = orc.newton_schulz(Xn, len(SCHEDULE), coeffs=SCHEDULE[::-1])
+    assert np.abs(rev - got).max() > 1e-3
+
+
+def test_constant_schedule_is_the_fixed_step():
+    """A schedule that repeats (a, b, c) is the fixed-coefficient step, bit
+    for bit, through the whole Muon and Dimuon step."""
+    rng = np.random.default_rng(21)
+    shape = (24, 40)
+    W, G, M = 0.02 * rng.standard_normal(shape), rng.standard_normal(shape), rng.standard_normal(shape)
+    er, ec = rng.exponential(1.0, shape[0]), rng.exponential(1.0, shape[1])
+    fixed = orc.HParams(ns_steps=4)
+    sched = orc.HParams(ns_steps=4, ns_coeffs=((orc.NS_A, orc.NS_B, orc.NS_C),) * 4)
+    for cond in (False, True):
+        a = orc.optimizer_step(W, G, M, fixed, conditioned=cond, e_row_prev=er, e_col_prev=ec)
+        b = orc.optimizer_step(W, G, M, sched, conditioned=cond, e_row_prev=er, e_col_prev=ec)
+        np.testing.assert_array_equal(a.O, b.O)
+        np.testing.assert_array_equal(a.W, b.W)
+
+
+def _taylor_quintic():
+    """Coefficients of x (1 + u/2 + 3u^2/8), u = 1 - x^2: the second-order
+    binomial series of x (1 - u)^(-1/2) = x / |x|, written from the series'
+    coefficients binom(-1/2, k) (-1)^k, k = 0, 1, 2."""
+    t = [1.0, 0.5, 0.375]
+    # x (t0 + t1 (1 - x^2) + t2 (1 - x^2)^2) = a x + b x^3 + c x^5
+    return (t[0] + t[1] + t[2], -(t[1] + 2 * t[2]), t[2])
+
+
+def test_schedule_ending_in_taylor_steps_reaches_the_polar_factor():
+    """Five page iterations followed by Taylor steps (fixed point 1 with zero
+    slope) drive every singular value to 1: the result is the LAPACK polar
+    factor U V^T to 1e-9 ([MuonNote], 'Why orthogonalise')."""
+    a, b, c = _taylor_quintic()
+    assert (a, b, c) == (1.875, -1.25, 0.375)
+    sched = ((orc.NS_A, orc.NS_B, orc.NS_C),) * 5 + ((a, b, c),) * 6
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((20, 50))   # well conditioned: sigma_min / ||X|| ~ 0.1
+    Xn, _ = orc.frobenius_normalise(X)
+    got = orc.newton_schulz(Xn, len(sched), coeffs=sched)
+    np.testing.assert_allclose(got, orc.polar_factor_svd(X), atol=1e-9, rtol=0)
+
+
+@pytest.mark.parametrize("shape", [(4, 7), (7, 4)])
+def test_schedule_brute_force_step(shape):
+    """Pure-Python loops with a per-iteration schedule reproduce the oracle's
+    Muon and Dimuon step (wide and tall)."""
+    rng = np.random.default_rng(shape[0] * 7 + shape[1])
+    W = 0.02 * rng.standard_normal(shape)
+    G = rng.standard_normal(shape)
+    M = rng.standard_normal(shape)
+    e_r, e_c = rng.exponential(1.0, shape[0]), rng.exponential(1.0, shape[1])
+    hp = orc.HParams(mu=0.9, lr=0.03, weight_decay=0.02, ns_steps=len(SCHEDULE),
+                     ns_coeffs=SCHEDULE)
+    h = hp.as_f32()
+    for cond in (False, True):
+        want = brute_force_step(W.tolist(), G.tolist(), M.tolist(), h.mu, h.lr,
+                                h.weight_decay, h.a, h.b, h.c, h.ns_steps, h.cond_eps,
+                                h.scale_coef, False, e_r.tolist() if cond else None,
+                                e_c.tolist() if cond else None, coeffs=h.ns_coeffs)
+        got = orc.optimizer_step(W, G, M, hp, conditioned=cond, e_row_prev=e_r,
+                                 e_col_prev=e_c, momentum_dtype="fp32", weight_dtype="fp32")
+        np.testing.assert_allclose(got.O, want[2], rtol=1e-10, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# torch.optim.Muon (a library implementation of the same step) pins the
+# Jordan and Moonshot scale rules and the update's structure.  Its momentum
+# is an average, buf <- mu buf + (1 - mu) g; with G = (1 - mu) g the
+# oracle's M_t = mu M_{t-1} + G is that buffer, and its Nesterov input
+# g + mu (buf - g) is the oracle's B_t = G + mu M_t.  Its adjustment
+# "original" is kappa = sqrt(max(1, rows / cols)) and "match_rms_adamw" is
+# kappa = 0.2 sqrt(max(rows, cols)).  It orthogonalises in bf16, hence the
+# bf16 tolerance on the update.  (Bernstein's rule has no such library
+# counterpart and stays unpinned.)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(96, 40), (40, 96), (64, 64)])
+def test_scale_rules_match_torch_muon_adjustment(shape):
+    from torch.optim import _muon
+    assert orc.scale_factor(orc.SCALE_JORDAN, 0.2, *shape) == pytest.approx(
+        _muon._adjust_lr(1.0, "original", torch.Size(shape)), rel=1e-15)
+    assert orc.scale_factor(orc.SCALE_MOONSHOT, 0.2, *shape) == pytest.approx(
+        _muon._adjust_lr(1.0, "match_rms_adamw", torch.Size(shape)), rel=1e-15)
+
+
+@pytest.mark.parametrize("shape", [(48, 20), (20, 48)])
+@pytest.mark.parametrize("rule", ["original", "match_rms_adamw"])
+@pytest.mark.parametrize("nesterov", [False, True])
+def test_step_matches_torch_muon(shape, rule, nesterov):
+    mode = orc.SCALE_JORDAN if rule == "original" else orc.SCALE_MOONSHOT
+    mu, lr, wd = 0.9, 0.05, 0.1
+    rng = np.random.default_rng(shape[0] + 3 * shape[1] + nesterov)
+    W0 = 0.02 * rng.standard_normal(shape)
+    p = torch.nn.Parameter(torch.from_numpy(W0.astype(np.float32)))
+    opt = torch.optim.Muon([p], lr=lr, weight_decay=wd, momentum=mu, nesterov=nesterov,
+                           adjust_lr_fn=rule)
+    W, M = np.float32(W0).astype(np.float64), np.zeros(shape)
+    hp = orc.HParams(mu=mu, lr=lr, weight_decay=wd, scale_mode=mode, nesterov=nesterov)
+    for t in range(3):
+        g = rng.standard_normal(shape).astype(np.float32)
+        p.grad = torch.from_numpy(g)
+        opt.step()
+        res = orc.muon_step(W, (1.0 - np.float32(mu)) * g.astype(np.float64), M, hp,
+                            momentum_dtype="fp32", weight_dtype="fp32")
+        Wt = p.detach().numpy().astype(np.float64)
+        # the update part of W, relative to its size (bf16 orthogonalisation)
+        dw_t, dw_o = Wt - (1 - lr * wd) * W, res.W - (1 - lr * wd) * W
+        assert np.linalg.norm(dw_t - dw_o) <= 3e-2 * np.linalg.norm(dw_o), t
+        # teacher forcing: continue both from torch's state
+        W = Wt
+        M = opt.state[p]["momentum_buffer"].numpy().astype(np.float64)

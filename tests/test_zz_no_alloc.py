@@ -4,6 +4,11 @@ device, or a latency-critical path where cudaMalloc would synchronise).  Its
 scratch memory is the library's own fixed 32 MiB device array, so its results
 must match the workspace-taking entry points on the same inputs, call after
 call, even though every call reuses what the previous one left in the array.
+
+Neither side may depend on scratch contents it did not write: the reference
+workspace is filled with 0xFF bytes (NaN as fp32 / bf16) before every call,
+and before the compared calls the array is left holding another group's
+results (other shapes, the other mode).
 """
 import numpy as np
 import pytest
@@ -13,6 +18,7 @@ import dimuon_optimizer_b200 as dm
 from gpu_harness import TOL_FP32, Group, rel_fro, storage_ulp, to_dev, to_host
 
 SHAPES = [(256, 384), (300, 200), (8, 512), (40, 100)]
+FOREIGN = [(520, 136), (2, 2056), (64, 96), (4096, 32)]
 
 
 def grads(step):
@@ -42,6 +48,14 @@ def test_noalloc_matches_workspace_entry_point(conditioned):
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     ws = None
     step_fn = dm.dm_dimuon_step if conditioned else dm.dm_muon_step
+    # another group, in the other mode, leaves its results in the array
+    other = Group(FOREIGN, dm.DM_BF16, dm.DM_BF16, dm.DM_FP32, cond=not conditioned, seed=32)
+    rng = np.random.default_rng(60)
+    for _ in range(2):
+        Gf = [to_dev(rng.standard_normal(s), dm.DM_BF16) for s in FOREIGN]
+        dm.check(dm.dm_step_noalloc(other.matrices(Gf), hp, 1 - conditioned, status))
+    torch.cuda.synchronize()
+    assert int(status.item()) == dm.DM_OK
     for step in range(2):  # two calls in a row on the shared array
         G = [to_dev(g, dm.DM_BF16) for g in grads(step)]
         mats_ref = ref.matrices(G)
@@ -49,6 +63,7 @@ def test_noalloc_matches_workspace_entry_point(conditioned):
             ws = torch.empty(dm.dm_workspace_size(mats_ref, hp, conditioned), dtype=torch.uint8,
                              device="cuda")
         assert dm.dm_workspace_size(mats_ref, hp, conditioned) <= dm.DM_NOALLOC_MAX_BYTES
+        ws.fill_(0xFF)  # poison: a read of scratch the step did not write shows up as NaN
         dm.check(step_fn(mats_ref, hp, ws))
         dm.check(dm.dm_step_noalloc(new.matrices(G), hp, conditioned, status))
         torch.cuda.synchronize()
