@@ -5,9 +5,17 @@
                     [--workload large_batch|large_batch_dimuon|large_batch_quarter|gpt2_small|
                                square1024|square4096|lora_r2|lora_r8|lora_r32|
                                vec_w1|vec_w2|vec_w8|vec_w32|vec_w128]
-                    [--no-cpu-baseline] [--debug-flags BITS]
+                    [--no-cpu-baseline] [--debug-flags BITS] [--sharded]
 
 Defaults: 50 timed steps after 10 warm-ups, the large batch, one GPU.
+
+--sharded times the data-parallel form instead of replicas: ONE copy of the
+workload split over the N ranks by whole matrices (dimuon_optimizer_b200.sharded:
+balanced ownership, flat rank-contiguous buffers); each step is the
+reduce-scatter of every rank's local gradients (NCCL), the library step on the
+owned matrices and the all-gather of the updated weights (NCCL).  Strong
+scaling: `value` is the workload's matrices per second; the line also gives
+the exchange's own time.
 
 One step = one optimizer step (momentum, normalisation, five Newton-Schulz
 iterations, scale, decay, apply) over every matrix of the workload.  The
@@ -303,6 +311,103 @@ def run_reference(args, spec, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def sharded_line(spec, world, steps, warmup, t_step, t_exchange, plan_loads, clocks, launches,
+                 slice_elems=0):
+    """JSON line of the --sharded mode (strong scaling over `world` ranks).
+    Exchange bytes per rank and step: the reduce-scatter sends and the
+    all-gather receives world - 1 bf16 slices each."""
+    n_mat = len(spec["shapes"])
+    cfg = config_of(spec, world)
+    cfg["parallelism"] = (f"whole-matrix sharding over {world} rank(s): reduce-scatter of "
+                          f"gradients, library step on owned matrices, all-gather of weights")
+    return {"metric": METRIC, "value": n_mat / t_step, "unit": "matrices/s", "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": t_step * 1e3,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) gradients, N(0,0.02^2) weights)",
+            "config": cfg, "exchange_ms_per_step": t_exchange * 1e3,
+            "exchange_bytes_per_step": 2 * (world - 1) * slice_elems * 2,
+            "plan_load_s": plan_loads, "clocks": clocks,
+            "gpu_launches": launches, "mode": "sharded"}
+
+
+def run_sharded(args, spec, rank, world, local):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import dimuon_optimizer_b200 as dm
+    from dimuon_optimizer_b200 import sharded
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    shapes = spec["shapes"]
+    plan = sharded.plan_shards(shapes, world)
+    mdt = torch.float32 if spec["mdt"] == "fp32" else torch.bfloat16
+    sw = sharded.ShardedWeights(plan, dtype=torch.bfloat16, device=dev)
+    sg = sharded.ShardedGrads(plan, dtype=torch.bfloat16, device=dev)
+    torch.manual_seed(spec["seed"] + 1000)
+    sw.flat.copy_((0.02 * torch.randn(sw.flat.numel(), device=dev)).to(torch.bfloat16))
+    own = plan.owned(rank)
+    M = {i: torch.zeros(shapes[i], dtype=mdt, device=dev) for i in own}
+    ER = {i: torch.zeros(shapes[i][0], device=dev) for i in own} if spec["cond"] else None
+    EC = {i: torch.zeros(shapes[i][1], device=dev) for i in own} if spec["cond"] else None
+    g_local = torch.Generator(device=dev)
+    g_local.manual_seed(spec["seed"] + 17 * rank)
+    local_grads = torch.randn(sg.flat.numel(), generator=g_local, device=dev).to(torch.bfloat16)
+    hp = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"],
+                               scale_mode=dm.DM_SCALE_MOONSHOT if spec["moonshot"]
+                               else dm.DM_SCALE_NONE, nesterov=spec.get("nesterov", 0))
+    nbytes = sharded.workspace_bytes(sw, rank, sg.views, M, hp, spec["cond"], ER, EC)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        sg.flat.copy_(local_grads)  # this rank's backward output
+        sharded.sharded_step(sw, rank, sg, M, hp, ws, conditioned=spec["cond"], row_energy=ER,
+                             col_energy=EC)
+
+    def exchange_only():
+        sg.reduce(rank)
+        sw.gather(rank)
+
+    def timed(fn, reps):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        t = e0.elapsed_time(e1) / 1e3
+        if world > 1:
+            x = torch.tensor([t], dtype=torch.float64, device=dev)
+            dist.all_reduce(x, op=dist.ReduceOp.MAX)
+            t = float(x.item())
+        return t
+
+    for _ in range(args.warmup):
+        step()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    t_step = timed(step, args.steps) / args.steps
+    clocks = sampler.stop()
+    t_ex = timed(exchange_only, args.steps) / args.steps
+    loads = [plan.load(q) for q in range(world)]
+    n_big = sum(1 for i in own if min(shapes[i]) > dm.DM_THIN_MAX)
+    launches = (2 + 3 * hp.ns_steps + (3 if spec["cond"] else 0)) if n_big else 0
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(sharded_line(spec, world, args.steps, args.warmup, t_step, t_ex, loads,
+                                      clocks, launches * args.steps, plan.slice_elems)),
+              flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -314,6 +419,8 @@ def main():
     ap.add_argument("--debug-flags", type=lambda v: int(v, 0), default=0,
                     help="library debug_flags (test hooks such as DM_DBG_TC_SINGLE; none skips "
                          "work)")
+    ap.add_argument("--sharded", action="store_true",
+                    help="one workload sharded over the ranks (strong scaling) instead of replicas")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     spec = workload_spec(args.workload)
@@ -322,6 +429,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, spec, rank, world)
+        return
+    if args.sharded:
+        run_sharded(args, spec, rank, world, local)
         return
 
     import torch

@@ -39,10 +39,12 @@ the repository's design notes):
     ([MuonNote], "Scaling up": AdamW's weight decay).
   * Tall matrices are orthogonalised on their short side: X is transposed so
     that rows <= cols; R and C swap roles; the result is transposed back.
-  * Degenerate norms: when ||X_0||_F is non-finite, or below 1e-15 (its
-    square below 1e-30, where fp32 cannot form 1/||X_0||^2), the update O_t
-    is zero and W is only decayed; a non-finite norm is also reported as a
-    flag.
+  * Degenerate norms: when ||X_0||_F is non-finite the update O_t is zero,
+    W is only decayed and a flag is reported.  Below 1e-15 the update is zero
+    too: that floor is not a reading of the pages (they are silent) but the
+    CUDA library's implementation limit (it carries 1/||X_0||^2 as an fp32
+    scalar, which overflows below it); the oracle applies the same floor so
+    that the two agree.
   * Hyper-parameters reach the CUDA library as float32; the oracle rounds each
     scalar through float32 before using it in fp64 arithmetic.
   * Nesterov (optional, off by default): the matrix fed to the
@@ -72,7 +74,7 @@ NS_C = 2.0315
 NS_STEPS = 5
 COND_EPS = 1e-4          # [Dimuon], Problem 4: (relative energy + 1e-4)^(-1/4)
 MOONSHOT_COEF = 0.2      # RMS-matching coefficient (see module docstring)
-NORM_FLOOR = 1e-15      # ||X_0||_F below this: zero update (see module docstring)
+NORM_FLOOR = 1e-15      # ||X_0||_F below this: zero update (library limit, see docstring)
 
 SCALE_NONE = 0
 SCALE_MOONSHOT = 1

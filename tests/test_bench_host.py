@@ -125,3 +125,20 @@ def test_l2_policy():
     assert bench.l2_flushed(bench.workload_spec("lora_r2"))
     assert not bench.l2_flushed(bench.workload_spec("large_batch"))
     assert "no flush" in bench.config_of(bench.workload_spec("large_batch"), 1)["l2"]
+
+
+def test_sharded_line_shape():
+    """The --sharded mode's JSON line: strong scaling, the workload's matrices
+    per second over the step time, the exchange time beside it."""
+    spec = bench.workload_spec("gpt2_small")
+    d = bench.sharded_line(spec, 4, 10, 5, 2e-3, 3e-4, [1.0, 1.0, 1.1, 0.9],
+                           {"sm_mhz": 1900.0}, 170, slice_elems=1000)
+    assert d["exchange_bytes_per_step"] == 2 * 3 * 1000 * 2
+    assert d["scaling"] == "strong" and d["mode"] == "sharded"
+    assert d["value"] == pytest.approx(72 / 2e-3)
+    assert d["ms_per_step"] == pytest.approx(2.0)
+    assert d["exchange_ms_per_step"] == pytest.approx(0.3)
+    assert d["n_gpus"] == 4 and d["steps"] == 10 and d["warmup"] == 5
+    assert "reduce-scatter" in d["config"]["parallelism"]
+    assert d["config"]["workload"] == spec["desc"]
+    json.dumps(d)
