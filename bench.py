@@ -398,8 +398,11 @@ def run_sharded(args, spec, rank, world, local):
     clocks = sampler.stop()
     t_ex = timed(exchange_only, args.steps) / args.steps
     loads = [plan.load(q) for q in range(world)]
-    n_big = sum(1 for i in own if min(shapes[i]) > dm.DM_THIN_MAX)
-    launches = (2 + 3 * hp.ns_steps + (3 if spec["cond"] else 0)) if n_big else 0
+    launches = 0
+    if own:
+        launches = dm.dm_step_launches(
+            [dm.dm_matrix(sw.views[i], sg.views[i], M[i], ER[i] if ER else None,
+                          EC[i] if EC else None) for i in own], hp, int(spec["cond"]))
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -637,28 +640,7 @@ def main():
 
     if rank != 0:
         return
-    thin = sum(1 for s in shapes if min(s) <= dm.DM_THIN_MAX)
-    big = n_mat - thin
-    launches = 0
-    if thin:
-        # per padded short side: thin_setup (448 factors per launch), then the
-        # Gram, r x r iteration and apply launches, or for r = 2 on the staged
-        # layout with the momentum fitting 96 KB of shared memory the one
-        # single-pass launch
-        pads = {}
-        for s in shapes:
-            r = min(s)
-            if r <= dm.DM_THIN_MAX:
-                pad = r if r <= 4 else 8 if r <= 8 else 16 if r <= 16 else 32
-                pads.setdefault(pad, []).append(s)
-        nest = 2 if hp.nesterov else 1
-        for pad, group in pads.items():
-            fused = (pad == 2 and not (args.debug_flags & dm.DM_DBG_THIN_STAGED) and
-                     all(min(s) == 2 and max(s) % 8 == 0 and max(s) * 2 * 4 * nest <= 96 * 1024
-                         for s in group))
-            launches += math.ceil(len(group) / 448) + (1 if fused else 3)
-    if big:
-        launches += 2 + 3 * hp.ns_steps + (3 if spec["cond"] else 0)
+    launches = dm.dm_step_launches(mats, hp, int(spec["cond"]))
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         full, sample = cpu_baseline(spec)

@@ -30,6 +30,7 @@ DM_ERR_WORKSPACE = 3
 DM_ERR_CUDA = 4
 DM_ERR_DEVICE_TIMEOUT = 5
 DM_ERR_NONFINITE = 6
+DM_ERR_CANARY = 7
 
 DM_BF16 = 0
 DM_FP32 = 1
@@ -47,11 +48,13 @@ DM_DBG_TC_PAIR = 0x4
 DM_DBG_FORCE_TIMEOUT = 0x8
 DM_DBG_THIN_REGS = 0x10
 DM_DBG_THIN_STAGED = 0x20
+DM_DBG_CANARY = 0x40
 
 DM_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 
-EXPORTED = ("dm_default_hparams", "dm_workspace_size", "dm_muon_step", "dm_dimuon_step",
-            "dm_read_device_status", "dm_step_noalloc", "dm_status_string", "dm_version")
+EXPORTED = ("dm_default_hparams", "dm_workspace_size", "dm_step_launches", "dm_muon_step",
+            "dm_dimuon_step", "dm_read_device_status", "dm_step_noalloc", "dm_status_string",
+            "dm_version")
 
 
 class dm_matrix_t(ctypes.Structure):
@@ -86,6 +89,9 @@ def _load():
     lib.dm_workspace_size.argtypes = [P(dm_matrix_t), c_int, P(dm_hparams_t), c_int,
                                       P(c_size_t)]
     lib.dm_workspace_size.restype = c_int
+    lib.dm_step_launches.argtypes = [P(dm_matrix_t), c_int, P(dm_hparams_t), c_int,
+                                     P(c_int64)]
+    lib.dm_step_launches.restype = c_int
     for name in ("dm_muon_step", "dm_dimuon_step"):
         fn = getattr(lib, name)
         fn.argtypes = [P(dm_matrix_t), c_int, P(dm_hparams_t), c_void_p, c_size_t, c_void_p]
@@ -207,6 +213,16 @@ def dm_workspace_size(mats, hp, conditioned):
     arr, n = _array(mats)
     out = c_size_t(0)
     st = _lib.dm_workspace_size(arr, n, ctypes.byref(hp), int(conditioned), ctypes.byref(out))
+    if st != DM_OK:
+        raise DimuonError(st)
+    return out.value
+
+
+def dm_step_launches(mats, hp, conditioned):
+    """Kernel launches one step enqueues (host-only query)."""
+    arr, n = _array(mats)
+    out = c_int64(0)
+    st = _lib.dm_step_launches(arr, n, ctypes.byref(hp), int(conditioned), ctypes.byref(out))
     if st != DM_OK:
         raise DimuonError(st)
     return out.value

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdimuon.so")
-SOURCES = ["api.cu", "api_noalloc.cu", "k_elementwise.cu", "k_ns_simt.cu", "k_ns_tc.cu", "k_ns_tc2.cu", "k_thin.cu", "k_thin_bulk.cu"]
+SOURCES = ["api.cu", "api_noalloc.cu", "k_elementwise.cu", "k_ns_simt.cu", "k_ns_tc.cu", "k_ns_tc2.cu", "k_thin.cu", "k_thin_bulk.cu", "k_thin_cluster.cu"]
 HEADERS = ["dm_common.cuh", "dm_internal.h", "dm_sm100.cuh", "dm_tiles.cuh", "dm_tc_epilogue.cuh", "dm_thin.cuh"]
 
 

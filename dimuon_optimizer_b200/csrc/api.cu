@@ -54,6 +54,9 @@ struct MatPlan {
 struct ThinLaunch {
   int pad;
   int combo;                // storage combination of the staged path, -1 = register path
+  int cs = 0;               // CTAs per factor of the single-launch cluster kernel, 0 = not used
+  bool fused = false;       // r = 2 single-pass kernel (one CTA per factor)
+  size_t fused_smem = 0;
   std::vector<int> idx;     // matrix indices
   std::vector<int> starts;  // first slab of each factor, plus the total
   size_t off_mats, off_starts, off_unit_f, off_part, off_rpart, off_T, off_fsc;
@@ -65,9 +68,14 @@ constexpr size_t THIN_CTR_OFFSET = 64;
 
 int thin_pad(int r) { return r <= 4 ? r : r <= 8 ? 8 : r <= 16 ? 16 : 32; }
 
+// Shared memory per CTA the cluster kernel's slices may take: with the
+// kernel's static arrays four to five CTAs stay resident per SM.
+constexpr size_t THIN_CL_BUDGET = 40 * 1024;
+
 struct Layout {
   std::vector<MatPlan> mats;
   std::vector<ThinLaunch> thin;
+  std::vector<uint32_t> canary;  // checked mode: 256-byte canary blocks (offset / 256)
   size_t bytes = 0;
   bool tc = false;
   bool cond = false;
@@ -111,11 +119,21 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
   L.tc = hp->precision == DM_PREC_BF16_TC;
   L.cond = cond != 0;
   const size_t esz = L.tc ? 2 : 4;
+  const bool canaries = (hp->debug_flags & DM_DBG_CANARY) != 0;
   size_t cur = HEADER_BYTES;
+  // checked mode: a 256-byte canary after the header and after every region
+  auto guard = [&]() {
+    if (!canaries) return;
+    cur = round_up(cur, 256);
+    L.canary.push_back((uint32_t)(cur / 256));
+    cur += 256;
+  };
+  guard();
   auto take = [&](size_t bytes, size_t align) {
     cur = round_up(cur, align);
     const size_t o = cur;
     cur += round_up(bytes, 16);
+    guard();
     return o;
   };
   for (int i = 0; i < n; ++i) {
@@ -197,6 +215,29 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
     tl.off_rpart = take(units * tl.pad * sizeof(float), 256);
     tl.off_T = take(count * tl.pad * tl.pad * sizeof(double), 256);
     tl.off_fsc = take(count * 4 * sizeof(double), 256);
+    // single-launch cluster kernel: the smallest cluster whose per-CTA slice
+    // of every factor of the group fits the budget
+    if (tl.combo >= 0 && (tl.pad == 2 || tl.pad == 4 || tl.pad == 8) &&
+        !(hp->debug_flags & (DM_DBG_THIN_STAGED | DM_DBG_THIN_REGS))) {
+      for (int cs = 1; cs <= THIN_CL_MAX_CS && !tl.cs; cs *= 2) {
+        bool ok = true;
+        for (int i : tl.idx) {
+          const MatPlan& p = L.mats[i];
+          const size_t b = thin_cluster_smem(tl.pad, tl.combo, cs, p.n, p.tall, hp->nesterov != 0);
+          ok = ok && b > 0 && b <= THIN_CL_BUDGET;
+        }
+        if (ok) tl.cs = cs;
+      }
+    }
+    // else r = 2 on the staged layout whose momentum (and Nesterov gradient)
+    // fits one CTA's shared memory: the single-pass kernel
+    if (!tl.cs) {
+      int64_t max_n = 0;
+      for (int i : tl.idx) max_n = std::max<int64_t>(max_n, L.mats[i].n);
+      tl.fused_smem = thin_fused_smem(tl.pad, max_n, hp->nesterov != 0);
+      tl.fused = tl.combo >= 0 && tl.pad == 2 && tl.fused_smem <= THIN_FUSED_MAX_SMEM &&
+                 !(hp->debug_flags & DM_DBG_THIN_STAGED);
+    }
     L.thin.push_back(std::move(tl));
   }
   L.bytes = round_up(cur, 1024);
@@ -442,6 +483,9 @@ float kappa_of(const dm_hparams_t* hp, int64_t rows, int64_t cols) {
     if ((x) != cudaSuccess) return DM_ERR_CUDA; \
   } while (0)
 
+dm_status_t run_body(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, const Layout& L,
+                     uint8_t* ws, cudaStream_t s, int cond, int dev);
+
 dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, void* workspace,
                      size_t ws_bytes, void* stream_v, int cond) {
   dm_status_t st = validate(mats, n, hp, cond);
@@ -454,15 +498,93 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
   int* status = reinterpret_cast<int*>(ws);
   int dev = 0;
   DM_CUDA(cudaGetDevice(&dev));
-  const float decay = 1.f - hp->lr * hp->weight_decay;
 
-  // status word and thin slab counters
-  DM_CUDA(cudaMemsetAsync(ws, 0, THIN_CTR_OFFSET + 2 * sizeof(int) * L.thin.size(), s));
+  // status word and thin slab counters; outside the checked mode the whole
+  // header, so a later checked step finds no stale arm word
+  const bool canaries = !L.canary.empty();
+  DM_CUDA(cudaMemsetAsync(ws, 0, canaries ? THIN_CTR_OFFSET + 2 * sizeof(int) * L.thin.size()
+                                          : HEADER_BYTES, s));
+  auto canary_pass = [&](int mode) -> cudaError_t {
+    static thread_local CanaryParams cp;
+    for (size_t b = 0; b < L.canary.size(); b += CANARY_MAX) {
+      cp.count = (int)std::min<size_t>(CANARY_MAX, L.canary.size() - b);
+      cp.mode = mode;
+      cp.status = status;
+      std::memcpy(cp.blk, L.canary.data() + b, sizeof(uint32_t) * cp.count);
+      const cudaError_t e = launch_canary(cp, s);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  };
+  if (canaries) DM_CUDA(canary_pass(0));
+  const dm_status_t body = run_body(mats, n, hp, L, ws, s, cond, dev);
+  if (body != DM_OK) return body;
+  if (canaries) DM_CUDA(canary_pass(1));
+  return DM_OK;
+}
+
+// The step's kernels (between the header clear and the canary check).
+dm_status_t run_body(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, const Layout& L,
+                     uint8_t* ws, cudaStream_t s, int cond, int dev) {
+  int* status = reinterpret_cast<int*>(ws);
+  const float decay = 1.f - hp->lr * hp->weight_decay;
   if (n == 0) return DM_OK;
 
   // ---------------------------- thin factors -------------------------------
   for (size_t gi = 0; gi < L.thin.size(); ++gi) {
     const ThinLaunch& tl = L.thin[gi];
+    auto thin_desc = [&](int idx) {
+      const dm_matrix_t& um = mats[idx];
+      ThinMat t;
+      std::memset(&t, 0, sizeof(t));
+      t.G = um.grad;
+      t.M = um.momentum;
+      t.W = um.weight;
+      t.upd = um.update_out;
+      t.e_row = cond ? um.row_energy : nullptr;
+      t.e_col = cond ? um.col_energy : nullptr;
+      t.rows = (int32_t)um.rows;
+      t.cols = (int32_t)um.cols;
+      t.gdt = (uint8_t)um.grad_dtype;
+      t.mdt = (uint8_t)um.momentum_dtype;
+      t.wdt = (uint8_t)um.weight_dtype;
+      t.kappa = kappa_of(hp, um.rows, um.cols);
+      auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+      t.vec = (uint8_t)(al16(um.grad) && al16(um.momentum) && al16(um.weight) && al16(um.update_out));
+      return t;
+    };
+    if (tl.cs > 0) {
+      // one launch per THIN_CL_MAX factors, no set-up launch, no workspace
+      const int count = (int)tl.idx.size();
+      for (int first = 0; first < count; first += THIN_CL_MAX) {
+        static thread_local ThinClusterParams cp;
+        std::memset(&cp, 0, sizeof(cp));
+        cp.count = std::min(THIN_CL_MAX, count - first);
+        cp.conditioned = cond;
+        cp.nesterov = hp->nesterov;
+        cp.ns_steps = hp->ns_steps;
+        cp.mu = hp->mu;
+        cp.lr = hp->lr;
+        cp.decay = decay;
+        cp.eps = hp->cond_eps;
+        for (int k = 1; k <= hp->ns_steps; ++k) {
+          const Coef q = coef_of(hp, k);
+          cp.coef[k - 1][0] = q.a;
+          cp.coef[k - 1][1] = q.b;
+          cp.coef[k - 1][2] = q.c;
+        }
+        cp.status = status;
+        size_t smem = 0;
+        for (int q = 0; q < cp.count; ++q) {
+          const int i = tl.idx[first + q];
+          cp.mats[q] = thin_desc(i);
+          smem = std::max(smem, thin_cluster_smem(tl.pad, tl.combo, tl.cs, L.mats[i].n, L.mats[i].tall,
+                                                  hp->nesterov != 0));
+        }
+        DM_CUDA(launch_thin_cluster(cp, tl.pad, tl.combo, tl.cs, smem, s));
+      }
+      continue;
+    }
     ThinMat* mats_dev = reinterpret_cast<ThinMat*>(ws + tl.off_mats);
     int* starts_dev = reinterpret_cast<int*>(ws + tl.off_starts);
     double* fsc = reinterpret_cast<double*>(ws + tl.off_fsc);
@@ -478,24 +600,7 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
       sp.unit_f_dst = reinterpret_cast<int*>(ws + tl.off_unit_f);
       sp.fsc = fsc;
       for (int q = 0; q <= sp.count; ++q) sp.starts[q] = tl.starts[first + q];
-      for (int q = 0; q < sp.count; ++q) {
-        const dm_matrix_t& um = mats[tl.idx[first + q]];
-        ThinMat& t = sp.mats[q];
-        t.G = um.grad;
-        t.M = um.momentum;
-        t.W = um.weight;
-        t.upd = um.update_out;
-        t.e_row = cond ? um.row_energy : nullptr;
-        t.e_col = cond ? um.col_energy : nullptr;
-        t.rows = (int32_t)um.rows;
-        t.cols = (int32_t)um.cols;
-        t.gdt = (uint8_t)um.grad_dtype;
-        t.mdt = (uint8_t)um.momentum_dtype;
-        t.wdt = (uint8_t)um.weight_dtype;
-        t.kappa = kappa_of(hp, um.rows, um.cols);
-        auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
-        t.vec = (uint8_t)(al16(um.grad) && al16(um.momentum) && al16(um.weight) && al16(um.update_out));
-      }
+      for (int q = 0; q < sp.count; ++q) sp.mats[q] = thin_desc(tl.idx[first + q]);
       DM_CUDA(launch_thin_setup(sp, s));
     }
     ThinParams tp;
@@ -525,16 +630,8 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
     tp.T = reinterpret_cast<double*>(ws + tl.off_T);
     tp.fsc = fsc;
     tp.counters = reinterpret_cast<int*>(ws + THIN_CTR_OFFSET) + 2 * gi;
-    // r = 2 on the staged layout whose momentum (and Nesterov gradient) fits
-    // one CTA's shared memory: the single-pass kernel
-    int64_t max_n = 0;
-    for (int i : tl.idx) max_n = std::max<int64_t>(max_n, L.mats[i].n);
-    const size_t fused_smem = thin_fused_smem(tl.pad, max_n, hp->nesterov != 0);
-    const bool fused = tl.combo >= 0 && tl.pad == 2 &&
-                       fused_smem <= THIN_FUSED_MAX_SMEM &&
-                       !(hp->debug_flags & DM_DBG_THIN_STAGED);
-    if (fused)
-      DM_CUDA(launch_thin_fused(tp, fused_smem, s));
+    if (tl.fused)
+      DM_CUDA(launch_thin_fused(tp, tl.fused_smem, s));
     else if (tl.combo >= 0)
       DM_CUDA(launch_thin_bulk(tp, tl.combo, sm_count(dev), s));
     else
@@ -781,6 +878,29 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
   return DM_OK;
 }
 
+// Kernel launches run_step enqueues for this layout (the header memset is
+// not a kernel).
+int64_t count_launches(const Layout& L, const dm_hparams_t* hp, int cond) {
+  auto chunks = [](int64_t count, int64_t per) { return (count + per - 1) / per; };
+  int64_t k = 0;
+  for (const ThinLaunch& tl : L.thin) {
+    const int64_t count = (int64_t)tl.idx.size();
+    if (tl.cs > 0)
+      k += chunks(count, THIN_CL_MAX);
+    else
+      k += chunks(count, THIN_MAX) + (tl.fused ? 1 : 3);
+  }
+  k += 2 * (int64_t)((L.canary.size() + CANARY_MAX - 1) / CANARY_MAX);
+  int64_t big = 0;
+  for (const MatPlan& p : L.mats) big += p.thin ? 0 : 1;
+  if (big == 0) return k;
+  if (cond) k += chunks(big, K0_MAX);
+  k += chunks(big, K1_MAX) + chunks(big, K1B_MAX);
+  k += (int64_t)hp->ns_steps * 3 * chunks(big, L.tc ? TC_MAX : SIMT_MAX);
+  if (cond) k += 2 * chunks(big, K3_MAX);
+  return k;
+}
+
 }  // namespace
 }  // namespace dm
 
@@ -812,6 +932,19 @@ dm_status_t dm_workspace_size(const dm_matrix_t* mats, int n, const dm_hparams_t
     const dm_status_t st = dm::validate(mats, n, hp, conditioned);
     if (st != DM_OK) return st;
     *bytes = dm::make_layout(mats, n, hp, conditioned).bytes;
+    return DM_OK;
+  } catch (...) {
+    return DM_ERR_INVALID_ARG;
+  }
+}
+
+dm_status_t dm_step_launches(const dm_matrix_t* mats, int n, const dm_hparams_t* hp,
+                             int conditioned, int64_t* launches) {
+  if (!launches) return DM_ERR_INVALID_ARG;
+  try {
+    const dm_status_t st = dm::validate(mats, n, hp, conditioned);
+    if (st != DM_OK) return st;
+    *launches = dm::count_launches(dm::make_layout(mats, n, hp, conditioned), hp, conditioned);
     return DM_OK;
   } catch (...) {
     return DM_ERR_INVALID_ARG;
@@ -856,6 +989,7 @@ const char* dm_status_string(int32_t status) {
     case DM_ERR_CUDA: return "CUDA call failed";
     case DM_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case DM_ERR_NONFINITE: return "non-finite Frobenius norm (update set to zero)";
+    case DM_ERR_CANARY: return "workspace canary overwritten";
     default: return "unknown status";
   }
 }

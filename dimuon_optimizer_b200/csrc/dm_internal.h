@@ -43,7 +43,7 @@ enum {
 };
 
 // Device status codes (mirror dm_status_t).
-enum { ST_OK = 0, ST_TIMEOUT = 5, ST_NONFINITE = 6 };
+enum { ST_OK = 0, ST_TIMEOUT = 5, ST_NONFINITE = 6, ST_CANARY = 7 };
 // int32 index, after the status word, of the step's abort word (set with
 // ST_TIMEOUT; both live in the workspace header that each step clears).
 constexpr int STATUS_ABORT_WORD = 1;
@@ -272,6 +272,23 @@ size_t thin_fused_smem(int pad, int64_t n, bool nesterov);
 cudaError_t launch_thin_fused(const ThinParams& p, size_t smem, cudaStream_t s);
 int thin_slab(int pad);
 
+// ----------------------------- canaries -----------------------------------
+// Checked-workspace mode: 256-byte canaries (64 words) at the listed 256-byte
+// blocks of the workspace.  mode 0 (step start): check them if the arm word
+// holds CANARY_ARMED, then fill; mode 1 (step end): check, then arm.
+constexpr uint32_t CANARY_FILL = 0xA5C3A5C3u;
+constexpr uint32_t CANARY_ARMED = 0x43414E59u;
+constexpr int CANARY_ARM_WORD = 255;      // int32 index in the 1 KB header
+constexpr int CANARY_MAX = 7000;          // canaries per launch
+struct CanaryParams {
+  int count;
+  int mode;
+  int* status;                // the workspace base (status word first)
+  uint32_t blk[CANARY_MAX];   // canary offsets / 256
+};
+static_assert(sizeof(CanaryParams) <= 32764, "kernel parameter space");
+cudaError_t launch_canary(const CanaryParams& p, cudaStream_t s);
+
 // ------------------------------ launches ----------------------------------
 cudaError_t launch_k0(const K0Params& p, cudaStream_t s);
 cudaError_t launch_k1(const K1Params& p, int total_tiles, cudaStream_t s);
@@ -291,5 +308,26 @@ cudaError_t launch_thin_iterate(const ThinParams& p, cudaStream_t s);
 // shared-memory staged thin path (k_thin_bulk.cu)
 int thin_bulk_combo(int gdt, int mdt, int wdt);
 cudaError_t launch_thin_bulk(ThinParams& p, int combo, int nsm, cudaStream_t s);
+// single-launch cluster path (k_thin_cluster.cu): one cluster of cs CTAs per
+// factor, the factor held in the cluster's shared memory; r = pad in {2, 4, 8},
+// long side a multiple of 8 cs, staged storage combinations and alignment
+constexpr int THIN_CL_MAX = 448;      // factors per launch (kernel parameter space)
+constexpr int THIN_CL_MAX_CS = 8;     // portable cluster size
+constexpr size_t THIN_CL_MAX_SMEM = 60 * 1024;
+struct ThinClusterParams {
+  int count;              // factors (clusters) in this launch
+  int conditioned;
+  int nesterov;
+  int ns_steps;
+  float mu, lr, decay, eps;
+  float coef[64][3];      // (a_k, b_k, c_k) of Newton-Schulz iteration k
+  int* status;
+  ThinMat mats[THIN_CL_MAX];
+};
+static_assert(sizeof(ThinClusterParams) <= 32764, "kernel parameter space");
+// Dynamic shared memory of one CTA (0 if this (pad, combo, cs, n) has no kernel).
+size_t thin_cluster_smem(int pad, int combo, int cs, int64_t n, bool tall, bool nest);
+cudaError_t launch_thin_cluster(const ThinClusterParams& p, int pad, int combo, int cs, size_t smem,
+                                cudaStream_t s);
 
 }  // namespace dm

@@ -118,6 +118,126 @@ __device__ __forceinline__ Geo geometry(const ThinMat& mt, int conditioned) {
   return q;
 }
 
+// ---------------------------------------------------------------------------
+// The r x r Newton-Schulz iteration of one factor by one warp (RP <= 8; no
+// block-wide barrier).  The iterate is X_k = P_k X_0 with P_k an r x r
+// polynomial in A_0 = X_0 X_0^T ("From PCG to Muon", section 6 "Muon's Gram
+// Matrix"): P_k = Q_k P_{k-1}, A_k = Q_k A_{k-1} Q_k with
+// Q_k = a_k I + b_k A_{k-1} + c_k A_{k-1}^2 (sitech.ge Muon post, "Instead of
+// SVD - Newton-Schulz"), A normalised by ||X_0||_F^2 = tr A_0.
+// ---------------------------------------------------------------------------
+template <int RP>
+struct WarpIterSmem {
+  double G[RP][RP + 1], H[RP][RP + 1], P[RP][RP + 1], A[RP][RP + 1], Q[RP][RP + 1], S[RP][RP + 1];
+  double R[RP];
+};
+
+template <int RP>
+__device__ __forceinline__ void mm_warp(double (*C)[RP + 1], double (*A)[RP + 1], double (*B)[RP + 1]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (RP == 8) {
+    const int g = lane >> 2, t = lane & 3;
+    double d0 = 0.0, d1 = 0.0;
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) dmma(d0, d1, A[g][kb * 4 + t], B[kb * 4 + t][g]);
+    __syncwarp();  // every lane has read A and B (C may alias neither, but keep order)
+    C[g][2 * t] = d0;
+    C[g][2 * t + 1] = d1;
+  } else {
+    static_assert(RP * RP <= 32, "one lane per element");
+    if (lane < RP * RP) {
+      const int i = lane / RP, j = lane % RP;
+      double s = 0.0;
+#pragma unroll
+      for (int k = 0; k < RP; ++k) s = fma(A[i][k], B[k][j], s);
+      C[i][j] = s;
+    }
+  }
+  __syncwarp();
+}
+
+// What the iteration needs besides the two Gram sums.
+struct IterIn {
+  double sc, sr;          // sums of the previous long- / short-side energies
+  bool cond;              // Dimuon energies given
+  int r;                  // short side (<= RP)
+  const float* e_r;       // previous short-side energies (read before they are replaced)
+  float eps;              // conditioning damping
+  const float (*coef)[3]; // (a_k, b_k, c_k) per iteration
+  int ns_steps;
+  float kappa;            // update scale
+  int* status;            // device status word (non-finite norm)
+};
+
+// On entry s.G and s.H hold S_1 = sum_j C_j^2 b_j b_j^T and S_2 = sum_j C_j^4
+// b_j b_j^T.  On return s.R holds R, s.P holds P_5, and the result is the
+// update factor kappa / ||X_0|| (times ||X_5|| / ||R X_5 C|| when
+// conditioning is on; "Dimuon: LoRA 에 맞춰 다시 짠 Muon", Problem 4 (c)), 0
+// for a degenerate norm; *on_out tells whether conditioning was on.
+template <int RP>
+__device__ double iterate_gram_warp(const IterIn& in, WarpIterSmem<RP>& s, bool* on_out) {
+  const int lane = threadIdx.x & 31;
+  const int r = in.r;
+  const bool on = in.cond && in.sr > 0.0 && in.sc > 0.0;
+  if (lane < RP) {
+    double rv = lane < r ? 1.0 : 0.0;
+    if (on && lane < r) rv = 1.0 / sqrt(sqrt((double)in.e_r[lane] * ((double)r / in.sr) + (double)in.eps));
+    s.R[lane] = rv;
+  }
+  __syncwarp();
+  double tr = 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP, j = idx % RP;
+    const double rr = s.R[i] * s.R[j];
+    s.G[i][j] *= rr;
+    s.H[i][j] *= rr;
+    if (i == j) tr += s.G[i][j];
+  }
+  const double s2 = warp_sum_d(tr);
+  const bool finite = isfinite(s2);
+  const bool valid = finite && s2 >= NORM2_FLOOR;
+  const double inv_s2 = valid ? 1.0 / s2 : 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP, j = idx % RP;
+    s.A[i][j] = valid ? s.G[i][j] * inv_s2 : 0.0;
+    s.P[i][j] = i == j ? 1.0 : 0.0;
+  }
+  __syncwarp();
+  for (int it = 0; it < in.ns_steps; ++it) {
+    const double a = in.coef[it][0], b = in.coef[it][1], c = in.coef[it][2];
+    mm_warp<RP>(s.Q, s.A, s.A);
+    for (int idx = lane; idx < RP * RP; idx += 32) {
+      const int i = idx / RP, j = idx % RP;
+      s.Q[i][j] = c * s.Q[i][j] + b * s.A[i][j] + (i == j ? a : 0.0);
+    }
+    __syncwarp();
+    mm_warp<RP>(s.S, s.Q, s.P);
+    for (int idx = lane; idx < RP * RP; idx += 32) s.P[idx / RP][idx % RP] = s.S[idx / RP][idx % RP];
+    __syncwarp();
+    mm_warp<RP>(s.S, s.Q, s.A);
+    mm_warp<RP>(s.A, s.S, s.Q);
+  }
+  // ||X_5||^2 s^2 = tr(P A_0 P^T); ||R X_5 C||^2 s^2 = sum_i R_i^2 (P H P^T)_ii
+  mm_warp<RP>(s.S, s.P, s.G);
+  double nx = 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) nx += s.S[idx / RP][idx % RP] * s.P[idx / RP][idx % RP];
+  nx = warp_sum_d(nx);
+  mm_warp<RP>(s.Q, s.P, s.H);
+  double ny = 0.0;
+  for (int idx = lane; idx < RP * RP; idx += 32) {
+    const int i = idx / RP;
+    ny += s.R[i] * s.R[i] * s.Q[i][idx % RP] * s.P[i][idx % RP];
+  }
+  ny = warp_sum_d(ny);
+  double factor = 0.0;
+  if (valid) {
+    factor = (double)in.kappa / sqrt(s2);
+    if (on) factor = ny > 0.0 ? factor * sqrt(nx / ny) : 0.0;
+  }
+  if (!finite && lane == 0) raise_status(in.status, ST_NONFINITE);
+  *on_out = on;
+  return factor;
+}
 
 }  // namespace thin
 }  // namespace dm

@@ -470,106 +470,23 @@ __device__ __forceinline__ void mm(double (*C)[TCfg<RP>::SLD], double (*A)[TCfg<
   __syncthreads();
 }
 
-// ---- one warp per factor for RP <= 8 (no block-wide barriers) -------------
-template <int RP>
-struct WarpIterSmem {
-  double G[RP][RP + 1], H[RP][RP + 1], P[RP][RP + 1], A[RP][RP + 1], Q[RP][RP + 1], S[RP][RP + 1];
-  double R[RP];
-};
-
-template <int RP>
-__device__ __forceinline__ void mm_warp(double (*C)[RP + 1], double (*A)[RP + 1], double (*B)[RP + 1]) {
-  const int lane = threadIdx.x & 31;
-  if constexpr (RP == 8) {
-    const int g = lane >> 2, t = lane & 3;
-    double d0 = 0.0, d1 = 0.0;
-#pragma unroll
-    for (int kb = 0; kb < 2; ++kb) dmma(d0, d1, A[g][kb * 4 + t], B[kb * 4 + t][g]);
-    __syncwarp();  // every lane has read A and B (C may alias neither, but keep order)
-    C[g][2 * t] = d0;
-    C[g][2 * t + 1] = d1;
-  } else {
-    if (lane < RP * RP) {
-      const int i = lane / RP, j = lane % RP;
-      double s = 0.0;
-#pragma unroll
-      for (int k = 0; k < RP; ++k) s = fma(A[i][k], B[k][j], s);
-      C[i][j] = s;
-    }
-  }
-  __syncwarp();
-}
-
-// The r x r iteration of factor f by one warp.  On entry s.G and s.H hold
-// S_1 and S_2; the previous short-side energies are read here for R (before
-// the caller replaces them).  On return s.R holds R, s.P holds P_5 and the
-// result is the update factor kappa / ||X_0|| (times ||X_5|| / ||R X_5 C||
-// when conditioning is on), 0 for a degenerate norm; *on_out tells whether
-// conditioning was on.
+// The r x r iteration of factor f by one warp (iterate_gram_warp in
+// dm_thin.cuh) with this launch's parameters.
 template <int RP>
 __device__ double iterate_factor_warp(const ThinParams& p, int f, const ThinMat& mt, const Geo& q,
                                       WarpIterSmem<RP>& s, bool* on_out) {
-  const int lane = threadIdx.x & 31;
-  const int r = q.r;
-  const double sc = p.fsc[4 * f], sr = p.fsc[4 * f + 1];
-  const bool on = q.cond && sr > 0.0 && sc > 0.0;
-  if (lane < RP) {
-    double rv = lane < r ? 1.0 : 0.0;
-    if (on && lane < r) rv = 1.0 / sqrt(sqrt((double)q.e_r[lane] * ((double)r / sr) + (double)p.eps));
-    s.R[lane] = rv;
-  }
-  __syncwarp();
-  double tr = 0.0;
-  for (int idx = lane; idx < RP * RP; idx += 32) {
-    const int i = idx / RP, j = idx % RP;
-    const double rr = s.R[i] * s.R[j];
-    s.G[i][j] *= rr;
-    s.H[i][j] *= rr;
-    if (i == j) tr += s.G[i][j];
-  }
-  const double s2 = warp_sum_d(tr);
-  const bool finite = isfinite(s2);
-  const bool valid = finite && s2 >= NORM2_FLOOR;
-  const double inv_s2 = valid ? 1.0 / s2 : 0.0;
-  for (int idx = lane; idx < RP * RP; idx += 32) {
-    const int i = idx / RP, j = idx % RP;
-    s.A[i][j] = valid ? s.G[i][j] * inv_s2 : 0.0;
-    s.P[i][j] = i == j ? 1.0 : 0.0;
-  }
-  __syncwarp();
-  for (int it = 0; it < p.ns_steps; ++it) {
-    const double a = p.coef[it][0], b = p.coef[it][1], c = p.coef[it][2];
-    mm_warp<RP>(s.Q, s.A, s.A);
-    for (int idx = lane; idx < RP * RP; idx += 32) {
-      const int i = idx / RP, j = idx % RP;
-      s.Q[i][j] = c * s.Q[i][j] + b * s.A[i][j] + (i == j ? a : 0.0);
-    }
-    __syncwarp();
-    mm_warp<RP>(s.S, s.Q, s.P);
-    for (int idx = lane; idx < RP * RP; idx += 32) s.P[idx / RP][idx % RP] = s.S[idx / RP][idx % RP];
-    __syncwarp();
-    mm_warp<RP>(s.S, s.Q, s.A);
-    mm_warp<RP>(s.A, s.S, s.Q);
-  }
-  mm_warp<RP>(s.S, s.P, s.G);
-  double nx = 0.0;
-  for (int idx = lane; idx < RP * RP; idx += 32) nx += s.S[idx / RP][idx % RP] * s.P[idx / RP][idx % RP];
-  nx = warp_sum_d(nx);
-  mm_warp<RP>(s.Q, s.P, s.H);
-  double ny = 0.0;
-  for (int idx = lane; idx < RP * RP; idx += 32) {
-    const int i = idx / RP;
-    ny += s.R[i] * s.R[i] * s.Q[i][idx % RP] * s.P[i][idx % RP];
-  }
-  ny = warp_sum_d(ny);
-  double factor = 0.0;
-  if (valid) {
-    factor = (double)mt.kappa / sqrt(s2);
-    if (on) factor = ny > 0.0 ? factor * sqrt(nx / ny) : 0.0;
-  }
-  if (!finite && lane == 0) raise_status(p.status, ST_NONFINITE);
-  *on_out = on;
-  return factor;
+  IterIn in;
+  in.sc = p.fsc[4 * f];
+  in.sr = p.fsc[4 * f + 1];
+  in.cond = q.cond;
+  in.r = q.r;
+  in.e_r = q.e_r;
+  in.eps = p.eps;
+  in.coef = p.coef;
+  in.ns_steps = p.ns_steps;
+  in.kappa = mt.kappa;
+  in.status = p.status;
+  return iterate_gram_warp<RP>(in, s, on_out);
 }
 
 template <int RP>

@@ -76,10 +76,13 @@ typedef enum {
   DM_ERR_WORKSPACE = 3,       /* workspace null, misaligned or too small      */
   DM_ERR_CUDA = 4,            /* a CUDA runtime / driver call failed          */
   DM_ERR_DEVICE_TIMEOUT = 5,  /* device status: a bounded wait gave up        */
-  DM_ERR_NONFINITE = 6        /* device status: non-finite ||X_0||_F; that
+  DM_ERR_NONFINITE = 6,       /* device status: non-finite ||X_0||_F; that
                                  matrix got O = 0 (its W was only decayed).
                                  A norm below 1e-15 also gives O = 0, without
                                  a status (nothing to normalise).             */
+  DM_ERR_CANARY = 7           /* device status (DM_DBG_CANARY only): a canary
+                                 word between workspace regions was changed,
+                                 during the step or since the previous one    */
 } dm_status_t;
 
 typedef enum { DM_BF16 = 0, DM_FP32 = 1 } dm_dtype_t;
@@ -170,9 +173,22 @@ typedef struct {
                                      (256 x 256 tiles) only                */
 #define DM_DBG_THIN_REGS 0x10u    /* thin factors always take the register
                                      path (no shared-memory staging)       */
-#define DM_DBG_THIN_STAGED 0x20u  /* thin factors of r = 2 take the
-                                     two-pass staged kernels instead of the
-                                     single-pass one (one CTA per factor)  */
+#define DM_DBG_THIN_STAGED 0x20u  /* thin factors take the two-pass staged
+                                     kernels instead of the single-launch
+                                     ones (one cluster per factor, or for
+                                     r = 2 one CTA per factor)             */
+#define DM_DBG_CANARY 0x40u      /* checked workspace: 256 canary bytes
+                                     after the header and after every
+                                     workspace region (dm_workspace_size
+                                     grows accordingly; pass the flag to
+                                     both calls).  The step fills them at
+                                     its start, after checking those a
+                                     previous canary step left (the first
+                                     canary after the header sits at byte
+                                     1024), and checks them all at its end;
+                                     a changed byte sets DM_ERR_CANARY.
+                                     Costs two small launches; the
+                                     arithmetic is unchanged.              */
 #define DM_DBG_FORCE_TIMEOUT 0x8u /* failure-detection hook: each
                                      tensor-core product launch makes one
                                      bounded wait run out (20 ms, on a
@@ -200,6 +216,13 @@ void dm_default_hparams(dm_hparams_t* hp);
 dm_status_t dm_workspace_size(const dm_matrix_t* mats, int n,
                               const dm_hparams_t* hp, int conditioned,
                               size_t* bytes);
+
+/* Number of kernel launches one step over `mats[0..n)` enqueues with these
+ * hyper-parameters (conditioned = 0: dm_muon_step, 1: dm_dimuon_step), for
+ * sizing CUDA graphs or checking a profile.  Host-only; validates like
+ * dm_workspace_size. */
+dm_status_t dm_step_launches(const dm_matrix_t* mats, int n, const dm_hparams_t* hp,
+                             int conditioned, int64_t* launches);
 
 /* One Muon step over the group (steps 1, 3, 5, 6 above; row_energy and
  * col_energy are ignored).  Asynchronous on `stream`. */

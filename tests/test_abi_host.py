@@ -111,6 +111,30 @@ def test_every_scale_mode_is_accepted(mode):
     assert dm.dm_workspace_size([m], hp, 0) > 0
 
 
+def test_launch_counts():
+    """Kernel launches per step, from the planner (host-only)."""
+    hp = dm.dm_default_hparams()
+    big = [fake_matrix(4096, 4096)] * 8 + [fake_matrix(4096, 14336)] * 8
+    # K1, K1b, 5 x 3 products
+    assert dm.dm_step_launches(big, hp, 0) == 2 + 15
+    # + K0, and K3a + K3
+    assert dm.dm_step_launches(big, hp, 1) == 1 + 2 + 15 + 2
+    # 448 rank-8 LoRA factors: one launch of the cluster kernel
+    lora = [fake_matrix(8, 4096), fake_matrix(4096, 8)] * 224
+    for m in lora:
+        m.momentum_dtype = dm.DM_FP32
+    assert dm.dm_step_launches(lora, hp, 1) == 1
+    # the two-pass staged kernels: set-up, Gram, iteration, apply
+    staged = dm.dm_default_hparams(debug_flags=dm.DM_DBG_THIN_STAGED)
+    assert dm.dm_step_launches(lora, staged, 1) == 4
+    # rank 32 has no cluster kernel
+    lora32 = [fake_matrix(32, 4096), fake_matrix(4096, 32)] * 224
+    for m in lora32:
+        m.momentum_dtype = dm.DM_FP32
+    assert dm.dm_step_launches(lora32, hp, 1) == 4
+    assert dm.dm_step_launches([], hp, 0) == 0
+
+
 def test_coefficient_schedule_is_accepted():
     """A finite per-iteration schedule passes validation (the call then stops
     at the missing workspace); its length sets ns_steps; the default has none."""
@@ -155,3 +179,14 @@ def test_header_constants_match_binding():
     # debug flags are distinct bits
     bits = [v for k, v in consts.items() if k.startswith("DM_DBG_")]
     assert all(b & (b - 1) == 0 for b in bits) and len(set(bits)) == len(bits)
+
+
+def test_checked_mode_sizes():
+    """The checked-workspace mode adds a 256-byte canary after the header and
+    after every region, and two launches (fill, check)."""
+    hp = dm.dm_default_hparams()
+    hpc = dm.dm_default_hparams(debug_flags=dm.DM_DBG_CANARY)
+    mats = [fake_matrix(300, 500), fake_matrix(8, 4096)]
+    assert dm.dm_workspace_size(mats, hpc, 1) >= dm.dm_workspace_size(mats, hp, 1) + 256 * 10
+    assert dm.dm_step_launches(mats, hpc, 1) == dm.dm_step_launches(mats, hp, 1) + 2
+    assert dm.dm_status_string(dm.DM_ERR_CANARY) == "workspace canary overwritten"
