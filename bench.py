@@ -206,12 +206,15 @@ def l2_flushed(spec):
     return resident_bytes(spec) < 3 * L2_BYTES
 
 
-def config_of(spec, world):
+def config_of(spec, world, precision="bf16"):
     """The workload description both arms print."""
-    return {"workload": spec["desc"], "matrices": len(spec["shapes"]),
-            "parallelism": f"replica per GPU x{world}",
-            "l2": ("512 MB written between timed steps (per-step CUDA events)" if l2_flushed(spec)
-                   else "inputs larger than L2 (no flush)")}
+    cfg = {"workload": spec["desc"], "matrices": len(spec["shapes"]),
+           "parallelism": f"replica per GPU x{world}",
+           "l2": ("512 MB written between timed steps (per-step CUDA events)" if l2_flushed(spec)
+                  else "inputs larger than L2 (no flush)")}
+    if precision == "fp32":
+        cfg["products"] = "fp32 (DM_PREC_FP32)"
+    return cfg
 
 
 def interleaved_order(shapes):
@@ -303,7 +306,7 @@ def run_reference(args, spec, rank, world):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(spec, world),
+            "config": config_of(spec, world, args.precision),
             "cpu_baseline": {"value": value, "unit": "matrices/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "matrices/s", "h2d_bytes_per_step": 0,
@@ -422,6 +425,8 @@ def main():
     ap.add_argument("--debug-flags", type=lambda v: int(v, 0), default=0,
                     help="library debug_flags (test hooks such as DM_DBG_TC_SINGLE; none skips "
                          "work)")
+    ap.add_argument("--precision", default="bf16", choices=["bf16", "fp32"],
+                    help="Newton-Schulz products on bf16 tensor cores (default) or fp32 SIMT")
     ap.add_argument("--sharded", action="store_true",
                     help="one workload sharded over the ranks (strong scaling) instead of replicas")
     args = ap.parse_args()
@@ -486,10 +491,11 @@ def main():
         EC.append(torch.zeros(c, device=dev, dtype=torch.float32) if spec["cond"] else None)
     G_flat.copy_(G_host_flat)
     mats = [dm.dm_matrix(W[i], G[i], M[i], ER[i], EC[i]) for i in range(len(shapes))]
+    prec = dm.DM_PREC_FP32 if args.precision == "fp32" else dm.DM_PREC_BF16_TC
     hp = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"],
                                scale_mode=dm.DM_SCALE_MOONSHOT if spec["moonshot"]
                                else dm.DM_SCALE_NONE, nesterov=spec.get("nesterov", 0),
-                               debug_flags=args.debug_flags)
+                               debug_flags=args.debug_flags, precision=prec)
     step_fn = dm.dm_dimuon_step if spec["cond"] else dm.dm_muon_step
     ws = torch.empty(dm.dm_workspace_size(mats, hp, int(spec["cond"])), dtype=torch.uint8,
                      device=dev)
@@ -556,7 +562,7 @@ def main():
     reps = max(2, min(args.steps, 5))
     hp1 = dm.dm_default_hparams(lr=spec["lr"], weight_decay=spec["wd"], ns_steps=1,
                                 scale_mode=hp.scale_mode, nesterov=hp.nesterov,
-                                debug_flags=args.debug_flags)
+                                debug_flags=args.debug_flags, precision=prec)
     g1 = capture(hp1)
     g1.replay()
     t5 = timed(graph, reps) / reps
@@ -565,9 +571,23 @@ def main():
     per_iter_flops = ns_flops([s for s in shapes if min(s) > dm.DM_THIN_MAX])
     peaks, peak_kind = load_peaks()
     tc_launches = 3 * 4
-    if per_iter_flops > 0 and t5 > t1:
+    if per_iter_flops > 0 and t5 > t1 and args.precision == "fp32":
+        # fp32 SIMT products: bound by the FMA pipes, 148 SMs x 128 fp32 lanes x 2
+        # flops per clock at the sampled SM clock (74.5 TF/s at 1965 MHz)
         achieved = 4 * per_iter_flops / (t5 - t1) / 1e12
-        peak = peaks.get("bf16_tflops_sustained", 1400.0)
+        mhz = clocks.get("sm_mhz") or 1965.0
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None, "kernel": "simt_ns_product",
+                    "avg_launch_ms": (t5 - t1) / tc_launches * 1e3,
+                    "peak_kind": f"derived fp32 FMA peak at the sampled {mhz:.0f} MHz"}
+    elif per_iter_flops > 0 and t5 > t1:
+        achieved = 4 * per_iter_flops / (t5 - t1) / 1e12
+        # the sustained figure (a seconds-long loop under the power cap) when
+        # the timed region ran power-capped, else the burst figure
+        capped = "sw_power_cap" in (clocks.get("reasons") or [])
+        peak = (peaks.get("bf16_tflops_sustained", 1400.0) if capped
+                else peaks.get("bf16_tflops", 1590.0))
         traffic = None
         if args.workload in TRAFFIC_CAPTURED and kernel_build_hash() == TRAFFIC_BUILD:
             traffic = TRAFFIC_CAPTURED[args.workload]
@@ -576,15 +596,19 @@ def main():
                     "kernel": "tc_ns_product_pair" if args.workload.startswith("large_batch")
                     else "tc_ns_product(_pair)",
                     "avg_launch_ms": (t5 - t1) / tc_launches * 1e3,
-                    "peak_kind": f"{peak_kind} bf16 dense, sustained"}
+                    "peak_kind": f"{peak_kind} bf16 dense, "
+                                 f"{'sustained (run power-capped)' if capped else 'burst'}"}
     else:
         gbs = step_bytes(spec) / (ms_step / 1e3) / 1e9
         peak = peaks.get("hbm_gbs", 6650.0)
+        per_step = dm.dm_step_launches(mats, hp, int(spec["cond"]))
+        label = ("thin_cluster (the whole step in one launch per 448 factors)"
+                 if per_step <= -(-len(shapes) // 448) else
+                 "thin path (thin_setup, thin_gram, thin_iterate, thin_apply; or thin_fused)")
         roofline = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                     "frac": gbs / peak, "traffic": None,
-                    "kernel": "thin path (thin_setup, then thin_gram + thin_iterate + thin_apply, "
-                              "or thin_fused for r = 2), algorithmic bytes of the whole step over "
-                              "the step time",
+                    "kernel": label + ": algorithmic bytes of the whole step over the step time",
+                    "launches_per_step": per_step,
                     "peak_kind": f"{peak_kind} HBM copy"}
 
     # end to end through the public API: every step's gradients copied in from
@@ -648,9 +672,10 @@ def main():
                "kind": "oracle", "sample": sample}
     line = {"metric": METRIC, "value": value, "unit": "matrices/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if args.precision == "fp32" else "bf16",
             "data": "synthetic (seeded N(0,1) gradients, N(0,0.02^2) weights)",
-            "config": config_of(spec, world), "cuda_graph": True,
+            "config": config_of(spec, world, args.precision), "cuda_graph": True,
             "ns_tflops_step": ns_flops(shapes) * hp.ns_steps / (ms_step / 1e3) / 1e12,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": launches * args.steps}

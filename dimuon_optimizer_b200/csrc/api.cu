@@ -70,7 +70,10 @@ int thin_pad(int r) { return r <= 4 ? r : r <= 8 ? 8 : r <= 16 ? 16 : 32; }
 
 // Shared memory per CTA the cluster kernel's slices may take: with the
 // kernel's static arrays four to five CTAs stay resident per SM.
-constexpr size_t THIN_CL_BUDGET = 40 * 1024;
+#ifndef DM_THIN_CL_BUDGET_KB
+#define DM_THIN_CL_BUDGET_KB 40
+#endif
+constexpr size_t THIN_CL_BUDGET = DM_THIN_CL_BUDGET_KB * 1024;
 
 struct Layout {
   std::vector<MatPlan> mats;
@@ -216,9 +219,13 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
     tl.off_T = take(count * tl.pad * tl.pad * sizeof(double), 256);
     tl.off_fsc = take(count * 4 * sizeof(double), 256);
     // single-launch cluster kernel: the smallest cluster whose per-CTA slice
-    // of every factor of the group fits the budget
-    if (tl.combo >= 0 && (tl.pad == 2 || tl.pad == 4 || tl.pad == 8) &&
-        !(hp->debug_flags & (DM_DBG_THIN_STAGED | DM_DBG_THIN_REGS))) {
+    // of every factor of the group fits the budget.  By default for r <= 4;
+    // at r = 8 the two-pass staged kernels measured faster on the LoRA batch
+    // (448 factors of width 4096: 0.109 against 0.150 ms per step), so the
+    // cluster kernel takes r = 8 only under DM_DBG_THIN_CLUSTER.
+    const bool cl_pad = tl.pad == 2 || tl.pad == 4 ||
+                        (tl.pad == 8 && (hp->debug_flags & DM_DBG_THIN_CLUSTER));
+    if (tl.combo >= 0 && cl_pad && !(hp->debug_flags & (DM_DBG_THIN_STAGED | DM_DBG_THIN_REGS))) {
       for (int cs = 1; cs <= THIN_CL_MAX_CS && !tl.cs; cs *= 2) {
         bool ok = true;
         for (int i : tl.idx) {

@@ -313,7 +313,7 @@ cudaError_t launch_thin_bulk(ThinParams& p, int combo, int nsm, cudaStream_t s);
 // long side a multiple of 8 cs, staged storage combinations and alignment
 constexpr int THIN_CL_MAX = 448;      // factors per launch (kernel parameter space)
 constexpr int THIN_CL_MAX_CS = 8;     // portable cluster size
-constexpr size_t THIN_CL_MAX_SMEM = 60 * 1024;
+constexpr size_t THIN_CL_MAX_SMEM = 200 * 1024;
 struct ThinClusterParams {
   int count;              // factors (clusters) in this launch
   int conditioned;

@@ -39,7 +39,10 @@ namespace {
 using namespace thin;
 using namespace sm100;
 
-constexpr int CT = 128;  // threads per CTA
+#ifndef DM_CL_THREADS
+#define DM_CL_THREADS 256
+#endif
+constexpr int CT = DM_CL_THREADS;  // threads per CTA
 constexpr int CW = CT / 32;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(CT) thin_cluster(const __grid_constant__ ThinC
   __shared__ double red_d[32];
   __shared__ float erp[RP];  // previous short-side energies, this CTA's copy
   __shared__ __align__(8) uint64_t bar_in, bar_w;
-  __shared__ int flag_sh[2];  // [0] slice in place, [1] write outputs
+  __shared__ int flag_sh[3];  // [0] slice in place, [1] write outputs, [2] zero update
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int CS = (int)cluster_size();  // CTAs per factor (1 without a cluster launch)
@@ -416,12 +419,18 @@ __global__ void __launch_bounds__(CT) thin_cluster(const __grid_constant__ ThinC
     // the new short-side energies (the previous ones were read at the start
     // by every CTA of the cluster, before the barrier)
     if (rank == 0 && !bad && q.cond && lane < RP) q.e_r[lane] = er_new;
-    if (lane == 0) flag_sh[1] = bad ? 0 : 1;
+    if (lane == 0) {
+      flag_sh[1] = bad ? 0 : 1;
+      // a degenerate norm: O = 0 exactly (W only decayed), even where the
+      // momentum is not finite
+      flag_sh[2] = factor == 0.0 ? 1 : 0;
+    }
   } else {
     cluster_arrive();
   }
   __syncthreads();
   const bool write = flag_sh[1] != 0;
+  const bool zero = flag_sh[2] != 0;
 
   // ---- 4. pass 2: O = C^2 T B, W, long-side energies ---------------------
   bool have_w = false;
@@ -459,7 +468,7 @@ __global__ void __launch_bounds__(CT) thin_cluster(const __grid_constant__ ThinC
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int j = 8 * cg + 2 * t + e;
-          const float ov = (float)o[e];
+          const float ov = zero ? 0.f : (float)o[e];
           TW* wp = Ws + wi(g, j);
           Ty<TW>::st(wp, decay * Ty<TW>::ld(wp) - lr * ov);
           if (mt.upd) mt.upd[q.tall ? (c0 + j) * RP + g : (int64_t)g * n + c0 + j] = ov;
@@ -487,7 +496,7 @@ __global__ void __launch_bounds__(CT) thin_cluster(const __grid_constant__ ThinC
           double y = 0.0;
 #pragma unroll
           for (int k = 0; k < RP; ++k) y = fma(tm[i][k], x[k], y);
-          const float ov = (float)y;
+          const float ov = zero ? 0.f : (float)y;
           TW* wp = Ws + wi(i, j);
           Ty<TW>::st(wp, decay * Ty<TW>::ld(wp) - lr * ov);
           if (mt.upd) mt.upd[q.tall ? (c0 + j) * RP + i : (int64_t)i * n + c0 + j] = ov;

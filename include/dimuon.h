@@ -177,6 +177,10 @@ typedef struct {
                                      kernels instead of the single-launch
                                      ones (one cluster per factor, or for
                                      r = 2 one CTA per factor)             */
+#define DM_DBG_THIN_CLUSTER 0x80u /* thin factors of r = 8 take the
+                                     single-launch cluster kernel as well
+                                     (by default only r <= 4 does; r = 8
+                                     takes the two-pass staged kernels)   */
 #define DM_DBG_CANARY 0x40u      /* checked workspace: 256 canary bytes
                                      after the header and after every
                                      workspace region (dm_workspace_size

@@ -119,14 +119,21 @@ def test_launch_counts():
     assert dm.dm_step_launches(big, hp, 0) == 2 + 15
     # + K0, and K3a + K3
     assert dm.dm_step_launches(big, hp, 1) == 1 + 2 + 15 + 2
-    # 448 rank-8 LoRA factors: one launch of the cluster kernel
+    # 448 rank-8 LoRA factors: the two-pass staged kernels (set-up, Gram,
+    # iteration, apply), or one launch of the cluster kernel
     lora = [fake_matrix(8, 4096), fake_matrix(4096, 8)] * 224
     for m in lora:
         m.momentum_dtype = dm.DM_FP32
-    assert dm.dm_step_launches(lora, hp, 1) == 1
-    # the two-pass staged kernels: set-up, Gram, iteration, apply
+    assert dm.dm_step_launches(lora, hp, 1) == 4
+    cl = dm.dm_default_hparams(debug_flags=dm.DM_DBG_THIN_CLUSTER)
+    assert dm.dm_step_launches(lora, cl, 1) == 1
+    # rank 2: the cluster kernel by default
+    lora2 = [fake_matrix(2, 4096), fake_matrix(4096, 2)] * 224
+    for m in lora2:
+        m.momentum_dtype = dm.DM_FP32
+    assert dm.dm_step_launches(lora2, hp, 1) == 1
     staged = dm.dm_default_hparams(debug_flags=dm.DM_DBG_THIN_STAGED)
-    assert dm.dm_step_launches(lora, staged, 1) == 4
+    assert dm.dm_step_launches(lora2, staged, 1) == 4
     # rank 32 has no cluster kernel
     lora32 = [fake_matrix(32, 4096), fake_matrix(4096, 32)] * 224
     for m in lora32:

@@ -28,8 +28,9 @@ def grads(seed):
 
 @pytest.mark.parametrize("prec,path", [(dm.DM_PREC_BF16_TC, 0), (dm.DM_PREC_FP32, 0),
                                        (dm.DM_PREC_BF16_TC, dm.DM_DBG_THIN_STAGED),
-                                       (dm.DM_PREC_BF16_TC, dm.DM_DBG_THIN_REGS)],
-                         ids=["tc", "fp32", "thin-staged", "thin-regs"])
+                                       (dm.DM_PREC_BF16_TC, dm.DM_DBG_THIN_REGS),
+                                       (dm.DM_PREC_BF16_TC, dm.DM_DBG_THIN_CLUSTER)],
+                         ids=["tc", "fp32", "thin-staged", "thin-regs", "thin-cluster"])
 @pytest.mark.parametrize("cond", [False, True])
 def test_checked_mode_leaves_canaries_and_results(prec, path, cond):
     plain = Group(SHAPES, BF, BF, F32, cond=cond, seed=81)

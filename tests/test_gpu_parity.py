@@ -110,11 +110,17 @@ def test_ns_step_counts(ns_steps):
 # --------------------------------------------------------------------------
 THIN_SHAPES = [(4, 16), (2, 100), (8, 4096), (4096, 8), (17, 333), (32, 4096), (4096, 32),
                (1, 50), (50, 1), (31, 31), (16, 1000), (2, 2056), (3000, 4), (8, 24),
-               (1001, 8), (4099, 16), (777, 32), (13, 8)]
+               (1001, 8), (4099, 16), (777, 32), (13, 8), (2, 5128), (5128, 2), (4, 4096),
+               (4096, 4)]
 
 
-@pytest.mark.parametrize("path", [0, dm.DM_DBG_THIN_STAGED, dm.DM_DBG_THIN_REGS],
-                         ids=["default", "staged", "regs"])
+# default: the cluster kernel for r <= 4 (r = 2 factors whose long side is an
+# odd multiple of 8 above 2560, such as 5128, take the one-CTA single-pass
+# kernel), the staged kernels for r = 8 .. 32; cluster: r = 8 on the cluster
+# kernel too
+@pytest.mark.parametrize("path", [0, dm.DM_DBG_THIN_STAGED, dm.DM_DBG_THIN_REGS,
+                                  dm.DM_DBG_THIN_CLUSTER],
+                         ids=["default", "staged", "regs", "cluster"])
 @pytest.mark.parametrize("cond", [False, True])
 @pytest.mark.parametrize("mdt", [F32, BF])
 def test_thin_path(cond, mdt, path):
@@ -330,8 +336,9 @@ def test_large_batch_dimuon_sampled():
     assert len(rep.sv_err) == len(LARGE_SAMPLE)
 
 
-@pytest.mark.parametrize("r", [2, 8, 32])
-def test_lora_batch_twenty_steps(r):
+@pytest.mark.parametrize("r,path", [(2, 0), (8, 0), (8, dm.DM_DBG_THIN_CLUSTER), (32, 0)],
+                         ids=["r2", "r8", "r8-cluster", "r32"])
+def test_lora_batch_twenty_steps(r, path):
     """224 projections (A r x 4096, B 4096 x r), fp32 momentum, bf16 weights,
     Dimuon, 20 steps: teacher-forced parity on a sample each step, dead rows
     of B capped at a 10x per-side gain, and a free-running oracle rerun of
@@ -340,7 +347,7 @@ def test_lora_batch_twenty_steps(r):
     stream = workloads.LoraGradStream(r)
     grp = Group(shapes, BF, BF, F32, cond=True, seed=4)
     lr = {2: 0.018, 8: 0.010, 32: 0.010}[r]
-    hp = hparams(dm.DM_PREC_BF16_TC, lr=lr)
+    hp = hparams(dm.DM_PREC_BF16_TC, lr=lr, debug_flags=path)
     ws = None
     h = orc.HParams(lr=lr)
     free = None
@@ -436,8 +443,10 @@ SCHED_SHAPES = [(384, 640), (700, 260), (40, 100), (8, 4096), (4096, 8), (2, 205
 @pytest.mark.parametrize("prec,dbg,tol", [
     (dm.DM_PREC_BF16_TC, 0, TOL_BF16), (dm.DM_PREC_BF16_TC, dm.DM_DBG_TC_SINGLE, TOL_BF16),
     (dm.DM_PREC_FP32, 0, TOL_FP32), (dm.DM_PREC_FP32, dm.DM_DBG_THIN_STAGED, TOL_FP32),
-    (dm.DM_PREC_FP32, dm.DM_DBG_THIN_REGS, TOL_FP32)],
-    ids=["tc-pair", "tc-single", "simt+thin-fused", "simt+thin-staged", "simt+thin-regs"])
+    (dm.DM_PREC_FP32, dm.DM_DBG_THIN_REGS, TOL_FP32),
+    (dm.DM_PREC_FP32, dm.DM_DBG_THIN_CLUSTER, TOL_FP32)],
+    ids=["tc-pair", "tc-single", "simt+thin-default", "simt+thin-staged", "simt+thin-regs",
+         "simt+thin-cluster"])
 @pytest.mark.parametrize("cond", [False, True])
 def test_coefficient_schedule(prec, dbg, tol, cond):
     """Iteration k applies its own (a_k, b_k, c_k) on every path: tensor-core
