@@ -107,6 +107,25 @@ def step_bytes(spec):
     return sum(r * c for r, c in spec["shapes"]) * (2 + 2 * mb + 4)
 
 
+def thin_fp64_flops(spec, thin_max=32):
+    """Algorithmic fp64 flops of the thin-factor path per step: per long-side
+    column of a factor with short side r, the Gram sums S_1 (and S_2 when
+    conditioned), r (r + 1) / 2 multiply-adds each, and O = T b, r^2; two
+    flops per multiply-add.  (The r x r iteration is O(r^3) per factor.)"""
+    tot = 0.0
+    for rows, cols in spec["shapes"]:
+        r, n = min(rows, cols), max(rows, cols)
+        if r > thin_max:
+            continue
+        tot += 2.0 * n * (r * (r + 1) / 2 * (2 if spec["cond"] else 1) + r * r)
+    return tot
+
+
+# fp64 fused multiply-adds per clock of one B200 SM (NVIDIA's 40 TF/s fp64 figure:
+# 148 SMs x 64 FMA x 2 flops at the boost clock)
+FP64_FMA_PER_SM_CLK = 64
+
+
 # DRAM traffic of the tensor-core product per launch (ncu dram__bytes_read.sum +
 # dram__bytes_write.sum of the quarter batch, same shapes, scaled by 4), valid
 # only for the kernel build the ncu capture was taken from.
@@ -605,11 +624,26 @@ def main():
         label = ("thin_cluster (the whole step in one launch per 448 factors)"
                  if per_step <= -(-len(shapes) // 448) else
                  "thin path (thin_setup, thin_gram, thin_iterate, thin_apply; or thin_fused)")
-        roofline = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                    "frac": gbs / peak, "traffic": None,
-                    "kernel": label + ": algorithmic bytes of the whole step over the step time",
-                    "launches_per_step": per_step,
-                    "peak_kind": f"{peak_kind} HBM copy"}
+        # the bound is the slower floor: the step's algorithmic bytes at the HBM
+        # copy rate, or its fp64 arithmetic at the fp64 FMA rate (r = 32)
+        mhz = clocks.get("sm_mhz") or 1965.0
+        f64_peak = 148 * FP64_FMA_PER_SM_CLK * 2 * mhz * 1e6 / 1e12
+        flops = thin_fp64_flops(spec)
+        if flops / (f64_peak * 1e12) > step_bytes(spec) / (peak * 1e9):
+            roofline = {"bound": "alu", "achieved": flops / (ms_step / 1e3) / 1e12,
+                        "peak": f64_peak, "unit": "TFLOP/s",
+                        "frac": flops / (ms_step / 1e3) / 1e12 / f64_peak, "traffic": None,
+                        "kernel": label + ": algorithmic fp64 flops of the whole step over the "
+                                          "step time",
+                        "launches_per_step": per_step, "hbm_GBps": gbs, "hbm_frac": gbs / peak,
+                        "peak_kind": f"derived fp64 FMA peak at the sampled {mhz:.0f} MHz"}
+        else:
+            roofline = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                        "frac": gbs / peak, "traffic": None,
+                        "kernel": label + ": algorithmic bytes of the whole step over the step "
+                                          "time",
+                        "launches_per_step": per_step,
+                        "peak_kind": f"{peak_kind} HBM copy"}
 
     # end to end through the public API: every step's gradients copied in from
     # pinned host memory, its status word read back.  Two device gradient sets:

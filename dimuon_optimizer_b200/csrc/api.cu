@@ -511,11 +511,26 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
   const bool canaries = !L.canary.empty();
   DM_CUDA(cudaMemsetAsync(ws, 0, canaries ? THIN_CTR_OFFSET + 2 * sizeof(int) * L.thin.size()
                                           : HEADER_BYTES, s));
+  // signature of this layout (FNV-1a over the size and the canary blocks):
+  // only a checked step of the same layout arms the between-steps check, so
+  // a workspace last used with other shapes (or reused memory) is not
+  // mistaken for a damaged one
+  uint32_t sig = 2166136261u;
+  auto mix = [&](uint64_t v) {
+    for (int k = 0; k < 8; ++k) {
+      sig ^= (uint32_t)((v >> (8 * k)) & 0xFFu);
+      sig *= 16777619u;
+    }
+  };
+  mix(L.bytes);
+  for (uint32_t b : L.canary) mix(b);
+  if (sig == 0) sig = 1;
   auto canary_pass = [&](int mode) -> cudaError_t {
     static thread_local CanaryParams cp;
     for (size_t b = 0; b < L.canary.size(); b += CANARY_MAX) {
       cp.count = (int)std::min<size_t>(CANARY_MAX, L.canary.size() - b);
       cp.mode = mode;
+      cp.arm = sig;
       cp.status = status;
       std::memcpy(cp.blk, L.canary.data() + b, sizeof(uint32_t) * cp.count);
       const cudaError_t e = launch_canary(cp, s);

@@ -275,14 +275,15 @@ int thin_slab(int pad);
 // ----------------------------- canaries -----------------------------------
 // Checked-workspace mode: 256-byte canaries (64 words) at the listed 256-byte
 // blocks of the workspace.  mode 0 (step start): check them if the arm word
-// holds CANARY_ARMED, then fill; mode 1 (step end): check, then arm.
+// holds this layout's signature (left by a checked step of the same layout),
+// then fill; mode 1 (step end): check, then write the signature.
 constexpr uint32_t CANARY_FILL = 0xA5C3A5C3u;
-constexpr uint32_t CANARY_ARMED = 0x43414E59u;
 constexpr int CANARY_ARM_WORD = 255;      // int32 index in the 1 KB header
 constexpr int CANARY_MAX = 7000;          // canaries per launch
 struct CanaryParams {
   int count;
   int mode;
+  uint32_t arm;               // layout signature (never 0)
   int* status;                // the workspace base (status word first)
   uint32_t blk[CANARY_MAX];   // canary offsets / 256
 };

@@ -43,6 +43,10 @@
  *     return an error before launching anything; otherwise they enqueue all
  *     work on `stream` (a cudaStream_t; NULL = legacy default stream) and
  *     return without synchronising.  No C++ exception crosses this ABI.
+ *   - Streams are passed as void* (a cudaStream_t cast to void*) so that the
+ *     header needs no CUDA header; device status values are returned as
+ *     int32_t holding a dm_status_t code, for a fixed width across
+ *     compilers.
  *   - Conditions found on the device (a non-finite Frobenius norm, a bounded
  *     wait that ran out) are written to a status word inside the workspace;
  *     dm_read_device_status synchronises the stream and reads it.  Each step
@@ -187,10 +191,12 @@ typedef struct {
                                      grows accordingly; pass the flag to
                                      both calls).  The step fills them at
                                      its start, after checking those a
-                                     previous canary step left (the first
-                                     canary after the header sits at byte
-                                     1024), and checks them all at its end;
-                                     a changed byte sets DM_ERR_CANARY.
+                                     previous checked step of the same
+                                     shapes left in this workspace (the
+                                     first canary after the header sits at
+                                     byte 1024), and checks them all at its
+                                     end; a changed byte sets
+                                     DM_ERR_CANARY.
                                      Costs two small launches; the
                                      arithmetic is unchanged.              */
 #define DM_DBG_FORCE_TIMEOUT 0x8u /* failure-detection hook: each

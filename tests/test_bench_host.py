@@ -142,3 +142,19 @@ def test_sharded_line_shape():
     assert "reduce-scatter" in d["config"]["parallelism"]
     assert d["config"]["workload"] == spec["desc"]
     json.dumps(d)
+
+
+def test_thin_fp64_flops():
+    """Per column of a rank-r factor: S_1 and S_2 (conditioned) upper
+    triangles and O = T b, two flops per multiply-add; matrices with a short
+    side above 32 are not thin."""
+    spec = {"shapes": [(8, 100), (100, 8), (64, 64)], "cond": True}
+    per_col = 2 * (36 * 2 + 64)
+    assert bench.thin_fp64_flops(spec) == 2 * 100 * per_col
+    spec["cond"] = False
+    assert bench.thin_fp64_flops(spec) == 2 * 100 * 2 * (36 + 64)
+    # the LoRA rank-32 batch is bound by fp64 arithmetic, rank 8 by HBM
+    r32, r8 = bench.workload_spec("lora_r32"), bench.workload_spec("lora_r8")
+    f64 = 148 * bench.FP64_FMA_PER_SM_CLK * 2 * 1965e6
+    assert bench.thin_fp64_flops(r32) / f64 > bench.step_bytes(r32) / 6.5e12
+    assert bench.thin_fp64_flops(r8) / f64 < bench.step_bytes(r8) / 6.5e12
