@@ -50,6 +50,7 @@ DM_DBG_THIN_REGS = 0x10
 DM_DBG_THIN_STAGED = 0x20
 DM_DBG_CANARY = 0x40
 DM_DBG_THIN_CLUSTER = 0x80
+DM_DBG_CANARY_SELFTEST = 0x100
 
 DM_NOALLOC_MAX_BYTES = 32 * 1024 * 1024
 

@@ -158,8 +158,8 @@ Layout make_layout(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, int c
       if (L.tc)  // enough (sum x^2, sum y^2) slots for either tensor-core kernel
         p.n_part = (int)std::max(ceil_div(p.rows, TC_BM) * ceil_div(p.cols, TC_BN) * 8,
                                  ceil_div(p.rows, TC2_BM) * ceil_div(p.cols, TC2_BN) * 16);
-      else
-        p.n_part = (int)(ceil_div(p.rows, 128) * ceil_div(p.cols, 128));
+      else  // fp32 products: one (sum x^2, sum y^2) per tile, tiles of 64 at the most
+        p.n_part = (int)(ceil_div(p.rows, 64) * ceil_div(p.cols, 64));
       p.off_scal = take(SC_COUNT * sizeof(float), 256);
       p.off_psum = take((size_t)p.k1_rt * p.k1_ct * sizeof(float), 256);
       if (L.cond) {
@@ -506,31 +506,15 @@ dm_status_t run_step(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, voi
   int dev = 0;
   DM_CUDA(cudaGetDevice(&dev));
 
-  // status word and thin slab counters; outside the checked mode the whole
-  // header, so a later checked step finds no stale arm word
+  // status word and thin slab counters
   const bool canaries = !L.canary.empty();
-  DM_CUDA(cudaMemsetAsync(ws, 0, canaries ? THIN_CTR_OFFSET + 2 * sizeof(int) * L.thin.size()
-                                          : HEADER_BYTES, s));
-  // signature of this layout (FNV-1a over the size and the canary blocks):
-  // only a checked step of the same layout arms the between-steps check, so
-  // a workspace last used with other shapes (or reused memory) is not
-  // mistaken for a damaged one
-  uint32_t sig = 2166136261u;
-  auto mix = [&](uint64_t v) {
-    for (int k = 0; k < 8; ++k) {
-      sig ^= (uint32_t)((v >> (8 * k)) & 0xFFu);
-      sig *= 16777619u;
-    }
-  };
-  mix(L.bytes);
-  for (uint32_t b : L.canary) mix(b);
-  if (sig == 0) sig = 1;
+  DM_CUDA(cudaMemsetAsync(ws, 0, THIN_CTR_OFFSET + 2 * sizeof(int) * L.thin.size(), s));
   auto canary_pass = [&](int mode) -> cudaError_t {
     static thread_local CanaryParams cp;
     for (size_t b = 0; b < L.canary.size(); b += CANARY_MAX) {
       cp.count = (int)std::min<size_t>(CANARY_MAX, L.canary.size() - b);
       cp.mode = mode;
-      cp.arm = sig;
+      cp.plant = (hp->debug_flags & DM_DBG_CANARY_SELFTEST) != 0 && b == 0;
       cp.status = status;
       std::memcpy(cp.blk, L.canary.data() + b, sizeof(uint32_t) * cp.count);
       const cudaError_t e = launch_canary(cp, s);
@@ -829,9 +813,8 @@ dm_status_t run_body(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, con
         }
   } else {
     static thread_local SimtParams ps;
-    for (int k = 1; k <= hp->ns_steps; ++k)
-      for (int ph = 0; ph < 3; ++ph)
-        for (size_t b = 0; b < big.size(); b += SIMT_MAX) {
+    const int nsm = sm_count(dev);
+    auto build_simt = [&](size_t b, int ph, int k, int tb) {
           std::memset(&ps, 0, sizeof(ps));
           ps.lr = hp->lr;
           ps.decay = decay;
@@ -841,7 +824,7 @@ dm_status_t run_body(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, con
             const MatPlan& p = *big[q];
             SimtMat& sm = ps.mats[ps.count];
             const OperandSrc src = fill_gemm(sm.g, p, mats[p.idx], hp, ws, ph, k, cond != 0,
-                                             kappa_of(hp, p.rows, p.cols), 128, 128);
+                                             kappa_of(hp, p.rows, p.cols), tb, tb);
             auto ptr = [&](int buf) -> const float* {
               return reinterpret_cast<const float*>(
                   ws + (buf < 2 ? p.off_X[buf] : (buf == 2 ? p.off_A : p.off_B)));
@@ -852,10 +835,27 @@ dm_status_t run_body(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, con
             sm.lda = ld(src.a_buf);
             sm.ldb = ld(src.b_buf);
             ps.starts[ps.count++] = tiles;
-            tiles += gemm_tile_count(sm.g, 128, 128);
+            tiles += gemm_tile_count(sm.g, tb, tb);
           }
           ps.starts[ps.count] = tiles;
-          DM_CUDA(launch_simt(ps, tiles, s));
+          return tiles;
+    };
+    for (int k = 1; k <= hp->ns_steps; ++k)
+      for (int ph = 0; ph < 3; ++ph)
+        for (size_t b = 0; b < big.size(); b += SIMT_MAX) {
+          // 128 x 128 tiles, or 64 x 64 when those would leave SMs idle
+          int tb = 128;
+          int tiles = build_simt(b, ph, k, tb);
+          if (tiles < 2 * nsm) {
+            tb = 64;
+            tiles = build_simt(b, ph, k, tb);
+          }
+          DM_CUDA(launch_simt(ps, tiles, tb, s));
+          if (k == hp->ns_steps && ph == PH_GEMM)
+            for (size_t q = b; q < std::min(big.size(), b + SIMT_MAX); ++q) {
+              const MatPlan& p = *big[q];
+              final_npart[p.idx] = (int)(ceil_div(p.rows, tb) * ceil_div(p.cols, tb));
+            }
         }
   }
   // K3a / K3
@@ -886,7 +886,7 @@ dm_status_t run_body(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, con
         k.wdt = um.weight_dtype;
         k.vec = (p.cols % 8 == 0) && !(reinterpret_cast<uintptr_t>(um.weight) & 15u) &&
                 !(reinterpret_cast<uintptr_t>(um.update_out) & 15u);
-        k.n_part = L.tc ? final_npart[p.idx] : p.n_part;
+        k.n_part = final_npart[p.idx];
         k.n_rt = p.k1_rt;
         k.n_ct = p.k1_ct;
         k.kappa = kappa_of(hp, p.rows, p.cols);

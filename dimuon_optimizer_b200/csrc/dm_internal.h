@@ -274,16 +274,15 @@ int thin_slab(int pad);
 
 // ----------------------------- canaries -----------------------------------
 // Checked-workspace mode: 256-byte canaries (64 words) at the listed 256-byte
-// blocks of the workspace.  mode 0 (step start): check them if the arm word
-// holds this layout's signature (left by a checked step of the same layout),
-// then fill; mode 1 (step end): check, then write the signature.
+// blocks of the workspace.  mode 0 (step start): fill; mode 1 (step end):
+// check.  `plant` (self-test hook) leaves the first word of the first canary
+// wrong at the fill.
 constexpr uint32_t CANARY_FILL = 0xA5C3A5C3u;
-constexpr int CANARY_ARM_WORD = 255;      // int32 index in the 1 KB header
 constexpr int CANARY_MAX = 7000;          // canaries per launch
 struct CanaryParams {
   int count;
   int mode;
-  uint32_t arm;               // layout signature (never 0)
+  int plant;
   int* status;                // the workspace base (status word first)
   uint32_t blk[CANARY_MAX];   // canary offsets / 256
 };
@@ -296,7 +295,8 @@ cudaError_t launch_k1(const K1Params& p, int total_tiles, cudaStream_t s);
 cudaError_t launch_k1b(const K1bParams& p, int total_blocks, cudaStream_t s);
 cudaError_t launch_k3a(const K3Params& p, cudaStream_t s);
 cudaError_t launch_k3(const K3Params& p, int total_tiles, cudaStream_t s);
-cudaError_t launch_simt(const SimtParams& p, int total_tiles, cudaStream_t s);
+// tile: 128 (128 x 128 tiles) or 64 (64 x 64 tiles)
+cudaError_t launch_simt(const SimtParams& p, int total_tiles, int tile, cudaStream_t s);
 cudaError_t launch_tc(const TcParams& p, int grid, cudaStream_t s);
 int tc_smem_bytes();
 constexpr int TC2_BM = 256, TC2_BN = 256;  // CTA-pair output tile

@@ -247,11 +247,10 @@ __global__ void __launch_bounds__(256) k3_apply(const __grid_constant__ K3Params
 __global__ void __launch_bounds__(64) k_canary(const __grid_constant__ CanaryParams p) {
   uint32_t* base = reinterpret_cast<uint32_t*>(p.status);
   uint32_t* c = base + (size_t)p.blk[blockIdx.x] * 64;
-  const bool check =
-      p.mode == 1 || reinterpret_cast<volatile uint32_t*>(base)[CANARY_ARM_WORD] == p.arm;
-  if (check && c[threadIdx.x] != CANARY_FILL) raise_status(p.status, ST_CANARY);
-  if (p.mode == 0) c[threadIdx.x] = CANARY_FILL;
-  if (p.mode == 1 && blockIdx.x == 0 && threadIdx.x == 0) base[CANARY_ARM_WORD] = p.arm;
+  if (p.mode == 0)
+    c[threadIdx.x] = (p.plant && blockIdx.x == 0 && threadIdx.x == 0) ? ~CANARY_FILL : CANARY_FILL;
+  else if (c[threadIdx.x] != CANARY_FILL)
+    raise_status(p.status, ST_CANARY);
 }
 
 cudaError_t launch_canary(const CanaryParams& p, cudaStream_t s) {

@@ -85,8 +85,8 @@ typedef enum {
                                  A norm below 1e-15 also gives O = 0, without
                                  a status (nothing to normalise).             */
   DM_ERR_CANARY = 7           /* device status (DM_DBG_CANARY only): a canary
-                                 word between workspace regions was changed,
-                                 during the step or since the previous one    */
+                                 word between workspace regions was changed
+                                 during the step                              */
 } dm_status_t;
 
 typedef enum { DM_BF16 = 0, DM_FP32 = 1 } dm_dtype_t;
@@ -190,15 +190,15 @@ typedef struct {
                                      workspace region (dm_workspace_size
                                      grows accordingly; pass the flag to
                                      both calls).  The step fills them at
-                                     its start, after checking those a
-                                     previous checked step of the same
-                                     shapes left in this workspace (the
-                                     first canary after the header sits at
-                                     byte 1024), and checks them all at its
+                                     its start and checks them all at its
                                      end; a changed byte sets
                                      DM_ERR_CANARY.
                                      Costs two small launches; the
                                      arithmetic is unchanged.              */
+#define DM_DBG_CANARY_SELFTEST 0x100u /* checker self-test hook (with
+                                     DM_DBG_CANARY): the fill leaves one
+                                     canary word wrong, so the step must
+                                     end with DM_ERR_CANARY                */
 #define DM_DBG_FORCE_TIMEOUT 0x8u /* failure-detection hook: each
                                      tensor-core product launch makes one
                                      bounded wait run out (20 ms, on a

@@ -1,9 +1,9 @@
 """Checked-workspace mode (DM_DBG_CANARY): 256 canary bytes after the
 workspace header and after every workspace region, filled at a step's start
-and checked at its end (and, at the next checked step's start, for writes
-between steps).  Stand-in for a memory sanitizer, which this pool does not
-offer: every path's kernels must leave all canaries intact, with results
-bit-equal to the unchecked mode, and a changed canary must be reported."""
+and checked at its end.  Stand-in for a memory sanitizer, which this pool
+does not offer: every path's kernels must leave all canaries intact, with
+results bit-equal to the unchecked mode, and a changed canary must be
+reported."""
 import numpy as np
 import pytest
 import torch
@@ -59,25 +59,27 @@ def test_checked_mode_leaves_canaries_and_results(prec, path, cond):
 
 
 def test_changed_canary_is_reported():
-    """A byte of the canary after the header (byte 1024) changed between two
-    checked steps is reported by the second; the step after that refills the
-    canaries and reads clean again."""
+    """The checker's self-test hook leaves one canary word wrong at the fill:
+    the step must end with DM_ERR_CANARY, and the next checked step (which
+    refills the canaries) reads clean again, with the same results as an
+    unchecked step."""
     grp = Group(SHAPES[:4], BF, BF, F32, cond=True, seed=82)
+    ref = Group(SHAPES[:4], BF, BF, F32, cond=True, seed=82)
     hp = dm.dm_default_hparams(debug_flags=dm.DM_DBG_CANARY)
+    bad = dm.dm_default_hparams(debug_flags=dm.DM_DBG_CANARY | dm.DM_DBG_CANARY_SELFTEST)
     G = [to_dev(g, BF) for g in grads(95)[:4]]
     mats = grp.matrices(G)
     ws = torch.empty(dm.dm_workspace_size(mats, hp, 1), dtype=torch.uint8, device="cuda")
-    dm.check(dm.dm_dimuon_step(mats, hp, ws))
-    assert dm.dm_read_device_status(ws) == dm.DM_OK
-    ws[1024 + 5] = ws[1024 + 5] ^ 0xFF
-    dm.check(dm.dm_dimuon_step(mats, hp, ws))
+    dm.check(dm.dm_dimuon_step(mats, bad, ws))
     assert dm.dm_read_device_status(ws) == dm.DM_ERR_CANARY
     dm.check(dm.dm_dimuon_step(mats, hp, ws))
     assert dm.dm_read_device_status(ws) == dm.DM_OK
-    # an unchecked step disarms the canaries: a later checked step does not
-    # take its leftovers for canaries
+    # the hook changes a canary, not the arithmetic
     hp0 = dm.dm_default_hparams()
-    dm.check(dm.dm_dimuon_step(mats, hp0, ws))
-    ws[1024 + 5] = 0
-    dm.check(dm.dm_dimuon_step(mats, hp, ws))
-    assert dm.dm_read_device_status(ws) == dm.DM_OK
+    mref = ref.matrices(G)
+    ws0 = torch.empty(dm.dm_workspace_size(mref, hp0, 1), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        dm.check(dm.dm_dimuon_step(mref, hp0, ws0))
+    for name in ("W", "M", "er", "ec", "upd"):
+        for a, b in zip(getattr(grp, name), getattr(ref, name)):
+            assert torch.equal(a, b), name
