@@ -385,10 +385,13 @@ def run_sharded(args, spec, rank, world, local):
     nbytes = sharded.workspace_bytes(sw, rank, sg.views, M, hp, spec["cond"], ER, EC)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
 
+    owned = sharded.owned_matrices(sw, rank, sg, M, conditioned=spec["cond"], row_energy=ER,
+                                   col_energy=EC)
+
     def step():
         sg.flat.copy_(local_grads)  # this rank's backward output
         sharded.sharded_step(sw, rank, sg, M, hp, ws, conditioned=spec["cond"], row_energy=ER,
-                             col_energy=EC)
+                             col_energy=EC, mats=owned)
 
     def exchange_only():
         sg.reduce(rank)

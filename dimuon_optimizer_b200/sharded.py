@@ -141,9 +141,25 @@ class ShardedGrads:
         self.flat[rank * s:(rank + 1) * s].copy_(self._recv)
 
 
+def owned_matrices(weights: ShardedWeights, rank: int, grads, momenta, *, conditioned=False,
+                   row_energy=None, col_energy=None, update_out=None):
+    """The library's matrix descriptors for the matrices `rank` owns, built
+    once: pass them to sharded_step as `mats` while the same tensors are used
+    step after step (the descriptors hold their addresses).  `grads` as in
+    sharded_step (a ShardedGrads: its views)."""
+    from . import _array, dm_matrix
+    views = grads.views if isinstance(grads, ShardedGrads) else grads
+    idx = weights.plan.owned(rank)
+    mats = [dm_matrix(weights.views[i], views[i], momenta[i],
+                      row_energy[i] if conditioned else None,
+                      col_energy[i] if conditioned else None,
+                      update_out.get(i) if update_out else None) for i in idx]
+    return _array(mats)[0] if mats else None
+
+
 def sharded_step(weights: ShardedWeights, rank: int, grads, momenta, hp, workspace, *,
                  conditioned=False, row_energy=None, col_energy=None, update_out=None,
-                 stream=None, group=None):
+                 stream=None, group=None, mats=None):
     """One sharded step: the library updates this rank's matrices in place in
     the flat buffer, then the slices are all-gathered.
 
@@ -154,6 +170,7 @@ def sharded_step(weights: ShardedWeights, rank: int, grads, momenta, hp, workspa
     momenta / row_energy / col_energy / update_out: dicts from matrix index to
               tensor, for the owned matrices only
     workspace: device buffer of at least workspace_bytes(...) for the owned set
+    mats:     optional descriptors from owned_matrices (skips rebuilding them)
     """
     from . import dm_dimuon_step, dm_matrix, dm_muon_step, check
     if isinstance(grads, ShardedGrads):
@@ -161,12 +178,13 @@ def sharded_step(weights: ShardedWeights, rank: int, grads, momenta, hp, workspa
         grads = grads.views
         if stream is not None:
             stream.wait_stream(torch.cuda.current_stream())
-    idx = weights.plan.owned(rank)
-    mats = [dm_matrix(weights.views[i], grads[i], momenta[i],
-                      row_energy[i] if conditioned else None,
-                      col_energy[i] if conditioned else None,
-                      update_out.get(i) if update_out else None) for i in idx]
-    if mats:
+    if mats is None:
+        idx = weights.plan.owned(rank)
+        mats = [dm_matrix(weights.views[i], grads[i], momenta[i],
+                          row_energy[i] if conditioned else None,
+                          col_energy[i] if conditioned else None,
+                          update_out.get(i) if update_out else None) for i in idx]
+    if mats is not None and len(mats):
         fn = dm_dimuon_step if conditioned else dm_muon_step
         check(fn(mats, hp, workspace, stream=stream))
     if stream is not None:

@@ -14,9 +14,10 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 
+@pytest.mark.parametrize("prebuilt", [False, True], ids=["per_call", "prebuilt"])
 @pytest.mark.parametrize("flat_grads", [False, True], ids=["grad_list", "grad_flat"])
 @pytest.mark.parametrize("cond", [False, True])
-def test_sharded_single_rank_matches_plain_step(cond, flat_grads):
+def test_sharded_single_rank_matches_plain_step(cond, flat_grads, prebuilt):
     shapes = workloads.gpt2_small_shapes(layers=1) + workloads.lora_shapes(8, projections=3)
     plan = sharded.plan_shards(shapes, 1)
     sw = sharded.ShardedWeights(plan, dtype=torch.bfloat16, device="cuda")
@@ -43,9 +44,11 @@ def test_sharded_single_rank_matches_plain_step(cond, flat_grads):
         grads = sharded.ShardedGrads(plan, dtype=torch.bfloat16, device="cuda")
         for v, g in zip(grads.views, G):
             v.copy_(g)
+    owned = (sharded.owned_matrices(sw, 0, grads, M1, conditioned=cond, row_energy=er1,
+                                    col_energy=ec1) if prebuilt else None)
     for _ in range(2):
         sharded.sharded_step(sw, 0, grads, M1, hp, ws1, conditioned=cond, row_energy=er1,
-                             col_energy=ec1)
+                             col_energy=ec1, mats=owned)
         dm.check((dm.dm_dimuon_step if cond else dm.dm_muon_step)(mats, hp, ws2))
     torch.cuda.synchronize()
     for i in range(len(shapes)):
