@@ -147,28 +147,216 @@ __device__ __forceinline__ void epilogue32(const GemmMat& g, float lr, float dec
   }
 }
 
+// ---------------------------------------------------------------------------
+// Staged epilogue for whole 32 x 32 blocks.  A thread holds one row of the
+// accumulator (tcgen05.ld 32x32b), so its own row accesses would make every
+// warp-wide load or store touch 32 rows.  Instead the warp moves whole blocks
+// through a 32 x 32 bf16 tile in shared memory: global loads and stores are
+// 16 bytes per lane covering 8 rows x 64 bytes per instruction (4 instructions
+// per block instead of 4 x 32 row segments), and the symmetric products'
+// mirrored block leaves the tile transposed the same way.  Diagonal blocks of
+// the symmetric products, partial blocks at the matrix edges and fp32 weights
+// keep the row-per-thread path (epilogue32).
+// ---------------------------------------------------------------------------
+constexpr int SP = 40;                             // tile pitch in bf16 (80 bytes)
+constexpr int STAGE_TILE_BYTES = 32 * SP * 2;      // one epilogue warp's tile
+
+// Lane l's slot of a block: row (l >> 2) + 8 i, columns 8 (l & 3) .. + 7.
+__device__ __forceinline__ void blk_ld(const __nv_bfloat16* base, int ld, int r0, int c0,
+                                       uint4 q[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    q[i] = *reinterpret_cast<const uint4*>(base + (int64_t)(r0 + (lane >> 2) + 8 * i) * ld + c0 +
+                                           8 * (lane & 3));
+}
+__device__ __forceinline__ void blk_st(__nv_bfloat16* base, int ld, int r0, int c0, const uint4 q[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint4*>(base + (int64_t)(r0 + (lane >> 2) + 8 * i) * ld + c0 + 8 * (lane & 3)) =
+        q[i];
+}
+__device__ __forceinline__ void tile_put_blk(__nv_bfloat16* st, const uint4 q[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint4*>(st + ((lane >> 2) + 8 * i) * SP + 8 * (lane & 3)) = q[i];
+}
+__device__ __forceinline__ void tile_get_blk(const __nv_bfloat16* st, uint4 q[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    q[i] = *reinterpret_cast<const uint4*>(st + ((lane >> 2) + 8 * i) * SP + 8 * (lane & 3));
+}
+// Row `lane` of the tile from / to 32 fp32 values (bf16 stores round to
+// nearest even, as the row-per-thread path does).
+__device__ __forceinline__ void tile_put_row(__nv_bfloat16* st, const float v[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) st_bf16x8(st + lane * SP + 8 * k, v + 8 * k);
+}
+__device__ __forceinline__ void tile_get_row(const __nv_bfloat16* st, float v[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) ld_bf16x8(st + lane * SP + 8 * k, v + 8 * k);
+}
+// Column `lane` of the tile (the transposed block).
+__device__ __forceinline__ void tile_put_col(__nv_bfloat16* st, const float v[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) st[q * SP + lane] = __float2bfloat16_rn(v[q]);
+}
+
+// Whether the block of rows r0 .. r0 + 31, columns c0 .. c0 + 31 takes the
+// staged path (warp-uniform).
+__device__ __forceinline__ bool staged_ok(const GemmMat& g, int r0, int c0) {
+  if (r0 + 32 > g.M || c0 + 32 > g.N) return false;
+  switch (g.epi) {
+    case EPI_SYRK:
+    case EPI_POLY:
+      return c0 >= r0 + 32 || c0 + 32 <= r0;  // off the diagonal
+    case EPI_GEMM:
+    case EPI_FINAL_DIMUON:
+      return true;
+    case EPI_FINAL_MUON:
+      return g.wdt == DT_BF16 && (g.ldw & 7) == 0 && aligned16(g.W);
+  }
+  return false;
+}
+
+// A finished bf16 block (thread = row) to rows r0.., columns c0.. of `out`.
+__device__ __forceinline__ void staged_store(__nv_bfloat16* st, __nv_bfloat16* out, int ld, int r0,
+                                             int c0, const float v[32]) {
+  uint4 q[4];
+  tile_put_row(st, v);
+  __syncwarp();
+  tile_get_blk(st, q);
+  blk_st(out, ld, r0, c0, q);
+  __syncwarp();
+}
+
+// The staged form of epilogue32 for one whole block; `ax` already holds the
+// thread's row of the aux block.
+__device__ __forceinline__ void staged_epilogue32(const GemmMat& g, float lr, float decay, int r,
+                                                  int r0, int c0, float v[32], const float ax[32],
+                                                  float S, float valid, float& sx, float& sy,
+                                                  __nv_bfloat16* st) {
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out);
+  switch (g.epi) {
+    case EPI_SYRK:
+    case EPI_POLY: {
+      if (c0 + 32 <= r0) break;  // below the diagonal: another tile's mirror
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        v[q] = g.epi == EPI_SYRK ? v[q] * S : fmaf(g.coef_acc, v[q], g.coef_aux * ax[q]);
+      staged_store(st, out, g.ldo, r0, c0, v);
+      // the mirrored block: element (c, r) at row c of the output
+      uint4 q4[4];
+      tile_put_col(st, v);
+      __syncwarp();
+      tile_get_blk(st, q4);
+      blk_st(out, g.ldo, c0, r0, q4);
+      __syncwarp();
+      break;
+    }
+    case EPI_GEMM: {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = fmaf(g.coef_aux, ax[q], v[q]) * S;
+      staged_store(st, out, g.ldo, r0, c0, v);
+      break;
+    }
+    case EPI_FINAL_DIMUON: {
+      const float rr = g.R[r];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        v[q] = round_to(fmaf(g.coef_aux, ax[q], v[q]) * S, DT_BF16);
+        const float y = rr * v[q] * g.C[c0 + q];
+        sx += v[q] * v[q];
+        sy += y * y;
+      }
+      staged_store(st, out, g.ldo, r0, c0, v);
+      break;
+    }
+    case EPI_FINAL_MUON: {
+      const float ks = valid != 0.f ? g.kappa * S : 0.f;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = (valid != 0.f) ? fmaf(g.coef_aux, ax[q], v[q]) * ks : 0.f;
+      __nv_bfloat16* W = reinterpret_cast<__nv_bfloat16*>(g.W);
+      uint4 q4[4];
+      float w[32];
+      blk_ld(W, g.ldw, r0, c0, q4);
+      tile_put_blk(st, q4);
+      __syncwarp();
+      tile_get_row(st, w);
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 32; ++q) w[q] = decay * w[q] - lr * v[q];
+      staged_store(st, W, g.ldw, r0, c0, w);
+      if (g.upd) {
+        const int64_t wi = (int64_t)r * g.ldw + c0;
+        if (aligned16(g.upd + wi)) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) st8(g.upd, wi + 8 * q, DT_FP32, v + 8 * q);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) g.upd[wi + q] = v[q];
+        }
+      }
+      break;
+    }
+  }
+}
+
 // Epilogue of chunks [ch_begin, ch_end) (32 columns each) of one accumulator
-// row: tcgen05.ld of each chunk, with the next chunk's aux row in flight while
-// the current one is processed.  Must be executed by all 32 lanes of the warp
+// row: tcgen05.ld of each chunk, with the next chunk's aux in flight while
+// the current one is processed (as a whole block for staged chunks, as the
+// thread's row otherwise).  Must be executed by all 32 lanes of the warp
 // (tcgen05.ld is warp-collective); rows outside the matrix only skip stores.
+// `st` is this warp's staging tile (STAGE_TILE_BYTES of shared memory).
 __device__ __forceinline__ void epilogue_row(const GemmMat& g, float lr, float decay, int r,
                                              bool row_ok, int col0, uint32_t taddr, int ch_begin,
-                                             int ch_end, int nch, float& sx, float& sy) {
+                                             int ch_end, int nch, float& sx, float& sy,
+                                             __nv_bfloat16* st) {
+  const int r0 = r - (int)(threadIdx.x & 31);
   const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
   const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
   const bool aux = needs_aux(g.epi);
   const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(g.aux);
   float axn[32];
-  if (aux && row_ok && ch_begin < nch) load_row32(ab, g.ldaux, r, col0 + ch_begin * 32, g.N, axn);
+  uint4 qn[4];
+  auto prefetch = [&](int ch) {
+    if (!aux || ch >= ch_end || ch >= nch) return;
+    const int c0 = col0 + ch * 32;
+    if (staged_ok(g, r0, c0))
+      blk_ld(ab, g.ldaux, r0, c0, qn);
+    else if (row_ok)
+      load_row32(ab, g.ldaux, r, c0, g.N, axn);
+  };
+  prefetch(ch_begin);
 #pragma unroll 1
   for (int ch = ch_begin; ch < ch_end; ++ch) {
     float v[32], ax[32];
+    uint4 q[4];
     tmem_ld32_at(taddr + (uint32_t)(ch * 32), v);
+    const int c0 = col0 + ch * 32;
+    const bool stg = ch < nch && staged_ok(g, r0, c0);
 #pragma unroll
-    for (int q = 0; q < 32; ++q) ax[q] = axn[q];
-    if (aux && row_ok && ch + 1 < ch_end && ch + 1 < nch)
-      load_row32(ab, g.ldaux, r, col0 + (ch + 1) * 32, g.N, axn);
-    if (row_ok && ch < nch) epilogue32(g, lr, decay, r, col0 + ch * 32, v, ax, S, valid, sx, sy);
+    for (int k = 0; k < 4; ++k) q[k] = qn[k];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) ax[k] = axn[k];
+    prefetch(ch + 1);
+    if (stg) {
+      if (aux) {
+        tile_put_blk(st, q);
+        __syncwarp();
+        tile_get_row(st, ax);
+        __syncwarp();
+      }
+      staged_epilogue32(g, lr, decay, r, r0, c0, v, ax, S, valid, sx, sy, st);
+    } else if (row_ok && ch < nch) {
+      epilogue32(g, lr, decay, r, c0, v, ax, S, valid, sx, sy);
+    }
   }
 }
 

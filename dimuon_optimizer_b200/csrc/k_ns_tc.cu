@@ -35,7 +35,9 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
 constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t TMEM_COLS = 512;             // two 128 x 256 fp32 accumulators
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+// + one 32 x 32 bf16 staging tile per epilogue warp (coalesced epilogue)
+constexpr int EPI_STAGE_BYTES = 8 * STAGE_TILE_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES + 1024;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // any single wait > 2 s is a hang
 constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
 constexpr uint64_t FORCED_LIMIT_NS = 20000000ull;   // forced-timeout hook: 20 ms
@@ -225,7 +227,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
       float sx = 0.f, sy = 0.f;
       epilogue_row(g, p.lr, p.decay, r, r < g.M, tl.tn * TC_BN,
                    tmem_base + (uint32_t)(acc * TC_BN) + ((uint32_t)(quarter * 32) << 16),
-                   half * CH_PER, half * CH_PER + CH_PER, nch, sx, sy);
+                   half * CH_PER, half * CH_PER + CH_PER, nch, sx, sy,
+                   reinterpret_cast<__nv_bfloat16*>(smem + STAGES * STAGE_BYTES + BAR_BYTES) +
+                       ew * (STAGE_TILE_BYTES / 2));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
