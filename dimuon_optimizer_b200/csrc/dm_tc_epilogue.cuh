@@ -308,32 +308,40 @@ __device__ __forceinline__ void staged_epilogue32(const GemmMat& g, float lr, fl
   }
 }
 
+// The aux of one chunk in flight: a whole block for staged chunks, the
+// thread's row otherwise.
+struct AuxPrefetch {
+  float row[32];
+  uint4 blk[4];
+};
+
+__device__ __forceinline__ void fetch_aux(const GemmMat& g, int r, bool row_ok, int col0, int ch,
+                                          int ch_end, int nch, AuxPrefetch& pf) {
+  if (!needs_aux(g.epi) || ch >= ch_end || ch >= nch) return;
+  const int r0 = r - (int)(threadIdx.x & 31);
+  const int c0 = col0 + ch * 32;
+  const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(g.aux);
+  if (staged_ok(g, r0, c0))
+    blk_ld(ab, g.ldaux, r0, c0, pf.blk);
+  else if (row_ok)
+    load_row32(ab, g.ldaux, r, c0, g.N, pf.row);
+}
+
 // Epilogue of chunks [ch_begin, ch_end) (32 columns each) of one accumulator
 // row: tcgen05.ld of each chunk, with the next chunk's aux in flight while
-// the current one is processed (as a whole block for staged chunks, as the
-// thread's row otherwise).  Must be executed by all 32 lanes of the warp
+// the current one is processed.  `pf` holds chunk ch_begin's aux, fetched by
+// the caller (fetch_aux) before it waited for the accumulator, since the aux
+// does not depend on it.  Must be executed by all 32 lanes of the warp
 // (tcgen05.ld is warp-collective); rows outside the matrix only skip stores.
 // `st` is this warp's staging tile (STAGE_TILE_BYTES of shared memory).
 __device__ __forceinline__ void epilogue_row(const GemmMat& g, float lr, float decay, int r,
                                              bool row_ok, int col0, uint32_t taddr, int ch_begin,
                                              int ch_end, int nch, float& sx, float& sy,
-                                             __nv_bfloat16* st) {
+                                             __nv_bfloat16* st, AuxPrefetch& pf) {
   const int r0 = r - (int)(threadIdx.x & 31);
   const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
   const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
   const bool aux = needs_aux(g.epi);
-  const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(g.aux);
-  float axn[32];
-  uint4 qn[4];
-  auto prefetch = [&](int ch) {
-    if (!aux || ch >= ch_end || ch >= nch) return;
-    const int c0 = col0 + ch * 32;
-    if (staged_ok(g, r0, c0))
-      blk_ld(ab, g.ldaux, r0, c0, qn);
-    else if (row_ok)
-      load_row32(ab, g.ldaux, r, c0, g.N, axn);
-  };
-  prefetch(ch_begin);
 #pragma unroll 1
   for (int ch = ch_begin; ch < ch_end; ++ch) {
     float v[32], ax[32];
@@ -342,10 +350,10 @@ __device__ __forceinline__ void epilogue_row(const GemmMat& g, float lr, float d
     const int c0 = col0 + ch * 32;
     const bool stg = ch < nch && staged_ok(g, r0, c0);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) q[k] = qn[k];
+    for (int k = 0; k < 4; ++k) q[k] = pf.blk[k];
 #pragma unroll
-    for (int k = 0; k < 32; ++k) ax[k] = axn[k];
-    prefetch(ch + 1);
+    for (int k = 0; k < 32; ++k) ax[k] = pf.row[k];
+    fetch_aux(g, r, row_ok, col0, ch + 1, ch_end, nch, pf);
     if (stg) {
       if (aux) {
         tile_put_blk(st, q);

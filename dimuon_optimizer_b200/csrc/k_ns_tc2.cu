@@ -268,17 +268,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product_pair(const __gri
       const GemmMat& g = p.mats[tl.g].g;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort, p.status, WAIT_LIMIT_NS)) break;
-      tc_fence_after();
       const int r = tl.tm * PAIR_BM + (int)rank * HALF + row_in_half;
       const int nch = min(PAIR_BN, g.N - tl.tn * PAIR_BN + 31) / 32;  // chunks holding columns < N
       constexpr int CH_PER = PAIR_BN / 32 / 2;
+      // the first chunk's aux is in flight while the products run
+      AuxPrefetch pf;
+      fetch_aux(g, r, r < g.M, tl.tn * PAIR_BN, half * CH_PER, half * CH_PER + CH_PER, nch, pf);
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort, p.status, WAIT_LIMIT_NS)) break;
+      tc_fence_after();
       float sx = 0.f, sy = 0.f;
       epilogue_row(g, p.lr, p.decay, r, r < g.M, tl.tn * PAIR_BN,
                    tmem_base + (uint32_t)(acc * PAIR_BN) + ((uint32_t)(quarter * 32) << 16),
                    half * CH_PER, half * CH_PER + CH_PER, nch, sx, sy,
                    reinterpret_cast<__nv_bfloat16*>(smem + STAGES * STAGE_BYTES + BAR_BYTES) +
-                       ew * (STAGE_TILE_BYTES / 2));
+                       ew * (STAGE_TILE_BYTES / 2),
+                   pf);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
