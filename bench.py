@@ -107,15 +107,17 @@ def step_bytes(spec):
     return sum(r * c for r, c in spec["shapes"]) * (2 + 2 * mb + 4)
 
 
-def thin_fp64_flops(spec, thin_max=32):
+def thin_fp64_flops(spec, thin_max=32, split_r32=False):
     """Algorithmic fp64 flops of the thin-factor path per step: per long-side
     column of a factor with short side r, the Gram sums S_1 (and S_2 when
     conditioned), r (r + 1) / 2 multiply-adds each, and O = T b, r^2; two
-    flops per multiply-add.  (The r x r iteration is O(r^3) per factor.)"""
+    flops per multiply-add.  (The r x r iteration is O(r^3) per factor.)
+    With split_r32 (bf16 tensor-core mode) the r = 32 factors take those sums
+    on bf16 tensor cores and add no fp64 work."""
     tot = 0.0
     for rows, cols in spec["shapes"]:
         r, n = min(rows, cols), max(rows, cols)
-        if r > thin_max:
+        if r > thin_max or (split_r32 and r == 32):
             continue
         tot += 2.0 * n * (r * (r + 1) / 2 * (2 if spec["cond"] else 1) + r * r)
     return tot
@@ -629,10 +631,11 @@ def main():
                  if per_step <= -(-len(shapes) // 448) else
                  "thin path (thin_setup, thin_gram, thin_iterate, thin_apply; or thin_fused)")
         # the bound is the slower floor: the step's algorithmic bytes at the HBM
-        # copy rate, or its fp64 arithmetic at the fp64 FMA rate (r = 32)
+        # copy rate, or its fp64 arithmetic at the fp64 FMA rate (r = 32 in fp32
+        # mode; in bf16 mode those sums run on bf16 tensor cores)
         mhz = clocks.get("sm_mhz") or 1965.0
         f64_peak = 148 * FP64_FMA_PER_SM_CLK * 2 * mhz * 1e6 / 1e12
-        flops = thin_fp64_flops(spec)
+        flops = thin_fp64_flops(spec, split_r32=args.precision == "bf16")
         if flops / (f64_peak * 1e12) > step_bytes(spec) / (peak * 1e9):
             roofline = {"bound": "alu", "achieved": flops / (ms_step / 1e3) / 1e12,
                         "peak": f64_peak, "unit": "TFLOP/s",

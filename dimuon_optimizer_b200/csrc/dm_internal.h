@@ -249,6 +249,8 @@ struct ThinParams {
   int conditioned;
   int nesterov;
   int ns_steps;
+  int split;              // r = 32 staged passes: Gram and apply sums on bf16 tensor
+                          // cores with hi / lo split operands (bf16 tensor-core mode)
   float mu, lr, decay, eps;
   float coef[64][3];      // (a_k, b_k, c_k) of Newton-Schulz iteration k < ns_steps
   int* status;

@@ -38,6 +38,40 @@ __device__ __forceinline__ void dmma(double& d0, double& d1, double a, double b)
                : "d"(a), "d"(b));
 }
 
+// Two fp32 values as bf16 pairs hi = RNE(x) and lo = RNE(x - hi): hi + lo
+// carries x to about 2^-17 relative (x - hi is exact in fp32), so a product
+// of two split operands taken as hi hi + hi lo + lo hi has an error of about
+// 2^-16 relative per term (the dropped lo lo term and the two roundings).
+// The first value goes to the low half, the k-slot order of the fragments.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// D (16x8, fp32) += A (16x16, bf16) * B (16x8, bf16).  Lane l = 4g + t holds
+// A rows g, g + 8 at k slots 2t, 2t + 1 (a[0], a[1]) and 2t + 8, 2t + 9
+// (a[2], a[3]); B column g at k slots 2t, 2t + 1 (b0) and 2t + 8, 2t + 9
+// (b1); D rows g (d[0], d[1]) and g + 8 (d[2], d[3]) at columns 2t, 2t + 1.
+__device__ __forceinline__ void hmma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D += A B for split operands: the small cross terms first, then hi hi.
+__device__ __forceinline__ void hmma_split(float (&d)[4], const uint32_t (&ah)[4],
+                                           const uint32_t (&al)[4], const uint32_t (&bh)[2],
+                                           const uint32_t (&bl)[2]) {
+  hmma16816(d, al, bh[0], bh[1]);
+  hmma16816(d, ah, bl[0], bl[1]);
+  hmma16816(d, ah, bh[0], bh[1]);
+}
+
 // C_j^2 = (e_j / mean(e) + eps)^(-1/2); the same expression in every launch.
 __device__ __forceinline__ float col_weight(float e, float inv_mean, float eps) {
   return rsqrtf(__fmaf_rn(e, inv_mean, eps));

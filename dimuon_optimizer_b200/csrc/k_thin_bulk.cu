@@ -579,7 +579,158 @@ __device__ __forceinline__ void gram_step_small(GramAcc<RP>& acc, const TM* Ms, 
   }
 }
 
-template <int RP, typename TG, typename TM>
+// ---------------------------------------------------------------------------
+// Split bf16 tensor-core sums (RP >= 16, bf16 tensor-core mode).  S_1 and S_2
+// are Y Y^T products (K = long-side columns): m16n8k16 tiles with fp32
+// accumulators, each operand split into bf16 hi + lo (three products per
+// tile).  Only the tiles meeting the upper triangle are formed: 16-row tile
+// mt against 8-column tile nt >= 2 mt.
+// ---------------------------------------------------------------------------
+template <int RP>
+struct SCfg {
+  static constexpr int NB = RP / 8;                      // 8-row blocks
+  static constexpr int MT = RP / 16;                     // 16-row tiles
+  static constexpr int NT = MT * NB - MT * (MT - 1);     // upper tiles
+};
+
+template <int RP>
+struct SplitGramAcc {
+  float s1[SCfg<RP>::NT][4];
+  float s2[SCfg<RP>::NT][4];
+  float er[SCfg<RP>::NB];
+};
+
+template <int RP, bool SP>
+struct GramAccOf {
+  using T = GramAcc<RP>;
+};
+template <int RP>
+struct GramAccOf<RP, true> {
+  using T = SplitGramAcc<RP>;
+};
+
+// 16 long-side columns c .. c + 15.  Lane (g, t) holds rows g + 8 b of the
+// columns at k slots q = 0..3, i.e. c + 2t, c + 2t + 1, c + 2t + 8,
+// c + 2t + 9 (the A and the B fragments of the m16n8k16 product use the same
+// values).  FULL = false predicates the columns against c1.
+template <int RP, typename TG, typename TM, bool TALL, bool ON, bool NEST, bool FULL>
+__device__ __forceinline__ void gram_step_split(SplitGramAcc<RP>& acc, const TM* Ms, const TG* Gs,
+                                                const double* wrow, TM* Mg, int64_t n, int cs, int c,
+                                                int c1, float mu, int g, int t) {
+  using L = GramBulk<RP, TG, TM>;
+  constexpr int NB = SCfg<RP>::NB, MT = SCfg<RP>::MT;
+  const int off[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+  bool okc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) okc[q] = FULL || c + off[q] < c1;
+  float mv[NB][4], gv[NB][4];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if constexpr (!TALL && FULL) {
+      const TM* pm = Ms + (g + 8 * b) * L::PM + cs + 2 * t;
+      const TG* pg = Gs + (g + 8 * b) * L::PG + cs + 2 * t;
+      El<TM>::ld2(pm, mv[b][0], mv[b][1]);
+      El<TM>::ld2(pm + 8, mv[b][2], mv[b][3]);
+      El<TG>::ld2(pg, gv[b][0], gv[b][1]);
+      El<TG>::ld2(pg + 8, gv[b][2], gv[b][3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int om = TALL ? (cs + off[q]) * RP + g + 8 * b : (g + 8 * b) * L::PM + cs + off[q];
+        const int og = TALL ? om : (g + 8 * b) * L::PG + cs + off[q];
+        mv[b][q] = okc[q] ? El<TM>::ld1(Ms + om) : 0.f;
+        gv[b][q] = okc[q] ? El<TG>::ld1(Gs + og) : 0.f;
+      }
+    }
+  }
+  float bx[NB][4];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float m = momentum_value(mu, mv[b][q], gv[b][q], El<TM>::DT);
+      mv[b][q] = m;
+      bx[b][q] = NEST ? fmaf(mu, m, gv[b][q]) : m;
+      acc.er[b] = fmaf(m, m, acc.er[b]);
+    }
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if constexpr (!TALL && FULL) {
+      TM* dst = Mg + (int64_t)(g + 8 * b) * n + c + 2 * t;
+      El<TM>::st2(dst, mv[b][0], mv[b][1]);
+      El<TM>::st2(dst + 8, mv[b][2], mv[b][3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (okc[q])
+          El<TM>::st1(Mg + (TALL ? (int64_t)(c + off[q]) * RP + g + 8 * b
+                                 : (int64_t)(g + 8 * b) * n + c + off[q]),
+                      mv[b][q]);
+    }
+  }
+  // A fragments of the 16-row tiles (rows 16 mt + g, + 8)
+  uint32_t ah[MT][4], al[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    split_bf16x2(bx[2 * mt][0], bx[2 * mt][1], ah[mt][0], al[mt][0]);
+    split_bf16x2(bx[2 * mt + 1][0], bx[2 * mt + 1][1], ah[mt][1], al[mt][1]);
+    split_bf16x2(bx[2 * mt][2], bx[2 * mt][3], ah[mt][2], al[mt][2]);
+    split_bf16x2(bx[2 * mt + 1][2], bx[2 * mt + 1][3], ah[mt][3], al[mt][3]);
+  }
+  // B fragments of the 8-column tiles: C^2-weighted (S_1) and C^4-weighted
+  // (S_2) rows 8 nt + g; unweighted, they are halves of the A fragments
+  uint32_t b1h[NB][2], b1l[NB][2], b2h[NB][2], b2l[NB][2];
+  if constexpr (ON) {
+    float w[4], w2[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      w[q] = (float)wrow[off[q]];
+      w2[q] = (float)wrow[L::NCOL + off[q]];
+    }
+#pragma unroll
+    for (int nt = 0; nt < NB; ++nt) {
+      split_bf16x2(w[0] * bx[nt][0], w[1] * bx[nt][1], b1h[nt][0], b1l[nt][0]);
+      split_bf16x2(w[2] * bx[nt][2], w[3] * bx[nt][3], b1h[nt][1], b1l[nt][1]);
+      split_bf16x2(w2[0] * bx[nt][0], w2[1] * bx[nt][1], b2h[nt][0], b2l[nt][0]);
+      split_bf16x2(w2[2] * bx[nt][2], w2[3] * bx[nt][3], b2h[nt][1], b2l[nt][1]);
+    }
+  } else {
+#pragma unroll
+    for (int nt = 0; nt < NB; ++nt) {
+      const int h = nt & 1;
+      b1h[nt][0] = ah[nt >> 1][h];
+      b1l[nt][0] = al[nt >> 1][h];
+      b1h[nt][1] = ah[nt >> 1][2 + h];
+      b1l[nt][1] = al[nt >> 1][2 + h];
+    }
+  }
+  int ti = 0;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 2 * mt; nt < NB; ++nt, ++ti) {
+      hmma_split(acc.s1[ti], ah[mt], al[mt], b1h[nt], b1l[nt]);
+      if constexpr (ON) hmma_split(acc.s2[ti], ah[mt], al[mt], b2h[nt], b2l[nt]);
+    }
+}
+
+template <int RP, typename TG, typename TM, bool TALL, bool ON, bool NEST>
+__device__ __forceinline__ void gram_stage_split(SplitGramAcc<RP>& acc, const TM* Ms, const TG* Gs,
+                                                 const double* wmine, TM* Mg, int64_t n, int c0,
+                                                 int c1, float mu, int warp, int g, int t) {
+  constexpr int CW = GramBulk<RP, TG, TM>::CW;
+  int k = 0;
+  for (int c = c0 + 16 * warp; c < c1; c += 16 * CW, ++k) {
+    if (c + 16 <= c1)
+      gram_step_split<RP, TG, TM, TALL, ON, NEST, true>(acc, Ms, Gs, wmine + 16 * k, Mg, n, c - c0, c,
+                                                        c1, mu, g, t);
+    else
+      gram_step_split<RP, TG, TM, TALL, ON, NEST, false>(acc, Ms, Gs, wmine + 16 * k, Mg, n, c - c0,
+                                                         c, c1, mu, g, t);
+  }
+}
+
+template <int RP, typename TG, typename TM, bool SP>
 __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>::MINB)
     thin_gram_bulk(const __grid_constant__ ThinParams p) {
   using L = GramBulk<RP, TG, TM>;
@@ -623,7 +774,7 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
   const float mu = p.mu, eps = p.eps;
   const bool nest = p.nesterov != 0;
   const int g = lane >> 2, t = lane & 3;
-  GramAcc<RP> acc;
+  typename GramAccOf<RP, SP>::T acc;
   int stage = 0;
   uint32_t ph = 0, nred = 0;
   for (;;) {
@@ -643,15 +794,37 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
     const TG* Gs = reinterpret_cast<const TG*>(base + L::OFF_G);
     const float* Es = reinterpret_cast<const float*>(base + L::OFF_E);
     if (first) {
+      if constexpr (SP) {
 #pragma unroll
-      for (int a = 0; a < (Cf::MMA ? Cf::NUB : RP); ++a)
+        for (int a = 0; a < SCfg<RP>::NT; ++a)
 #pragma unroll
-        for (int b = 0; b < (Cf::MMA ? 2 : RP); ++b) acc.s1[a][b] = acc.s2[a][b] = 0.0;
+          for (int b = 0; b < 4; ++b) acc.s1[a][b] = acc.s2[a][b] = 0.f;
 #pragma unroll
-      for (int a = 0; a < (Cf::MMA ? Cf::NB : RP); ++a) acc.er[a] = 0.f;
+        for (int a = 0; a < SCfg<RP>::NB; ++a) acc.er[a] = 0.f;
+      } else {
+#pragma unroll
+        for (int a = 0; a < (Cf::MMA ? Cf::NUB : RP); ++a)
+#pragma unroll
+          for (int b = 0; b < (Cf::MMA ? 2 : RP); ++b) acc.s1[a][b] = acc.s2[a][b] = 0.0;
+#pragma unroll
+        for (int a = 0; a < (Cf::MMA ? Cf::NB : RP); ++a) acc.er[a] = 0.f;
+      }
     }
 
-    if constexpr (Cf::MMA) {
+    if constexpr (SP) {
+      double* wmine = wsm + warp * 2 * L::NCOL;
+      if (on) stage_weights<16, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
+#define DM_GRAM_SPLIT(TALL_, ON_, NEST_) \
+  gram_stage_split<RP, TG, TM, TALL_, ON_, NEST_>(acc, Ms, Gs, wmine, Mg, n, c0, c1, mu, warp, g, t)
+      if (tall) {
+        if (on) { if (nest) DM_GRAM_SPLIT(true, true, true); else DM_GRAM_SPLIT(true, true, false); }
+        else { if (nest) DM_GRAM_SPLIT(true, false, true); else DM_GRAM_SPLIT(true, false, false); }
+      } else {
+        if (on) { if (nest) DM_GRAM_SPLIT(false, true, true); else DM_GRAM_SPLIT(false, true, false); }
+        else { if (nest) DM_GRAM_SPLIT(false, false, true); else DM_GRAM_SPLIT(false, false, false); }
+      }
+#undef DM_GRAM_SPLIT
+    } else if constexpr (Cf::MMA) {
       double* wmine = wsm + warp * 2 * L::NCOL;
       if (on) stage_weights<16, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
       int k = 0;
@@ -702,7 +875,35 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
       // redr before the partial buffers are written again
       if (!wait_phase(redr, (nred & 1u) ^ 1u, abort, p.status)) break;
       double* mine = red_s + warp * 2 * Cf::PART;
-      if constexpr (Cf::MMA) {
+      if constexpr (SP) {
+        // tile (mt, nt) holds 8x8 blocks (2 mt, nt) and (2 mt + 1, nt) in the
+        // DMMA accumulator layout (row g, columns 2t, 2t + 1); the upper ones
+        // go to their packed slot
+        constexpr int NB = SCfg<RP>::NB;
+        int ti = 0;
+#pragma unroll
+        for (int mt = 0; mt < SCfg<RP>::MT; ++mt)
+#pragma unroll
+          for (int nt = 2 * mt; nt < NB; ++nt, ++ti)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int bi = 2 * mt + hh, bj = nt;
+              if (bi > bj) continue;
+              const int ub = bi * NB - bi * (bi - 1) / 2 + (bj - bi);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                mine[ub * 64 + g * 8 + 2 * t + h] = (double)acc.s1[ti][2 * hh + h];
+                mine[Cf::PART + ub * 64 + g * 8 + 2 * t + h] = (double)acc.s2[ti][2 * hh + h];
+              }
+            }
+#pragma unroll
+        for (int blk = 0; blk < NB; ++blk) {
+          float e = acc.er[blk];
+          e += __shfl_xor_sync(0xffffffffu, e, 1);
+          e += __shfl_xor_sync(0xffffffffu, e, 2);
+          if (t == 0) red_e[warp * RP + g + 8 * blk] = e;
+        }
+      } else if constexpr (Cf::MMA) {
         constexpr int NB = Cf::NB, NUB = Cf::NUB;
 #pragma unroll
         for (int ub = 0; ub < NUB; ++ub)
@@ -998,6 +1199,164 @@ __device__ __forceinline__ void apply_step_small(const TM* Ms, const TG* Gs, con
   if constexpr (COND) El<float>::st4(ecg + c, ce);
 }
 
+// ---------------------------------------------------------------------------
+// Split bf16 tensor-core apply (RP >= 16, bf16 tensor-core mode): O = T X
+// with X = C^2 B, K = the short side, m16n8k16 tiles, T and X split into
+// bf16 hi + lo.  T's fragments stay in registers while the factor is the
+// same.
+// ---------------------------------------------------------------------------
+template <int RP>
+struct SplitT {
+  static constexpr int MT = RP / 16, KT = RP / 16;
+  uint32_t h[MT][KT][4], l[MT][KT][4];
+};
+
+// T is stored in the DMMA fragment order: T[i][k] at
+// ((i / 8) (RP / 4) + k / 4) 32 + (i % 8) 4 + k % 4.
+template <int RP>
+__device__ __forceinline__ void load_split_t(SplitT<RP>& f, const double* Tg, int g, int t) {
+  constexpr int KB = RP / 4;
+  auto tv = [&](int i, int k) {
+    return (float)__ldg(Tg + ((i >> 3) * KB + (k >> 2)) * 32 + (i & 7) * 4 + (k & 3));
+  };
+#pragma unroll
+  for (int mt = 0; mt < SplitT<RP>::MT; ++mt)
+#pragma unroll
+    for (int kt = 0; kt < SplitT<RP>::KT; ++kt) {
+      const int r0 = 16 * mt + g, r1 = r0 + 8, k0 = 16 * kt + 2 * t, k1 = k0 + 8;
+      split_bf16x2(tv(r0, k0), tv(r0, k0 + 1), f.h[mt][kt][0], f.l[mt][kt][0]);
+      split_bf16x2(tv(r1, k0), tv(r1, k0 + 1), f.h[mt][kt][1], f.l[mt][kt][1]);
+      split_bf16x2(tv(r0, k1), tv(r0, k1 + 1), f.h[mt][kt][2], f.l[mt][kt][2]);
+      split_bf16x2(tv(r1, k1), tv(r1, k1 + 1), f.h[mt][kt][3], f.l[mt][kt][3]);
+    }
+}
+
+// 32 long-side columns c .. c + 31 as four 8-column tiles.  For tile nt,
+// lane (g, t) supplies column c + 8 nt + g at rows 16 kt + {2t, 2t + 1,
+// 2t + 8, 2t + 9} (the B fragment) and receives O rows 16 mt + g, + 8 at
+// columns c + 8 nt + 2t, + 1.
+template <int RP, typename TG, typename TM, typename TW, bool TALL, bool ON, bool COND, bool FULL,
+          bool NEST>
+__device__ __forceinline__ void apply_step_split(const SplitT<RP>& tf, const TM* Ms, const TG* Gs,
+                                                 const TW* Ws, const double* wrow, TW* Wg, float* Ug,
+                                                 float* ecg, int64_t n, int cs, int c, int c1,
+                                                 float mu, float lr, float decay, bool zero, int g,
+                                                 int t) {
+  using L = ApplyBulk<RP, TG, TM, TW>;
+  constexpr int MT = SplitT<RP>::MT, KT = SplitT<RP>::KT;
+  const int off[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const int jl = 8 * nt + g;
+    const bool okj = FULL || c + jl < c1;
+    const float w = ON ? (float)wrow[jl] : 1.f;  // zero past c1
+    uint32_t bh[KT][2], bl[KT][2];
+    float sq = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < KT; ++kt) {
+      float mv[4], gv[4];
+      if constexpr (TALL) {
+        const int o = (cs + jl) * RP + 16 * kt + 2 * t;
+        if (okj) {
+          El<TM>::ld2(Ms + o, mv[0], mv[1]);
+          El<TM>::ld2(Ms + o + 8, mv[2], mv[3]);
+          if (NEST) {
+            El<TG>::ld2(Gs + o, gv[0], gv[1]);
+            El<TG>::ld2(Gs + o + 8, gv[2], gv[3]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mv[q] = gv[q] = 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k = 16 * kt + off[q];
+          mv[q] = okj ? El<TM>::ld1(Ms + k * L::PM + cs + jl) : 0.f;
+          gv[q] = (NEST && okj) ? El<TG>::ld1(Gs + k * L::PG + cs + jl) : 0.f;
+        }
+      }
+      float x[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if constexpr (COND) sq = fmaf(mv[q], mv[q], sq);
+        const float bv = NEST ? fmaf(mu, mv[q], gv[q]) : mv[q];
+        x[q] = ON ? w * bv : bv;
+      }
+      split_bf16x2(x[0], x[1], bh[kt][0], bl[kt][0]);
+      split_bf16x2(x[2], x[3], bh[kt][1], bl[kt][1]);
+    }
+    float d[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      d[mt][0] = d[mt][1] = d[mt][2] = d[mt][3] = 0.f;
+#pragma unroll
+      for (int kt = 0; kt < KT; ++kt) hmma_split(d[mt], tf.h[mt][kt], tf.l[mt][kt], bh[kt], bl[kt]);
+    }
+    if constexpr (COND) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+      if (t == 0 && okj) ecg[c + jl] = sq;
+    }
+    const int col = 8 * nt + 2 * t;  // this lane's first output column
+    const bool ok0 = FULL || c + col < c1, ok1 = FULL || c + col + 1 < c1;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int row = 16 * mt + g + 8 * hh;
+        const float o0 = zero ? 0.f : d[mt][2 * hh], o1 = zero ? 0.f : d[mt][2 * hh + 1];
+        if constexpr (!TALL) {
+          if (ok0 && ok1) {
+            float w0, w1;
+            El<TW>::ld2(Ws + row * L::PW + cs + col, w0, w1);
+            El<TW>::st2(Wg + (int64_t)row * n + c + col, decay * w0 - lr * o0, decay * w1 - lr * o1);
+            if (Ug) El<float>::st2(Ug + (int64_t)row * n + c + col, o0, o1);
+          } else if (ok0) {
+            const float w0 = El<TW>::ld1(Ws + row * L::PW + cs + col);
+            El<TW>::st1(Wg + (int64_t)row * n + c + col, decay * w0 - lr * o0);
+            if (Ug) Ug[(int64_t)row * n + c + col] = o0;
+          }
+        } else {
+          if (ok0) {
+            const float w0 = El<TW>::ld1(Ws + (cs + col) * RP + row);
+            El<TW>::st1(Wg + (int64_t)(c + col) * RP + row, decay * w0 - lr * o0);
+            if (Ug) Ug[(int64_t)(c + col) * RP + row] = o0;
+          }
+          if (ok1) {
+            const float w1 = El<TW>::ld1(Ws + (cs + col + 1) * RP + row);
+            El<TW>::st1(Wg + (int64_t)(c + col + 1) * RP + row, decay * w1 - lr * o1);
+            if (Ug) Ug[(int64_t)(c + col + 1) * RP + row] = o1;
+          }
+        }
+      }
+  }
+}
+
+template <int RP, typename TG, typename TM, typename TW, bool TALL, bool ON, bool COND, bool NEST>
+__device__ __forceinline__ void apply_stage_split(const SplitT<RP>& tf, const TM* Ms, const TG* Gs,
+                                                  const TW* Ws, const float* Es, double* wmine,
+                                                  TW* Wg, float* Ug, float* ecg, int64_t n, int c0,
+                                                  int c1, float mu, float lr, float decay,
+                                                  float inv_mc, float eps, bool zero, int warp,
+                                                  int lane) {
+  using L = ApplyBulk<RP, TG, TM, TW>;
+  constexpr int CW = L::CW;
+  const int g = lane >> 2, t = lane & 3;
+  if (ON) stage_weights<32, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
+  int k = 0;
+  for (int c = c0 + 32 * warp; c < c1; c += 32 * CW, ++k) {
+    if (c + 32 <= c1)
+      apply_step_split<RP, TG, TM, TW, TALL, ON, COND, true, NEST>(tf, Ms, Gs, Ws, wmine + 32 * k, Wg,
+                                                                   Ug, ecg, n, c - c0, c, c1, mu, lr,
+                                                                   decay, zero, g, t);
+    else
+      apply_step_split<RP, TG, TM, TW, TALL, ON, COND, false, NEST>(tf, Ms, Gs, Ws, wmine + 32 * k, Wg,
+                                                                    Ug, ecg, n, c - c0, c, c1, mu, lr,
+                                                                    decay, zero, g, t);
+  }
+}
+
 template <int RP, typename TG, typename TM, typename TW, bool TALL, bool ON, bool COND, bool NEST>
 __device__ __forceinline__ void apply_stage(const TM* Ms, const TG* Gs, const TW* Ws, const float* Es,
                                             double* wmine, const double* Tg, TW* Wg, float* Ug,
@@ -1027,7 +1386,16 @@ __device__ __forceinline__ void apply_stage(const TM* Ms, const TG* Gs, const TW
   }
 }
 
-template <int RP, typename TG, typename TM, typename TW>
+template <int RP, bool SP>
+struct SplitTOf {
+  struct T {};
+};
+template <int RP>
+struct SplitTOf<RP, true> {
+  using T = SplitT<RP>;
+};
+
+template <int RP, typename TG, typename TM, typename TW, bool SP>
 __global__ void __launch_bounds__(ApplyBulk<RP, TG, TM, TW>::BT, ApplyBulk<RP, TG, TM, TW>::MINB)
     thin_apply_bulk(const __grid_constant__ ThinParams p) {
   using L = ApplyBulk<RP, TG, TM, TW>;
@@ -1065,6 +1433,8 @@ __global__ void __launch_bounds__(ApplyBulk<RP, TG, TM, TW>::BT, ApplyBulk<RP, T
   const bool nest = p.nesterov != 0;
   int stage = 0;
   uint32_t ph = 0;
+  typename SplitTOf<RP, SP>::T tfr;  // split T fragments of factor tf_f
+  int tf_f = -1;
   for (;;) {
     if (!wait_phase(&full[stage], ph, abort, p.status)) break;
     const StageInfo& si = info[stage];
@@ -1084,9 +1454,24 @@ __global__ void __launch_bounds__(ApplyBulk<RP, TG, TM, TW>::BT, ApplyBulk<RP, T
     const float* Es = reinterpret_cast<const float*>(base + L::OFF_E);
     const TG* Gs = reinterpret_cast<const TG*>(base + L::OFF_G);
     const double* Tg = p.T + (size_t)si.f * RP * RP;
+    if constexpr (SP) {
+      if (si.f != tf_f) {
+        load_split_t<RP>(tfr, Tg, lane >> 2, lane & 3);
+        tf_f = si.f;
+      }
+    }
 #define DM_APPLY_STAGE(TALL_, ON_, COND_)                                                              \
   do {                                                                                                \
-    if (nest)                                                                                         \
+    if constexpr (SP) {                                                                               \
+      if (nest)                                                                                       \
+        apply_stage_split<RP, TG, TM, TW, TALL_, ON_, COND_, true>(                                   \
+            tfr, Ms, Gs, Ws, Es, wsm + warp * 2 * L::NCOL, Wg, Ug, ecg, n, c0, c1, mu, lr, decay,     \
+            inv_mc, eps, zero, warp, lane);                                                           \
+      else                                                                                            \
+        apply_stage_split<RP, TG, TM, TW, TALL_, ON_, COND_, false>(                                  \
+            tfr, Ms, Gs, Ws, Es, wsm + warp * 2 * L::NCOL, Wg, Ug, ecg, n, c0, c1, mu, lr, decay,     \
+            inv_mc, eps, zero, warp, lane);                                                           \
+    } else if (nest)                                                                                  \
       apply_stage<RP, TG, TM, TW, TALL_, ON_, COND_, true>(Ms, Gs, Ws, Es, wsm + warp * 2 * L::NCOL, \
                                                            Tg, Wg, Ug, ecg, n, c0, c1, mu, lr, decay, \
                                                            inv_mc, eps, zero, warp, lane);            \
@@ -1123,43 +1508,51 @@ int resident(K kernel, int threads, int smem) {
   return occ;
 }
 
-template <int RP, typename TG, typename TM, typename TW>
-cudaError_t launch_bulk_rp(ThinParams& p, int nsm, cudaStream_t st) {
+template <int RP, typename TG, typename TM, typename TW, bool SP>
+cudaError_t launch_bulk_sp(ThinParams& p, int nsm, cudaStream_t st) {
   using LG = GramBulk<RP, TG, TM>;
   using LA = ApplyBulk<RP, TG, TM, TW>;
   static DeviceOnce once;
   static int occ_g[MAX_DEVICES], occ_a[MAX_DEVICES][2];
   int dev = 0;
   cudaError_t e = device_once(once, &dev, [](int d) {
-    cudaError_t e = cudaFuncSetAttribute(thin_gram_bulk<RP, TG, TM>,
+    cudaError_t e = cudaFuncSetAttribute(thin_gram_bulk<RP, TG, TM, SP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, LG::SMEM);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(thin_apply_bulk<RP, TG, TM, TW>,
+      e = cudaFuncSetAttribute(thin_apply_bulk<RP, TG, TM, TW, SP>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, LA::smem(true));
     // shared memory over L1 for the staging rings
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(thin_gram_bulk<RP, TG, TM>,
+      e = cudaFuncSetAttribute(thin_gram_bulk<RP, TG, TM, SP>,
                                cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(thin_apply_bulk<RP, TG, TM, TW>,
+      e = cudaFuncSetAttribute(thin_apply_bulk<RP, TG, TM, TW, SP>,
                                cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    occ_g[d] = resident(thin_gram_bulk<RP, TG, TM>, LG::BT, LG::SMEM);
-    occ_a[d][0] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(false));
-    occ_a[d][1] = resident(thin_apply_bulk<RP, TG, TM, TW>, LA::BT, LA::smem(true));
+    occ_g[d] = resident(thin_gram_bulk<RP, TG, TM, SP>, LG::BT, LG::SMEM);
+    occ_a[d][0] = resident(thin_apply_bulk<RP, TG, TM, TW, SP>, LA::BT, LA::smem(false));
+    occ_a[d][1] = resident(thin_apply_bulk<RP, TG, TM, TW, SP>, LA::BT, LA::smem(true));
     return cudaSuccess;
   });
   if (e != cudaSuccess) return e;
   const bool nest = p.nesterov != 0;
   p.grid_gram = std::min(p.units, nsm * occ_g[dev]);
   p.grid_apply = std::min(p.units, nsm * occ_a[dev][nest ? 1 : 0]);
-  thin_gram_bulk<RP, TG, TM><<<p.grid_gram, LG::BT, LG::SMEM, st>>>(p);
+  thin_gram_bulk<RP, TG, TM, SP><<<p.grid_gram, LG::BT, LG::SMEM, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_thin_iterate(p, st);
   if (e != cudaSuccess) return e;
-  thin_apply_bulk<RP, TG, TM, TW><<<p.grid_apply, LA::BT, LA::smem(nest), st>>>(p);
+  thin_apply_bulk<RP, TG, TM, TW, SP><<<p.grid_apply, LA::BT, LA::smem(nest), st>>>(p);
   return cudaGetLastError();
+}
+
+template <int RP, typename TG, typename TM, typename TW>
+cudaError_t launch_bulk_rp(ThinParams& p, int nsm, cudaStream_t st) {
+  if constexpr (RP == 32) {
+    if (p.split) return launch_bulk_sp<RP, TG, TM, TW, true>(p, nsm, st);
+  }
+  return launch_bulk_sp<RP, TG, TM, TW, false>(p, nsm, st);
 }
 
 template <typename TG, typename TM, typename TW>

@@ -14,6 +14,23 @@ import oracle as orc
 TOL_FP32 = 1e-5      # relative Frobenius error of O_t, fp32 mode / thin path
 TOL_BF16 = 3e-2      # relative Frobenius error of O_t, bf16 tensor-core mode
 TOL_SV = 0.05        # singular values of O_t / kappa
+# staged r = 32 thin factors in bf16 tensor-core mode: Gram and apply sums on
+# bf16 tensor cores with hi / lo split operands (about 2^-16 relative per
+# term, fp32 accumulation) instead of fp64.  The Gram route squares the
+# factor's condition number, so the error grows with it: a few 1e-6 on
+# Gaussian factors (1e-4 bound here), up to 1.2e-3 on the first, unconditioned
+# step of the LoRA batch whose column scales span 1e-2 .. 1e6 (5e-3 bound);
+# both well inside the bf16 mode's 3e-2.
+TOL_THIN_SPLIT = 1e-4
+TOL_THIN_SPLIT_ILL = 5e-3
+
+
+def thin_tol(precision_bf16, split_tol=TOL_THIN_SPLIT):
+    """Tolerance of O_t for a thin-factor group: fp64 sums everywhere except
+    the r = 32 factors in bf16 tensor-core mode."""
+    if not precision_bf16:
+        return TOL_FP32
+    return lambda shape: split_tol if min(shape) == 32 else TOL_FP32
 
 
 def tdtype(code):
@@ -129,7 +146,8 @@ def step_and_compare(grp: Group, grads_host, hp, o_tol, *, ws=None, check_sv=Tru
         # the update
         e = rel_fro(Og, res.O)
         rep.o_err.append(e)
-        assert e <= o_tol, (i, grp.shapes[i], e)
+        tol = o_tol(grp.shapes[i]) if callable(o_tol) else o_tol
+        assert e <= tol, (i, grp.shapes[i], e)
         # the apply: W_t = (1 - lr wd) W_{t-1} - lr O_t with the GPU's own O_t
         decay = np.float32(1.0) - np.float32(hp.lr) * np.float32(hp.weight_decay)
         Wexp = store_round_np(float(decay) * W0 - float(np.float32(hp.lr)) * Og, grp.wdt)

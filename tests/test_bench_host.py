@@ -153,8 +153,11 @@ def test_thin_fp64_flops():
     assert bench.thin_fp64_flops(spec) == 2 * 100 * per_col
     spec["cond"] = False
     assert bench.thin_fp64_flops(spec) == 2 * 100 * 2 * (36 + 64)
-    # the LoRA rank-32 batch is bound by fp64 arithmetic, rank 8 by HBM
+    # the LoRA rank-32 batch is bound by fp64 arithmetic in fp32 mode, rank 8 by
+    # HBM; in bf16 mode the rank-32 sums run on bf16 tensor cores (no fp64)
     r32, r8 = bench.workload_spec("lora_r32"), bench.workload_spec("lora_r8")
     f64 = 148 * bench.FP64_FMA_PER_SM_CLK * 2 * 1965e6
     assert bench.thin_fp64_flops(r32) / f64 > bench.step_bytes(r32) / 6.5e12
     assert bench.thin_fp64_flops(r8) / f64 < bench.step_bytes(r8) / 6.5e12
+    assert bench.thin_fp64_flops(r32, split_r32=True) == 0.0
+    assert bench.thin_fp64_flops(r8, split_r32=True) == bench.thin_fp64_flops(r8)
