@@ -345,20 +345,26 @@ __device__ __forceinline__ void stage_weights(double* wmine, const float* Es, in
 // ===========================================================================
 // thin_gram_bulk: momentum, Gram partials, short-side energy partials
 // ===========================================================================
-template <int RP, typename TG, typename TM>
+// SP: the split bf16 tensor-core sums (r = 32, bf16 tensor-core mode), whose
+// fp32 accumulators need fewer registers and half the reduction space: six
+// consumer warps (one 16-column step each per stage of 96 columns) and three
+// stages, two CTAs per SM.
+template <int RP, typename TG, typename TM, bool SP = false>
 struct GramBulk {
-  static constexpr int CW = RP == 32 ? 4 : 8;  // consumer warps
-  static constexpr int NP = 2;                 // producer warps
+  static constexpr int CW = SP ? 6 : RP == 32 ? 4 : 8;  // consumer warps
+  static constexpr int NP = 2;                          // producer warps
   static constexpr int BT = 32 * (CW + NP);
-  static constexpr int MINB = RP == 8 || RP == 16 ? 3 : RP == 32 ? 2 : 1;  // resident CTAs
-  static constexpr int CH = RP <= 4 ? 1024 : RP == 8 ? 256 : RP == 16 ? 128 : 64;
-  static constexpr int NS = 4;
+  static constexpr int MINB = SP ? 2 : RP == 8 || RP == 16 ? 3 : RP == 32 ? 2 : 1;  // resident CTAs
+  static constexpr int CH = SP ? 96 : RP <= 4 ? 1024 : RP == 8 ? 256 : RP == 16 ? 128 : 64;
+  static constexpr int NS = SP ? 3 : 4;
   static constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH);
   static constexpr int OFF_G = opnd_bytes<TM>(RP, CH);
   static constexpr int OFF_E = OFF_G + opnd_bytes<TG>(RP, CH);
   static constexpr int STAGE_BYTES = (OFF_E + CH * 4 + 127) / 128 * 128;
-  // per-warp Gram and energy partials for the reduction at a run's end
-  static constexpr int RED_BYTES = CW * 2 * TCfg<RP>::PART * 8 + CW * RP * 4;
+  // per-warp Gram (fp64, or fp32 under SP) and energy partials for the
+  // reduction at a run's end
+  static constexpr int RED_S_BYTES = CW * 2 * TCfg<RP>::PART * (SP ? 4 : 8);
+  static constexpr int RED_BYTES = RED_S_BYTES + CW * RP * 4;
   static constexpr int NCOL = TCfg<RP>::MMA ? CH / CW : 0;  // columns of one consumer warp per stage
   static constexpr int WS_BYTES = CW * 2 * NCOL * 8;
   static constexpr int SMEM = NS * STAGE_BYTES + NS * (int)sizeof(StageInfo) + (2 * NS + 2) * 8 + 16 +
@@ -609,16 +615,64 @@ struct GramAccOf<RP, true> {
   using T = SplitGramAcc<RP>;
 };
 
+// Column factors of the split Gram sums, once per column and stage: entry
+// k SW + o of the warp's k-th step holds C = (C^2)^(1/2) and C^2 of that
+// column (zero past c1), so S_1 = sum (C b)(C b)^T and S_2 = sum (C^2 b)(C^2 b)^T.
+template <int CW, int NCOL>
+__device__ __forceinline__ void stage_col_factors(float* wmine, const float* Es, int c0, int c1,
+                                                  int warp, int lane, float inv_mc, float eps) {
+  for (int idx = lane; idx < NCOL; idx += 32) {
+    const int k = idx / 16, o = idx % 16;
+    const int col = c0 + 16 * (warp + CW * k) + o;
+    const float w = col < c1 ? col_weight(Es[col - c0], inv_mc, eps) : 0.f;
+    wmine[idx] = sqrtf(w);
+    wmine[NCOL + idx] = w;
+  }
+  __syncwarp();
+}
+
+// A (= B) fragments of one 16-row tile of the split products: rows
+// 16 mt + g (+ 8) at the lane's four k slots.
+template <int NB>
+__device__ __forceinline__ void split_rows(const float (&v)[NB][4], int mt, uint32_t (&h)[4],
+                                           uint32_t (&l)[4]) {
+  split_bf16x2(v[2 * mt][0], v[2 * mt][1], h[0], l[0]);
+  split_bf16x2(v[2 * mt + 1][0], v[2 * mt + 1][1], h[1], l[1]);
+  split_bf16x2(v[2 * mt][2], v[2 * mt][3], h[2], l[2]);
+  split_bf16x2(v[2 * mt + 1][2], v[2 * mt + 1][3], h[3], l[3]);
+}
+
+// S += V V^T over the lane's 16 columns for the upper tiles (mt, nt >= 2 mt):
+// the B fragment of 8-column tile nt is one half of the A fragment of
+// 16-row tile nt / 2.
+template <int RP>
+__device__ __forceinline__ void syrk_split(float (*S)[4], const float (&v)[RP / 8][4]) {
+  constexpr int NB = SCfg<RP>::NB, MT = SCfg<RP>::MT;
+  uint32_t h[MT][4], l[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) split_rows<NB>(v, mt, h[mt], l[mt]);
+  int ti = 0;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 2 * mt; nt < NB; ++nt, ++ti) {
+      const int hn = nt & 1;
+      const uint32_t bh[2] = {h[nt >> 1][hn], h[nt >> 1][2 + hn]};
+      const uint32_t bl[2] = {l[nt >> 1][hn], l[nt >> 1][2 + hn]};
+      hmma_split(S[ti], h[mt], l[mt], bh, bl);
+    }
+}
+
 // 16 long-side columns c .. c + 15.  Lane (g, t) holds rows g + 8 b of the
 // columns at k slots q = 0..3, i.e. c + 2t, c + 2t + 1, c + 2t + 8,
-// c + 2t + 9 (the A and the B fragments of the m16n8k16 product use the same
-// values).  FULL = false predicates the columns against c1.
+// c + 2t + 9 (the A and the B fragments of the m16n8k16 products use the
+// same values).  FULL = false predicates the columns against c1.
 template <int RP, typename TG, typename TM, bool TALL, bool ON, bool NEST, bool FULL>
 __device__ __forceinline__ void gram_step_split(SplitGramAcc<RP>& acc, const TM* Ms, const TG* Gs,
-                                                const double* wrow, TM* Mg, int64_t n, int cs, int c,
+                                                const float* wrow, TM* Mg, int64_t n, int cs, int c,
                                                 int c1, float mu, int g, int t) {
-  using L = GramBulk<RP, TG, TM>;
-  constexpr int NB = SCfg<RP>::NB, MT = SCfg<RP>::MT;
+  using L = GramBulk<RP, TG, TM, true>;
+  constexpr int NB = SCfg<RP>::NB;
   const int off[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
   bool okc[4];
 #pragma unroll
@@ -643,15 +697,14 @@ __device__ __forceinline__ void gram_step_split(SplitGramAcc<RP>& acc, const TM*
       }
     }
   }
-  float bx[NB][4];
 #pragma unroll
   for (int b = 0; b < NB; ++b)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float m = momentum_value(mu, mv[b][q], gv[b][q], El<TM>::DT);
       mv[b][q] = m;
-      bx[b][q] = NEST ? fmaf(mu, m, gv[b][q]) : m;
       acc.er[b] = fmaf(m, m, acc.er[b]);
+      if constexpr (NEST) gv[b][q] = fmaf(mu, m, gv[b][q]);  // B = G + mu M_t
     }
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
@@ -668,57 +721,36 @@ __device__ __forceinline__ void gram_step_split(SplitGramAcc<RP>& acc, const TM*
                       mv[b][q]);
     }
   }
-  // A fragments of the 16-row tiles (rows 16 mt + g, + 8)
-  uint32_t ah[MT][4], al[MT][4];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-    split_bf16x2(bx[2 * mt][0], bx[2 * mt][1], ah[mt][0], al[mt][0]);
-    split_bf16x2(bx[2 * mt + 1][0], bx[2 * mt + 1][1], ah[mt][1], al[mt][1]);
-    split_bf16x2(bx[2 * mt][2], bx[2 * mt][3], ah[mt][2], al[mt][2]);
-    split_bf16x2(bx[2 * mt + 1][2], bx[2 * mt + 1][3], ah[mt][3], al[mt][3]);
-  }
-  // B fragments of the 8-column tiles: C^2-weighted (S_1) and C^4-weighted
-  // (S_2) rows 8 nt + g; unweighted, they are halves of the A fragments
-  uint32_t b1h[NB][2], b1l[NB][2], b2h[NB][2], b2l[NB][2];
+  // the orthogonaliser's input columns b (B_t under Nesterov, else M_t)
+  float (&bx)[NB][4] = NEST ? gv : mv;
   if constexpr (ON) {
-    float w[4], w2[4];
+    float cf[4], c2[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      w[q] = (float)wrow[off[q]];
-      w2[q] = (float)wrow[L::NCOL + off[q]];
+      cf[q] = wrow[off[q]];
+      c2[q] = wrow[L::NCOL + off[q]];
     }
+    float v[NB][4];
 #pragma unroll
-    for (int nt = 0; nt < NB; ++nt) {
-      split_bf16x2(w[0] * bx[nt][0], w[1] * bx[nt][1], b1h[nt][0], b1l[nt][0]);
-      split_bf16x2(w[2] * bx[nt][2], w[3] * bx[nt][3], b1h[nt][1], b1l[nt][1]);
-      split_bf16x2(w2[0] * bx[nt][0], w2[1] * bx[nt][1], b2h[nt][0], b2l[nt][0]);
-      split_bf16x2(w2[2] * bx[nt][2], w2[3] * bx[nt][3], b2h[nt][1], b2l[nt][1]);
-    }
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[b][q] = cf[q] * bx[b][q];
+    syrk_split<RP>(acc.s1, v);
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[b][q] = c2[q] * bx[b][q];
+    syrk_split<RP>(acc.s2, v);
   } else {
-#pragma unroll
-    for (int nt = 0; nt < NB; ++nt) {
-      const int h = nt & 1;
-      b1h[nt][0] = ah[nt >> 1][h];
-      b1l[nt][0] = al[nt >> 1][h];
-      b1h[nt][1] = ah[nt >> 1][2 + h];
-      b1l[nt][1] = al[nt >> 1][2 + h];
-    }
+    syrk_split<RP>(acc.s1, bx);
   }
-  int ti = 0;
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int nt = 2 * mt; nt < NB; ++nt, ++ti) {
-      hmma_split(acc.s1[ti], ah[mt], al[mt], b1h[nt], b1l[nt]);
-      if constexpr (ON) hmma_split(acc.s2[ti], ah[mt], al[mt], b2h[nt], b2l[nt]);
-    }
 }
 
 template <int RP, typename TG, typename TM, bool TALL, bool ON, bool NEST>
 __device__ __forceinline__ void gram_stage_split(SplitGramAcc<RP>& acc, const TM* Ms, const TG* Gs,
-                                                 const double* wmine, TM* Mg, int64_t n, int c0,
+                                                 const float* wmine, TM* Mg, int64_t n, int c0,
                                                  int c1, float mu, int warp, int g, int t) {
-  constexpr int CW = GramBulk<RP, TG, TM>::CW;
+  constexpr int CW = GramBulk<RP, TG, TM, true>::CW;
   int k = 0;
   for (int c = c0 + 16 * warp; c < c1; c += 16 * CW, ++k) {
     if (c + 16 <= c1)
@@ -731,9 +763,9 @@ __device__ __forceinline__ void gram_stage_split(SplitGramAcc<RP>& acc, const TM
 }
 
 template <int RP, typename TG, typename TM, bool SP>
-__global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>::MINB)
+__global__ void __launch_bounds__(GramBulk<RP, TG, TM, SP>::BT, GramBulk<RP, TG, TM, SP>::MINB)
     thin_gram_bulk(const __grid_constant__ ThinParams p) {
-  using L = GramBulk<RP, TG, TM>;
+  using L = GramBulk<RP, TG, TM, SP>;
   using Cf = TCfg<RP>;
   constexpr int CH = L::CH, NS = L::NS, CW = L::CW;
   extern __shared__ uint8_t smem_raw[];
@@ -746,8 +778,10 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
   uint64_t* redf = empty + NS;  // run-end reduction: consumer warps wrote their partials
   uint64_t* redr = redf + 1;    // run-end reduction: consumer warps read the partials
   volatile int* abort = reinterpret_cast<volatile int*>(redr + 1);
-  double* red_s = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(redr + 1) + 16);
-  float* red_e = reinterpret_cast<float*>(red_s + CW * 2 * Cf::PART);
+  uint8_t* red_base = reinterpret_cast<uint8_t*>(redr + 1) + 16;
+  double* red_s = reinterpret_cast<double*>(red_base);  // fp64 partials
+  float* red_sf = reinterpret_cast<float*>(red_base);   // fp32 partials (SP)
+  float* red_e = reinterpret_cast<float*>(red_base + L::RED_S_BYTES);
   double* wsm = reinterpret_cast<double*>(red_e + CW * RP);  // CW * RP is even
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -812,8 +846,8 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
     }
 
     if constexpr (SP) {
-      double* wmine = wsm + warp * 2 * L::NCOL;
-      if (on) stage_weights<16, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
+      float* wmine = reinterpret_cast<float*>(wsm + warp * 2 * L::NCOL);
+      if (on) stage_col_factors<CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
 #define DM_GRAM_SPLIT(TALL_, ON_, NEST_) \
   gram_stage_split<RP, TG, TM, TALL_, ON_, NEST_>(acc, Ms, Gs, wmine, Mg, n, c0, c1, mu, warp, g, t)
       if (tall) {
@@ -875,6 +909,7 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
       // redr before the partial buffers are written again
       if (!wait_phase(redr, (nred & 1u) ^ 1u, abort, p.status)) break;
       double* mine = red_s + warp * 2 * Cf::PART;
+      float* minef = red_sf + warp * 2 * Cf::PART;
       if constexpr (SP) {
         // tile (mt, nt) holds 8x8 blocks (2 mt, nt) and (2 mt + 1, nt) in the
         // DMMA accumulator layout (row g, columns 2t, 2t + 1); the upper ones
@@ -892,8 +927,8 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
               const int ub = bi * NB - bi * (bi - 1) / 2 + (bj - bi);
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
-                mine[ub * 64 + g * 8 + 2 * t + h] = (double)acc.s1[ti][2 * hh + h];
-                mine[Cf::PART + ub * 64 + g * 8 + 2 * t + h] = (double)acc.s2[ti][2 * hh + h];
+                minef[ub * 64 + g * 8 + 2 * t + h] = acc.s1[ti][2 * hh + h];
+                minef[Cf::PART + ub * 64 + g * 8 + 2 * t + h] = acc.s2[ti][2 * hh + h];
               }
             }
 #pragma unroll
@@ -941,7 +976,8 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
       for (int i = tid; i < 2 * Cf::PART; i += 32 * CW) {
         double s = 0.0;
 #pragma unroll
-        for (int w = 0; w < CW; ++w) s += red_s[w * 2 * Cf::PART + i];
+        for (int w = 0; w < CW; ++w)
+          s += SP ? (double)red_sf[w * 2 * Cf::PART + i] : red_s[w * 2 * Cf::PART + i];
         dst[i] = s;
       }
       if (cond)
@@ -961,14 +997,17 @@ __global__ void __launch_bounds__(GramBulk<RP, TG, TM>::BT, GramBulk<RP, TG, TM>
 // ===========================================================================
 // thin_apply_bulk: O = C^2 T B, W update, long-side energies
 // ===========================================================================
-template <int RP, typename TG, typename TM, typename TW>
+// SP: the split bf16 tensor-core apply (r = 32, bf16 tensor-core mode): six
+// consumer warps, one 16-column step each per stage of 96 columns, three
+// stages, two CTAs per SM.
+template <int RP, typename TG, typename TM, typename TW, bool SP = false>
 struct ApplyBulk {
-  static constexpr int CW = RP == 32 ? 4 : 8;
+  static constexpr int CW = SP ? 6 : RP == 32 ? 4 : 8;
   static constexpr int NP = 2;                 // producer warps
   static constexpr int BT = 32 * (CW + NP);
-  static constexpr int MINB = RP == 8 || RP == 2 || RP == 32 ? 2 : 1;  // resident CTAs
-  static constexpr int CH = RP <= 4 ? 1024 : RP <= 16 ? 256 : 128;
-  static constexpr int NS = RP == 32 ? 3 : 4;
+  static constexpr int MINB = SP || RP == 8 || RP == 2 || RP == 32 ? 2 : 1;  // resident CTAs
+  static constexpr int CH = SP ? 96 : RP <= 4 ? 1024 : RP <= 16 ? 256 : 128;
+  static constexpr int NS = SP || RP == 32 ? 3 : 4;
   static constexpr int PM = pitch_elems<TM>(CH), PG = pitch_elems<TG>(CH), PW = pitch_elems<TW>(CH);
   static constexpr int OFF_W = opnd_bytes<TM>(RP, CH);
   static constexpr int OFF_E = OFF_W + opnd_bytes<TW>(RP, CH);
@@ -1231,7 +1270,7 @@ __device__ __forceinline__ void load_split_t(SplitT<RP>& f, const double* Tg, in
     }
 }
 
-// 32 long-side columns c .. c + 31 as four 8-column tiles.  For tile nt,
+// 16 long-side columns c .. c + 15 as two 8-column tiles.  For tile nt,
 // lane (g, t) supplies column c + 8 nt + g at rows 16 kt + {2t, 2t + 1,
 // 2t + 8, 2t + 9} (the B fragment) and receives O rows 16 mt + g, + 8 at
 // columns c + 8 nt + 2t, + 1.
@@ -1242,11 +1281,11 @@ __device__ __forceinline__ void apply_step_split(const SplitT<RP>& tf, const TM*
                                                  float* ecg, int64_t n, int cs, int c, int c1,
                                                  float mu, float lr, float decay, bool zero, int g,
                                                  int t) {
-  using L = ApplyBulk<RP, TG, TM, TW>;
+  using L = ApplyBulk<RP, TG, TM, TW, true>;
   constexpr int MT = SplitT<RP>::MT, KT = SplitT<RP>::KT;
   const int off[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
+  for (int nt = 0; nt < 2; ++nt) {
     const int jl = 8 * nt + g;
     const bool okj = FULL || c + jl < c1;
     const float w = ON ? (float)wrow[jl] : 1.f;  // zero past c1
@@ -1340,18 +1379,18 @@ __device__ __forceinline__ void apply_stage_split(const SplitT<RP>& tf, const TM
                                                   int c1, float mu, float lr, float decay,
                                                   float inv_mc, float eps, bool zero, int warp,
                                                   int lane) {
-  using L = ApplyBulk<RP, TG, TM, TW>;
+  using L = ApplyBulk<RP, TG, TM, TW, true>;
   constexpr int CW = L::CW;
   const int g = lane >> 2, t = lane & 3;
-  if (ON) stage_weights<32, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
+  if (ON) stage_weights<16, CW, L::NCOL>(wmine, Es, c0, c1, warp, lane, inv_mc, eps);
   int k = 0;
-  for (int c = c0 + 32 * warp; c < c1; c += 32 * CW, ++k) {
-    if (c + 32 <= c1)
-      apply_step_split<RP, TG, TM, TW, TALL, ON, COND, true, NEST>(tf, Ms, Gs, Ws, wmine + 32 * k, Wg,
+  for (int c = c0 + 16 * warp; c < c1; c += 16 * CW, ++k) {
+    if (c + 16 <= c1)
+      apply_step_split<RP, TG, TM, TW, TALL, ON, COND, true, NEST>(tf, Ms, Gs, Ws, wmine + 16 * k, Wg,
                                                                    Ug, ecg, n, c - c0, c, c1, mu, lr,
                                                                    decay, zero, g, t);
     else
-      apply_step_split<RP, TG, TM, TW, TALL, ON, COND, false, NEST>(tf, Ms, Gs, Ws, wmine + 32 * k, Wg,
+      apply_step_split<RP, TG, TM, TW, TALL, ON, COND, false, NEST>(tf, Ms, Gs, Ws, wmine + 16 * k, Wg,
                                                                     Ug, ecg, n, c - c0, c, c1, mu, lr,
                                                                     decay, zero, g, t);
   }
@@ -1396,9 +1435,9 @@ struct SplitTOf<RP, true> {
 };
 
 template <int RP, typename TG, typename TM, typename TW, bool SP>
-__global__ void __launch_bounds__(ApplyBulk<RP, TG, TM, TW>::BT, ApplyBulk<RP, TG, TM, TW>::MINB)
+__global__ void __launch_bounds__(ApplyBulk<RP, TG, TM, TW, SP>::BT, ApplyBulk<RP, TG, TM, TW, SP>::MINB)
     thin_apply_bulk(const __grid_constant__ ThinParams p) {
-  using L = ApplyBulk<RP, TG, TM, TW>;
+  using L = ApplyBulk<RP, TG, TM, TW, SP>;
   constexpr int CH = L::CH, NS = L::NS, CW = L::CW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
@@ -1510,8 +1549,8 @@ int resident(K kernel, int threads, int smem) {
 
 template <int RP, typename TG, typename TM, typename TW, bool SP>
 cudaError_t launch_bulk_sp(ThinParams& p, int nsm, cudaStream_t st) {
-  using LG = GramBulk<RP, TG, TM>;
-  using LA = ApplyBulk<RP, TG, TM, TW>;
+  using LG = GramBulk<RP, TG, TM, SP>;
+  using LA = ApplyBulk<RP, TG, TM, TW, SP>;
   static DeviceOnce once;
   static int occ_g[MAX_DEVICES], occ_a[MAX_DEVICES][2];
   int dev = 0;
