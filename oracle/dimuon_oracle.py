@@ -156,8 +156,28 @@ def store_round(x, dtype: str) -> np.ndarray:
 # Method steps.
 # ----------------------------------------------------------------------------
 def momentum_update(M_prev, G, mu: float) -> np.ndarray:
-    """M_t = mu * M_{t-1} + grad ([MuonNote], "Update rule", eq. (1))."""
-    return mu * np.asarray(M_prev, np.float64) + np.asarray(G, np.float64)
+    """M_t = mu * M_{t-1} + grad ([MuonNote], "Update rule", eq. (1)).
+
+    The stored momentum is the exact value of mu M_{t-1} + G rounded once to
+    its storage type.  mu, M_{t-1} and G are float32 (or bf16) values, so the
+    product is exact in float64 and the sum is exact as the float64 pair
+    (s, e) of a two-sum.  The value returned is s rounded to odd with e as
+    the sticky part: s itself when e = 0, else whichever of s and its float64
+    neighbour on the side of e has an odd last bit.  With at least two more
+    bits than the storage type, one later round-to-nearest-even to float32 or
+    bf16 of this value is the correctly rounded exact value (rounding to odd
+    carries the information a second rounding needs); rounding the float64
+    sum s directly would round twice."""
+    M_prev = np.asarray(M_prev, np.float64)
+    G = np.asarray(G, np.float64)
+    p = mu * M_prev                      # exact: 24-bit times 24-bit significands
+    s = p + G
+    bb = s - p
+    e = (p - (s - bb)) + (G - bb)        # s + e = p + G exactly (two-sum)
+    inexact = (e != 0.0) & np.isfinite(s)
+    odd = (s.view(np.int64) & 1) == 1
+    toward = np.nextafter(s, np.where(e > 0.0, np.inf, -np.inf))
+    return np.where(inexact & ~odd, toward, s)
 
 
 def energies(M) -> tuple[np.ndarray, np.ndarray]:

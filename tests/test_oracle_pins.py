@@ -338,19 +338,99 @@ def test_step_brute_force(shape, moonshot, wd):
             np.testing.assert_allclose(got.e_col, (Mt ** 2).sum(0), rtol=1e-12)
 
 
-def test_momentum_brute_force_bf16():
-    rng = np.random.default_rng(1)
-    M = orc.round_bf16(rng.standard_normal((4, 16)))
-    G = orc.round_bf16(rng.standard_normal((4, 16)))
-    mu = float(np.float32(0.95))
-    got = orc.store_round(orc.momentum_update(M, G, mu), "bf16")
-    for i in range(4):
-        for j in range(16):
-            v = float(torch.tensor(mu * M[i, j] + G[i, j], dtype=torch.float64)
-                      .float().bfloat16().float())
-            # fp64 -> bf16 directly may differ from fp64->fp32->bf16 only on a
-            # double-rounding tie; none occurs in this fixed draw
-            assert got[i, j] == v
+def exact_round(x, bits, qmin, maxval):
+    """Nearest binary float with `bits` significand bits to the rational x
+    (ties to even; quantum never below 2^qmin; beyond maxval -> inf), by
+    exact integer arithmetic."""
+    from fractions import Fraction
+    x = Fraction(x)
+    if x == 0:
+        return 0.0
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1                                   # 2^e <= a < 2^(e+1)
+    q = Fraction(2) ** max(e - bits + 1, qmin)
+    n = a / q
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    v = fl * q
+    out = math.inf if v > maxval else float(v)
+    return out if x > 0 else -out
+
+
+FP32_FMT = (24, -149, (2 - 2.0 ** -23) * 2.0 ** 127)
+BF16_FMT = (8, -133, (2 - 2.0 ** -7) * 2.0 ** 127)
+
+
+def exact_momentum(mu, m, g, fmt):
+    from fractions import Fraction
+    return exact_round(Fraction(mu) * Fraction(m) + Fraction(g), *fmt)
+
+
+def double_rounded_momentum(mu, m, g, dtype):
+    """The float64 sum rounded again to the storage type (two roundings)."""
+    v = np.float64(mu) * np.float64(m) + np.float64(g)
+    return float(orc.store_round(v, dtype))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_momentum_is_the_correctly_rounded_exact_value(dtype):
+    """[MuonNote] 'Update rule', eq. (1): M_t = mu M_{t-1} + G, stored once.
+    Brute force with exact rational arithmetic over random draws whose
+    magnitudes differ by up to 2^60 (where the float64 sum itself rounds)."""
+    rng = np.random.default_rng(11)
+    fmt = BF16_FMT if dtype == "bf16" else FP32_FMT
+    n = 400
+    M = rng.standard_normal(n) * np.exp2(rng.integers(-30, 30, n))
+    G = rng.standard_normal(n) * np.exp2(rng.integers(-30, 30, n))
+    M = orc.store_round(M, dtype)
+    G = orc.store_round(G, dtype)
+    for mu in (float(np.float32(0.95)), float(np.float32(0.9)), 0.75):
+        got = orc.store_round(orc.momentum_update(M, G, mu), dtype)
+        for i in range(n):
+            assert got[i] == exact_momentum(mu, M[i], G[i], fmt), (mu, M[i], G[i])
+
+
+def crafted_fp32_tie():
+    """mu, m, g (float32 values, 0.5 <= mu < 1) with mu m = 2^-24 (1 - d 2^-47),
+    0 < d < 2^18, and g = 1 + 2^-23: the float64 sum is exactly the float32
+    midpoint 1 + 2^-23 + 2^-24 (its ties-to-even neighbour is 1 + 2^-22),
+    while the exact value lies just below it (nearest: 1 + 2^-23)."""
+    for a in range(2 ** 24 - 1, 2 ** 23, -1):
+        b = 2 ** 47 // a
+        d = 2 ** 47 - a * b
+        if 0 < d < 2 ** 18 and 2 ** 23 <= b < 2 ** 24:
+            return a / 2.0 ** 24, b / 2.0 ** 47, 1.0 + 2.0 ** -23
+    raise AssertionError("no crafted case")
+
+
+def crafted_bf16_tie():
+    """mu = 0.75 and a bf16 m with mu m exactly a bf16 midpoint (odd k), and a
+    gradient 2^-80 of it pushing the exact value off the midpoint towards the
+    odd neighbour: the float64 sum rounds back onto the midpoint."""
+    m = 1.0 + 1.0 / 128
+    p = 0.75 * m                        # 0.7575...: a tie at bf16 precision
+    lo = float(orc.round_bf16(np.float64(p) - 2.0 ** -12))
+    down_is_even = orc.round_bf16(np.float64(p)) == lo
+    g = (2.0 ** -80) * (1.0 if down_is_even else -1.0)
+    return 0.75, m, g
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_momentum_double_rounding_case(dtype):
+    """A constructed case where rounding the float64 sum to the storage type
+    differs from rounding the exact value: the oracle gives the latter."""
+    mu, m, g = crafted_fp32_tie() if dtype == "fp32" else crafted_bf16_tie()
+    fmt = FP32_FMT if dtype == "fp32" else BF16_FMT
+    for v in (mu, m, g):
+        assert float(orc.store_round(v, "fp32")) == v   # all float32 values
+    exact = exact_momentum(mu, m, g, fmt)
+    assert double_rounded_momentum(mu, m, g, dtype) != exact
+    got = orc.store_round(orc.momentum_update(np.array([m]), np.array([g]), mu), dtype)
+    assert got[0] == exact
 
 
 def test_first_step_dimuon_equals_muon():
