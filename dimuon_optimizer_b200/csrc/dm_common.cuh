@@ -31,12 +31,19 @@ __device__ __forceinline__ float round_to(float v, int dt) {
   return dt == DT_BF16 ? __bfloat162float(__float2bfloat16_rn(v)) : v;
 }
 
-// M_t = mu M_{t-1} + G evaluated in fp64 and rounded once to the storage
-// dtype.  The product of an fp32 and a bf16 / fp32 value is exact in fp64, so
-// this is the correctly rounded momentum (no fp32 -> bf16 double rounding).
+// M_t = mu M_{t-1} + G: the exact value rounded once to the storage dtype
+// ("Muon Optimizer 정리", Update rule, eq. (1)).  fp32 storage: one fused
+// multiply-add rounds the exact value to nearest.  bf16 storage: the two
+// directed-rounding FMAs bracket the exact value; when they differ, the one
+// with an odd last bit is the value rounded to odd at fp32 precision, and
+// with 16 more bits than bf16 one rounding of it to nearest-even bf16 is the
+// correctly rounded exact value (rounding to odd keeps the sticky
+// information a second rounding needs).
 __device__ __forceinline__ float momentum_value(float mu, float mprev, float g, int dt) {
-  const double v = fma((double)mu, (double)mprev, (double)g);
-  return dt == DT_BF16 ? __bfloat162float(__double2bfloat16(v)) : __double2float_rn(v);
+  if (dt != DT_BF16) return __fmaf_rn(mu, mprev, g);
+  const float lo = __fmaf_rd(mu, mprev, g), hi = __fmaf_ru(mu, mprev, g);
+  const float odd = (__float_as_uint(lo) & 1u) ? lo : hi;
+  return __bfloat162float(__float2bfloat16_rn(lo == hi ? hi : odd));  // hi: +0 for an exact 0
 }
 
 // Squared Frobenius norms below this floor give a zero update (fp32 cannot

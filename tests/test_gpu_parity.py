@@ -16,6 +16,7 @@ import torch
 import dimuon_optimizer_b200 as dm
 import oracle as orc
 import workloads
+from rounding_cases import crafted_bf16_tie, crafted_fp32_tie
 from gpu_harness import (TOL_BF16, TOL_FP32, TOL_THIN_SPLIT_ILL, Group, oracle_hp, rel_fro,
                          run_gpu_step, step_and_compare, thin_tol, to_dev, to_host)
 
@@ -376,6 +377,39 @@ def test_lora_batch_twenty_steps(r, path):
             # R = (0 + eps)^(-1/4) = 10 on each side of X_5: O gains R^2 = 100
             assert abs(gain / 100.0 - 1.0) < 1e-3, gain
     assert rel_fro(to_host(grp.W[1]), free["W"]) < 3e-2
+
+
+# tensor-core path (K1), fp32 path, thin staged / cluster / register kernels
+ROUNDING_SHAPES = [(64, 96), (8, 512), (512, 8), (2, 512), (32, 256), (8, 24), (5, 40)]
+
+
+@pytest.mark.parametrize("mdt", [BF, F32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize("prec", [dm.DM_PREC_BF16_TC, dm.DM_PREC_FP32], ids=["tc", "fp32"])
+def test_momentum_rounds_the_exact_value_once(mdt, prec):
+    """Inputs built so that rounding the float64 sum mu M + G to the storage
+    type would round twice and differ from the exact value rounded once
+    ("Muon Optimizer 정리", Update rule, eq. (1)): every kernel that forms
+    M_t stores the correctly rounded value, bit-equal to the oracle."""
+    mu, m, g = crafted_bf16_tie() if mdt == BF else crafted_fp32_tie()
+    # (W, G, M) all bf16 or all fp32: storage combinations of every thin kernel
+    grp = Group(ROUNDING_SHAPES, mdt, mdt, mdt, cond=False, seed=61)
+    rng = np.random.default_rng(62)
+    grads = []
+    for i, s in enumerate(ROUNDING_SHAPES):
+        M0 = rng.standard_normal(s)
+        G0 = rng.standard_normal(s)
+        M0.flat[::7] = m
+        G0.flat[::7] = g
+        grp.M[i].copy_(to_dev(M0, mdt))
+        grads.append(G0)
+    hp = hparams(prec, mu=mu)
+    step_and_compare(grp, grads, hp, TOL_BF16 if prec == dm.DM_PREC_BF16_TC else TOL_FP32,
+                     check_sv=False)
+    # the constructed entries took the exact value's rounding
+    want = orc.store_round(orc.momentum_update(np.array([m]), np.array([g]), np.float32(mu)),
+                           "bf16" if mdt == BF else "fp32")[0]
+    for i in range(len(ROUNDING_SHAPES)):
+        assert np.all(to_host(grp.M[i]).flat[::7] == want)
 
 
 def dead_row_gain(O, M, e_prev, dead, eps):

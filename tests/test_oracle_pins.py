@@ -14,6 +14,7 @@ import torch
 
 import oracle as orc
 import workloads
+from rounding_cases import crafted_bf16_tie, crafted_fp32_tie
 
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
@@ -392,31 +393,6 @@ def test_momentum_is_the_correctly_rounded_exact_value(dtype):
         got = orc.store_round(orc.momentum_update(M, G, mu), dtype)
         for i in range(n):
             assert got[i] == exact_momentum(mu, M[i], G[i], fmt), (mu, M[i], G[i])
-
-
-def crafted_fp32_tie():
-    """mu, m, g (float32 values, 0.5 <= mu < 1) with mu m = 2^-24 (1 - d 2^-47),
-    0 < d < 2^18, and g = 1 + 2^-23: the float64 sum is exactly the float32
-    midpoint 1 + 2^-23 + 2^-24 (its ties-to-even neighbour is 1 + 2^-22),
-    while the exact value lies just below it (nearest: 1 + 2^-23)."""
-    for a in range(2 ** 24 - 1, 2 ** 23, -1):
-        b = 2 ** 47 // a
-        d = 2 ** 47 - a * b
-        if 0 < d < 2 ** 18 and 2 ** 23 <= b < 2 ** 24:
-            return a / 2.0 ** 24, b / 2.0 ** 47, 1.0 + 2.0 ** -23
-    raise AssertionError("no crafted case")
-
-
-def crafted_bf16_tie():
-    """mu = 0.75 and a bf16 m with mu m exactly a bf16 midpoint (odd k), and a
-    gradient 2^-80 of it pushing the exact value off the midpoint towards the
-    odd neighbour: the float64 sum rounds back onto the midpoint."""
-    m = 1.0 + 1.0 / 128
-    p = 0.75 * m                        # 0.7575...: a tie at bf16 precision
-    lo = float(orc.round_bf16(np.float64(p) - 2.0 ** -12))
-    down_is_even = orc.round_bf16(np.float64(p)) == lo
-    g = (2.0 ** -80) * (1.0 if down_is_even else -1.0)
-    return 0.75, m, g
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
