@@ -618,9 +618,9 @@ dm_status_t run_body(const dm_matrix_t* mats, int n, const dm_hparams_t* hp, con
     tp.nesterov = hp->nesterov;
     tp.ns_steps = hp->ns_steps;
     // bf16 tensor-core mode: the staged r = 32 passes take their sums on
-    // bf16 tensor cores (split operands, fp32 accumulation); fp32 mode keeps
-    // the fp64 sums
-    tp.split = L.tc && tl.pad == 32 ? 1 : 0;
+    // bf16 tensor cores (split operands, fp32 accumulation) and the r x r
+    // iteration in fp32; fp32 mode and the register path keep fp64
+    tp.split = L.tc && tl.pad == 32 && tl.combo >= 0 && !tl.fused && !tl.cs ? 1 : 0;
     tp.mu = hp->mu;
     tp.lr = hp->lr;
     tp.decay = decay;

@@ -313,7 +313,15 @@ __device__ __forceinline__ void staged_epilogue32(const GemmMat& g, float lr, fl
 struct AuxPrefetch {
   float row[32];
   uint4 blk[4];
+  float S, valid;  // the product's scalars (written by an earlier launch)
 };
+
+// The product's scalars, loaded with the first aux block before the wait on
+// the accumulator.
+__device__ __forceinline__ void fetch_scalars(const GemmMat& g, AuxPrefetch& pf) {
+  pf.S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
+  pf.valid = g.scal ? g.scal[SC_VALID] : 1.f;
+}
 
 __device__ __forceinline__ void fetch_aux(const GemmMat& g, int r, bool row_ok, int col0, int ch,
                                           int ch_end, int nch, AuxPrefetch& pf) {
@@ -329,9 +337,9 @@ __device__ __forceinline__ void fetch_aux(const GemmMat& g, int r, bool row_ok, 
 
 // Epilogue of chunks [ch_begin, ch_end) (32 columns each) of one accumulator
 // row: tcgen05.ld of each chunk, with the next chunk's aux in flight while
-// the current one is processed.  `pf` holds chunk ch_begin's aux, fetched by
-// the caller (fetch_aux) before it waited for the accumulator, since the aux
-// does not depend on it.  Must be executed by all 32 lanes of the warp
+// the current one is processed.  `pf` holds chunk ch_begin's aux and the
+// scalars, fetched by the caller (fetch_aux, fetch_scalars) before it waited
+// for the accumulator, since they do not depend on it.  Must be executed by all 32 lanes of the warp
 // (tcgen05.ld is warp-collective); rows outside the matrix only skip stores.
 // `st` is this warp's staging tile (STAGE_TILE_BYTES of shared memory).
 __device__ __forceinline__ void epilogue_row(const GemmMat& g, float lr, float decay, int r,
@@ -339,8 +347,7 @@ __device__ __forceinline__ void epilogue_row(const GemmMat& g, float lr, float d
                                              int ch_end, int nch, float& sx, float& sy,
                                              __nv_bfloat16* st, AuxPrefetch& pf) {
   const int r0 = r - (int)(threadIdx.x & 31);
-  const float S = g.scal_idx >= 0 ? g.scal[g.scal_idx] : 1.f;
-  const float valid = g.scal ? g.scal[SC_VALID] : 1.f;
+  const float S = pf.S, valid = pf.valid;
   const bool aux = needs_aux(g.epi);
 #pragma unroll 1
   for (int ch = ch_begin; ch < ch_end; ++ch) {

@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ns_product(const __grid_con
       constexpr int CH_PER = TC_BN / 32 / 2;
       // the first chunk's aux is in flight while the products run
       AuxPrefetch pf;
+      fetch_scalars(g, pf);
       fetch_aux(g, r, r < g.M, tl.tn * TC_BN, half * CH_PER, half * CH_PER + CH_PER, nch, pf);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort, p.status, WAIT_LIMIT_NS)) break;
       tc_fence_after();

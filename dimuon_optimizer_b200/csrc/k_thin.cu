@@ -416,10 +416,21 @@ __device__ __forceinline__ float sum_slabs_f(const float* base, size_t stride, i
   return e;
 }
 
+// Shared matrices of the one-CTA-per-factor iteration, in fp64, or in fp32
+// when the Gram sums came from the split bf16 tensor-core path (their
+// ~2^-16 relative error is far above fp32's, so fp64 buys nothing there).
+template <int RP, typename T>
+struct IterLd {
+  static constexpr int V = TCfg<RP>::SLD;
+};
 template <int RP>
+struct IterLd<RP, float> {
+  static constexpr int V = RP + 2;  // even: float2 rows
+};
+template <int RP, typename T = double>
 struct IterSmem {
-  double G[RP][TCfg<RP>::SLD], H[RP][TCfg<RP>::SLD], P[RP][TCfg<RP>::SLD],
-      A[RP][TCfg<RP>::SLD], Q[RP][TCfg<RP>::SLD], S[RP][TCfg<RP>::SLD];
+  static constexpr int LD = IterLd<RP, T>::V;
+  T G[RP][LD], H[RP][LD], P[RP][LD], A[RP][LD], Q[RP][LD], S[RP][LD];
   double R[RP];
   double red[32];
 };
@@ -427,6 +438,29 @@ struct IterSmem {
 // Threads of the one-CTA-per-factor iteration (RP = 16, 32).
 constexpr int IT = 256;
 constexpr int IW = IT / 32;
+
+// C = A * B for RP x RP fp32 matrices in shared memory: each thread forms
+// 2 x 2 outputs (rows 2i, 2i + 1; columns 2j, 2j + 1) with fp32 FMAs.
+template <int RP>
+__device__ __forceinline__ void mm(float (*C)[RP + 2], float (*A)[RP + 2], float (*B)[RP + 2]) {
+  constexpr int NBJ = RP / 2, NBLK = NBJ * NBJ;
+  for (int blk = threadIdx.x; blk < NBLK; blk += IT) {
+    const int i = 2 * (blk / NBJ), j = 2 * (blk % NBJ);
+    float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < RP; ++k) {
+      const float a0 = A[i][k], a1 = A[i + 1][k];
+      const float2 b = *reinterpret_cast<const float2*>(&B[k][j]);
+      c00 = fmaf(a0, b.x, c00);
+      c01 = fmaf(a0, b.y, c01);
+      c10 = fmaf(a1, b.x, c10);
+      c11 = fmaf(a1, b.y, c11);
+    }
+    *reinterpret_cast<float2*>(&C[i][j]) = make_float2(c00, c01);
+    *reinterpret_cast<float2*>(&C[i + 1][j]) = make_float2(c10, c11);
+  }
+  __syncthreads();
+}
 
 // C = A * B for RP x RP fp64 matrices in shared memory (padded rows); each
 // warp interleaves the k chains of its 8x8 output blocks.
@@ -540,12 +574,12 @@ __global__ void __launch_bounds__(TT) thin_iterate_warp(const __grid_constant__ 
   }
 }
 
-template <int RP>
+template <int RP, typename T>
 __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinParams p) {
   if (step_aborted(p.status)) return;  // an earlier launch of this step timed out
   using Cf = TCfg<RP>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  IterSmem<RP>& s = *reinterpret_cast<IterSmem<RP>*>(smem_raw);
+  IterSmem<RP, T>& s = *reinterpret_cast<IterSmem<RP, T>*>(smem_raw);
   const int tid = threadIdx.x;
   const int f = blockIdx.x;
   const ThinMat mt = p.mats[f];  // by value: stores cannot alias it
@@ -603,11 +637,11 @@ __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinP
   }
   __syncthreads();
   for (int it = 0; it < p.ns_steps; ++it) {
-    const double a = p.coef[it][0], b = p.coef[it][1], c = p.coef[it][2];
+    const T a = p.coef[it][0], b = p.coef[it][1], c = p.coef[it][2];
     mm<RP>(s.Q, s.A, s.A);  // Q = A A
     for (int idx = tid; idx < RP * RP; idx += IT) {
       const int i = idx / RP, j = idx % RP;
-      s.Q[i][j] = c * s.Q[i][j] + b * s.A[i][j] + (i == j ? a : 0.0);
+      s.Q[i][j] = c * s.Q[i][j] + b * s.A[i][j] + (i == j ? a : T(0));
     }
     __syncthreads();
     mm<RP>(s.S, s.Q, s.P);  // P <- Q P
@@ -619,13 +653,14 @@ __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinP
   // ||X_5||^2 s^2 = tr(P A_0 P^T); ||R X_5 C||^2 s^2 = sum_i R_i^2 (P H P^T)_ii
   mm<RP>(s.S, s.P, s.G);
   double nx = 0.0;
-  for (int idx = tid; idx < RP * RP; idx += IT) nx += s.S[idx / RP][idx % RP] * s.P[idx / RP][idx % RP];
+  for (int idx = tid; idx < RP * RP; idx += IT)
+    nx += (double)s.S[idx / RP][idx % RP] * (double)s.P[idx / RP][idx % RP];
   nx = block_sum_d(nx, s.red);
   mm<RP>(s.Q, s.P, s.H);
   double ny = 0.0;
   for (int idx = tid; idx < RP * RP; idx += IT) {
     const int i = idx / RP;
-    ny += s.R[i] * s.R[i] * s.Q[i][idx % RP] * s.P[i][idx % RP];
+    ny += s.R[i] * s.R[i] * (double)s.Q[i][idx % RP] * (double)s.P[i][idx % RP];
   }
   ny = block_sum_d(ny, s.red);
   double factor = 0.0;
@@ -636,7 +671,7 @@ __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinP
   if (!finite && tid == 0) raise_status(p.status, ST_NONFINITE);
   // T = f R P R; for RP >= 8 in MMA fragment order: T(8 bo + l/4, 4 kb + l%4)
   // at ((bo * KB + kb) * 32 + l)
-  double* T = p.T + (size_t)f * RP * RP;
+  double* Tm = p.T + (size_t)f * RP * RP;
   for (int idx = tid; idx < RP * RP; idx += IT) {
     int i, j;
     if constexpr (Cf::MMA) {
@@ -648,7 +683,7 @@ __global__ void __launch_bounds__(IT) thin_iterate(const __grid_constant__ ThinP
       i = idx / RP;
       j = idx % RP;
     }
-    T[idx] = factor * s.R[i] * s.P[i][j] * s.R[j];
+    Tm[idx] = factor * s.R[i] * (double)s.P[i][j] * s.R[j];
   }
   if (tid == 0) {
     p.fsc[4 * f + 2] = on ? 1.0 : 0.0;
@@ -1248,21 +1283,29 @@ int resident_ctas(K kernel, int smem) {
   return occ;
 }
 
+template <int RP, typename T>
+cudaError_t launch_iter_t(const ThinParams& p, cudaStream_t st) {
+  const int iter_bytes = (int)sizeof(IterSmem<RP, T>);
+  static DeviceOnce once;
+  const cudaError_t e = device_once(once, nullptr, [&](int) {
+    return cudaFuncSetAttribute(thin_iterate<RP, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                iter_bytes);
+  });
+  if (e != cudaSuccess) return e;
+  thin_iterate<RP, T><<<p.count, IT, iter_bytes, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <int RP>
 cudaError_t launch_iter_rp(const ThinParams& p, cudaStream_t st) {
   if constexpr (RP <= 8) {
     thin_iterate_warp<RP><<<(p.count + TW - 1) / TW, TT, 0, st>>>(p);
     return cudaGetLastError();
+  } else {
+    // the split-sum passes (bf16 tensor-core mode) feed an fp32 iteration
+    if (p.split) return launch_iter_t<RP, float>(p, st);
+    return launch_iter_t<RP, double>(p, st);
   }
-  const int iter_bytes = (int)sizeof(IterSmem<RP>);
-  static DeviceOnce once;
-  const cudaError_t e = device_once(once, nullptr, [&](int) {
-    return cudaFuncSetAttribute(thin_iterate<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                iter_bytes);
-  });
-  if (e != cudaSuccess) return e;
-  thin_iterate<RP><<<p.count, IT, iter_bytes, st>>>(p);
-  return cudaGetLastError();
 }
 
 template <int RP>
