@@ -133,16 +133,18 @@ def test_thin_path(cond, mdt, path):
                                  thin_tol(True), ws=ws)
 
 
+@pytest.mark.parametrize("prec", [dm.DM_PREC_FP32, dm.DM_PREC_BF16_TC], ids=["fp32", "bf16"])
 @pytest.mark.parametrize("cond", [False, True])
-def test_thin_path_fp32_storage(cond):
-    """fp32 gradients, momentum and weights (the third staged combination)."""
-    shapes = [(8, 512), (512, 16), (32, 256), (4, 96), (2, 40)]
+def test_thin_path_fp32_storage(cond, prec):
+    """fp32 gradients, momentum and weights (the third staged combination),
+    with Nesterov; in bf16 mode the rank-32 factors take the split sums."""
+    shapes = [(8, 512), (512, 16), (32, 256), (256, 32), (4, 96), (2, 40)]
     grp = Group(shapes, F32, F32, F32, cond=cond, seed=17)
-    hp = hparams(dm.DM_PREC_FP32, nesterov=1)
+    hp = hparams(prec, nesterov=1)
     ws = None
     for t in range(3):
-        _, ws = step_and_compare(grp, gaussian(shapes, 700 + t, scale_cols=True), hp, TOL_FP32,
-                                 ws=ws)
+        _, ws = step_and_compare(grp, gaussian(shapes, 700 + t, scale_cols=True), hp,
+                                 thin_tol(prec == dm.DM_PREC_BF16_TC), ws=ws)
 
 
 def test_thin_threshold_hook_matches_ns_path():
@@ -162,14 +164,20 @@ def test_thin_threshold_hook_matches_ns_path():
 def test_nesterov(prec, tol, cond):
     """B_t = G + mu M_t feeds the orthogonaliser on every path (Newton-Schulz
     and thin)."""
-    shapes = [(200, 330), (330, 200), (8, 600), (600, 16)]
+    shapes = [(200, 330), (330, 200), (8, 600), (600, 16), (32, 600), (600, 32)]
     grp = Group(shapes, BF, BF, F32, cond=cond, seed=21)
     hp = hparams(prec, nesterov=1, weight_decay=0.02)
     ws = None
+    thin = thin_tol(prec == dm.DM_PREC_BF16_TC)
+
+    def tol_of(shape):  # Newton-Schulz matrices at the mode's tolerance, thin factors at theirs
+        if min(shape) > 32:
+            return tol
+        return thin(shape) if callable(thin) else thin
+
     for t in range(3):
-        thin_tol = [tol, tol, TOL_FP32, TOL_FP32]
-        _, ws = step_and_compare(grp, gaussian(shapes, 900 + t, scale_cols=True), hp,
-                                 max(thin_tol), ws=ws)
+        _, ws = step_and_compare(grp, gaussian(shapes, 900 + t, scale_cols=True), hp, tol_of,
+                                 ws=ws)
 
 
 @pytest.mark.parametrize("prec,tol", [(dm.DM_PREC_FP32, TOL_FP32), (dm.DM_PREC_BF16_TC, TOL_BF16)])
