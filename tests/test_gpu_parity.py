@@ -210,10 +210,13 @@ def test_first_dimuon_step_equals_muon():
 
 
 def test_nonfinite_gradient_reports_and_only_decays():
-    shapes = [(64, 128), (8, 256)]
+    # Newton-Schulz, thin (fp64 sums) and rank-32 thin (split sums in bf16 mode)
+    shapes = [(64, 128), (8, 256), (32, 256), (256, 32)]
     g = gaussian(shapes, 800)
     g[0][3, 5] = np.inf
     g[1][2, 7] = np.nan
+    g[2][30, 200] = -np.inf
+    g[3][100, 31] = np.nan
     grp = Group(shapes, F32, F32, F32, cond=False, seed=18)
     W0 = [to_host(w) for w in grp.W]
     hp = hparams(dm.DM_PREC_BF16_TC, weight_decay=0.5, lr=0.1)
@@ -230,7 +233,7 @@ def test_nonfinite_gradient_reports_and_only_decays():
 
 
 def test_zero_gradient_gives_zero_update():
-    shapes = [(64, 128), (4, 64)]
+    shapes = [(64, 128), (4, 64), (32, 96), (96, 32)]
     for prec in (dm.DM_PREC_FP32, dm.DM_PREC_BF16_TC):
         for cond in (False, True):
             grp = Group(shapes, F32, F32, F32, cond=cond, seed=19)
