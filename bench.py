@@ -74,6 +74,9 @@ def workload_spec(name):
         return dict(shapes=workloads.single_square_shapes(4096), cond=False, mdt="bf16",
                     lr=0.02, wd=0.0, moonshot=False, seed=1,
                     desc="one 4096x4096 bf16 matrix, Muon, 5 NS5 iterations")
+    if name == "toy":  # the 4x16 toy factor; latency-bound, read as microseconds per step
+        return dict(shapes=[(4, 16)], cond=True, mdt="fp32", lr=0.02, wd=0.0, moonshot=False,
+                    seed=0, desc="one 4x16 factor (bf16 W/G, fp32 M), Dimuon; latency-bound")
     if name.startswith("lora_r"):
         r = int(name[6:])
         return dict(shapes=workloads.lora_shapes(r), cond=True, mdt="fp32",

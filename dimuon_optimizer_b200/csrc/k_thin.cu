@@ -417,15 +417,16 @@ __device__ __forceinline__ float sum_slabs_f(const float* base, size_t stride, i
 }
 
 // Shared matrices of the one-CTA-per-factor iteration, in fp64, or in fp32
-// when the Gram sums came from the split bf16 tensor-core path (their
-// ~2^-16 relative error is far above fp32's, so fp64 buys nothing there).
+// (products on tf32 tensor cores with split operands) when the Gram sums
+// came from the split bf16 tensor-core path (their ~2^-16 relative error is
+// far above fp32's, so fp64 buys nothing there).
 template <int RP, typename T>
 struct IterLd {
   static constexpr int V = TCfg<RP>::SLD;
 };
 template <int RP>
 struct IterLd<RP, float> {
-  static constexpr int V = RP + 2;  // even: float2 rows
+  static constexpr int V = RP + 4;  // A-fragment reads on distinct banks; even for float2
 };
 template <int RP, typename T = double>
 struct IterSmem {
@@ -439,25 +440,49 @@ struct IterSmem {
 constexpr int IT = 256;
 constexpr int IW = IT / 32;
 
-// C = A * B for RP x RP fp32 matrices in shared memory: each thread forms
-// 2 x 2 outputs (rows 2i, 2i + 1; columns 2j, 2j + 1) with fp32 FMAs.
+// x = hi + lo with hi, lo tf32 values (round to nearest, ties away: the PTX
+// conversion); hi + lo carries x to about 2^-22 relative.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(x - __uint_as_float(hi)));
+}
+
+// D (16x8, fp32) += A (16x8, tf32) * B (8x8, tf32).  Lane l = 4g + t holds
+// A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]; B[t][g], B[t+4][g]; D rows g
+// and g + 8 at columns 2t, 2t + 1.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// C = A * B for RP x RP fp32 matrices in shared memory on tensor cores: one
+// 16 x 8 output tile per warp, each operand split into tf32 hi + lo and each
+// product taken as hi hi + hi lo + lo hi (fp32-level accuracy).
 template <int RP>
-__device__ __forceinline__ void mm(float (*C)[RP + 2], float (*A)[RP + 2], float (*B)[RP + 2]) {
-  constexpr int NBJ = RP / 2, NBLK = NBJ * NBJ;
-  for (int blk = threadIdx.x; blk < NBLK; blk += IT) {
-    const int i = 2 * (blk / NBJ), j = 2 * (blk % NBJ);
-    float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < RP; ++k) {
-      const float a0 = A[i][k], a1 = A[i + 1][k];
-      const float2 b = *reinterpret_cast<const float2*>(&B[k][j]);
-      c00 = fmaf(a0, b.x, c00);
-      c01 = fmaf(a0, b.y, c01);
-      c10 = fmaf(a1, b.x, c10);
-      c11 = fmaf(a1, b.y, c11);
+__device__ __forceinline__ void mm(float (*C)[RP + 4], float (*A)[RP + 4], float (*B)[RP + 4]) {
+  constexpr int MT = RP / 16, NT = RP / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  for (int tile = warp; tile < MT * NT; tile += IW) {
+    const int i0 = 16 * (tile / NT), j0 = 8 * (tile % NT);
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k0 = 0; k0 < RP; k0 += 8) {
+      uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
+      split_tf32(A[i0 + g][k0 + t], ah[0], al[0]);
+      split_tf32(A[i0 + g + 8][k0 + t], ah[1], al[1]);
+      split_tf32(A[i0 + g][k0 + t + 4], ah[2], al[2]);
+      split_tf32(A[i0 + g + 8][k0 + t + 4], ah[3], al[3]);
+      split_tf32(B[k0 + t][j0 + g], bh0, bl0);
+      split_tf32(B[k0 + t + 4][j0 + g], bh1, bl1);
+      mma_tf32(d, al, bh0, bh1);
+      mma_tf32(d, ah, bl0, bl1);
+      mma_tf32(d, ah, bh0, bh1);
     }
-    *reinterpret_cast<float2*>(&C[i][j]) = make_float2(c00, c01);
-    *reinterpret_cast<float2*>(&C[i + 1][j]) = make_float2(c10, c11);
+    *reinterpret_cast<float2*>(&C[i0 + g][j0 + 2 * t]) = make_float2(d[0], d[1]);
+    *reinterpret_cast<float2*>(&C[i0 + g + 8][j0 + 2 * t]) = make_float2(d[2], d[3]);
   }
   __syncthreads();
 }

@@ -44,7 +44,7 @@ def test_ns_flops_uses_the_short_side():
 @pytest.mark.parametrize("name,count", [
     ("large_batch", 16), ("large_batch_dimuon", 16), ("large_batch_quarter", 4),
     ("gpt2_small", 72), ("square1024", 1), ("square4096", 1), ("lora_r2", 448), ("lora_r8", 448),
-    ("lora_r32", 448), ("vec_w1", 64), ("vec_w32", 64), ("vec_w128", 64)])
+    ("lora_r32", 448), ("vec_w1", 64), ("vec_w32", 64), ("vec_w128", 64), ("toy", 1)])
 def test_workload_table(name, count):
     spec = bench.workload_spec(name)
     assert len(spec["shapes"]) == count
