@@ -10,8 +10,11 @@
 // Two producer warps stream it through a ring of shared-memory stages, taking
 // alternate stages, with 1-D bulk async copies (cp.async.bulk, completion on
 // an mbarrier): the copies of the next stages are in flight while the
-// consumer warps (8, or 4 for r = 32) work on the current one, so the loads
-// need neither registers nor per-lane address arithmetic.  Full steps run
+// consumer warps (8; 4 for r = 32, 6 for r = 32 on the split path) work on
+// the current one, so the loads need neither registers nor per-lane address
+// arithmetic.  Sums: fp64 (FMA for r <= 4, DMMA for r >= 8), or for r = 32 in
+// bf16 tensor-core mode bf16 tensor-core products of hi / lo split operands
+// with fp32 accumulation (the SP kernels).  Full steps run
 // branch-free code specialised on the layout (wide / tall), on whether Dimuon
 // conditioning is on and on whether energies are written; partial steps at a
 // factor's end take a predicated version.  Consumers write their results
@@ -586,7 +589,7 @@ __device__ __forceinline__ void gram_step_small(GramAcc<RP>& acc, const TM* Ms, 
 }
 
 // ---------------------------------------------------------------------------
-// Split bf16 tensor-core sums (RP >= 16, bf16 tensor-core mode).  S_1 and S_2
+// Split bf16 tensor-core sums (RP = 32, bf16 tensor-core mode).  S_1 and S_2
 // are Y Y^T products (K = long-side columns): m16n8k16 tiles with fp32
 // accumulators, each operand split into bf16 hi + lo (three products per
 // tile).  Only the tiles meeting the upper triangle are formed: 16-row tile
@@ -1239,7 +1242,7 @@ __device__ __forceinline__ void apply_step_small(const TM* Ms, const TG* Gs, con
 }
 
 // ---------------------------------------------------------------------------
-// Split bf16 tensor-core apply (RP >= 16, bf16 tensor-core mode): O = T X
+// Split bf16 tensor-core apply (RP = 32, bf16 tensor-core mode): O = T X
 // with X = C^2 B, K = the short side, m16n8k16 tiles, T and X split into
 // bf16 hi + lo.  T's fragments stay in registers while the factor is the
 // same.
