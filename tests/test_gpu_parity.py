@@ -112,7 +112,7 @@ def test_ns_step_counts(ns_steps):
 THIN_SHAPES = [(4, 16), (2, 100), (8, 4096), (4096, 8), (17, 333), (32, 4096), (4096, 32),
                (1, 50), (50, 1), (31, 31), (16, 1000), (2, 2056), (3000, 4), (8, 24),
                (1001, 8), (4099, 16), (777, 32), (13, 8), (2, 5128), (5128, 2), (4, 4096),
-               (4096, 4)]
+               (4096, 4), (32, 1032), (1032, 32)]
 
 
 # default: the cluster kernel for r <= 4 (r = 2 factors whose long side is an
