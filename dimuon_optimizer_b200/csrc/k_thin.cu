@@ -16,8 +16,8 @@
 //   thin_setup   one CTA per factor (up to THIN_MAX per launch): descriptor
 //                into the workspace, sums of the previous energies
 //   thin_gram    persistent CTAs taking slabs of long-side columns from a
-//                device counter: M_t = mu M_{t-1} + G (fp64, one rounding,
-//                stored), the slab's S_1 / S_2 partials (fp64), short-side
+//                device counter: M_t = mu M_{t-1} + G (the exact value rounded
+//                once, stored), the slab's S_1 / S_2 partials (fp64), short-side
 //                energy partials
 //   thin_iterate one CTA per factor: partials summed in slab order, R, the
 //                r x r iteration, T, the new short-side energies
@@ -1060,7 +1060,7 @@ __global__ void __launch_bounds__(TT) thin_apply(const __grid_constant__ ThinPar
 // block-reduced sums go through the r x r iteration on one warp; pass 2
 // applies O = T (C^2 B) to the kept momentum and streams W once, writing the
 // new long-side energies.  Per element the arithmetic is that of thin_gram /
-// thin_apply (fp64 momentum with one rounding, fp64 Gram sums and products);
+// thin_apply (exactly rounded momentum, fp64 Gram sums and products);
 // the HBM traffic is the algorithmic one (G 2, M 4 + 4, W 2 + 2 bytes per
 // element with fp32 momentum), without the two-pass path's second read of
 // M_t, and one launch replaces three.

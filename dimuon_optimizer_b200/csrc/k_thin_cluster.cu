@@ -12,7 +12,7 @@
 //      G and the previous long-side energies at once, so the whole slice is
 //      in flight together, and sums the previous energies (all of them, in
 //      the same order in every CTA of the cluster);
-//   2. pass 1: M_t = mu M_{t-1} + G (fp64, one rounding) in place in shared
+//   2. pass 1: M_t = mu M_{t-1} + G (exact value, one rounding) in place in shared
 //      memory, S_1 / S_2 partial sums (fp64; fp64 tensor-core MMA for r = 8),
 //      short-side energy partials; M_t goes back to global memory by a bulk
 //      store, and the slice of W is fetched into the space G used (unless

@@ -139,7 +139,7 @@ def step_and_compare(grp: Group, grads_host, hp, o_tol, *, ws=None, check_sv=Tru
                                  e_col_prev=ec0, momentum_dtype=sname(grp.mdt),
                                  weight_dtype=sname(grp.wdt))
         Mg, Wg, Og = to_host(grp.M[i]), to_host(grp.W[i]), to_host(grp.upd[i])
-        # momentum: both sides round the fp64 value of mu M + G once -> equal
+        # momentum: both sides round the exact value of mu M + G once -> equal
         dM = np.abs(Mg - res.M)
         rep.m_mismatch.append(int((dM > 0).sum()))
         assert rep.m_mismatch[-1] == 0, (i, dM.max())
