@@ -201,11 +201,33 @@ __device__ __forceinline__ void tile_get_row(const __nv_bfloat16* st, float v[32
 #pragma unroll
   for (int k = 0; k < 4; ++k) ld_bf16x8(st + lane * SP + 8 * k, v + 8 * k);
 }
-// Column `lane` of the tile (the transposed block).
-__device__ __forceinline__ void tile_put_col(__nv_bfloat16* st, const float v[32]) {
+// Transposes the bf16 tile in place: its 16 8x8 blocks are read transposed
+// into registers (ldmatrix .trans, four blocks per instruction; lane 8q + i
+// gives the address of row i of block q), then written back with stmatrix
+// to the mirrored block positions.  Rows are 80 bytes apart, so the eight
+// 16-byte rows of a block fall on distinct banks.
+__device__ __forceinline__ void tile_transpose(__nv_bfloat16* st) {
   const int lane = threadIdx.x & 31;
+  const int q = lane >> 3, i = lane & 7;
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(st));
+  uint32_t f[4][4];  // f[a][b]: block (a, b) of the tile, transposed
 #pragma unroll
-  for (int q = 0; q < 32; ++q) st[q * SP + lane] = __float2bfloat16_rn(v[q]);
+  for (int a = 0; a < 4; ++a) {
+    const uint32_t addr = base + (uint32_t)(((8 * a + i) * SP + 8 * q) * 2);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(f[a][0]), "=r"(f[a][1]), "=r"(f[a][2]), "=r"(f[a][3])
+                 : "r"(addr)
+                 : "memory");
+  }
+  __syncwarp();
+#pragma unroll
+  for (int d = 0; d < 4; ++d) {  // block (d, b) of the transpose is block (b, d) transposed
+    const uint32_t addr = base + (uint32_t)(((8 * d + i) * SP + 8 * q) * 2);
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};"
+                 :
+                 : "r"(addr), "r"(f[0][d]), "r"(f[1][d]), "r"(f[2][d]), "r"(f[3][d])
+                 : "memory");
+  }
 }
 
 // Whether the block of rows r0 .. r0 + 31, columns c0 .. c0 + 31 takes the
@@ -250,10 +272,10 @@ __device__ __forceinline__ void staged_epilogue32(const GemmMat& g, float lr, fl
 #pragma unroll
       for (int q = 0; q < 32; ++q)
         v[q] = g.epi == EPI_SYRK ? v[q] * S : fmaf(g.coef_acc, v[q], g.coef_aux * ax[q]);
-      staged_store(st, out, g.ldo, r0, c0, v);
+      staged_store(st, out, g.ldo, r0, c0, v);  // leaves the bf16 block in the tile
       // the mirrored block: element (c, r) at row c of the output
       uint4 q4[4];
-      tile_put_col(st, v);
+      tile_transpose(st);
       __syncwarp();
       tile_get_blk(st, q4);
       blk_st(out, g.ldo, c0, r0, q4);
