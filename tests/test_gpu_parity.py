@@ -253,7 +253,7 @@ def test_empty_group():
 
 
 def test_cuda_graph_capture_matches_eager():
-    shapes = [(256, 384), (384, 256), (8, 512)]
+    shapes = [(256, 384), (384, 256), (8, 512), (32, 512), (512, 32)]
     g = gaussian(shapes, 900)
     hp = hparams(dm.DM_PREC_BF16_TC)
     eager = Group(shapes, BF, BF, BF, cond=True, seed=20)

@@ -17,7 +17,7 @@ import torch
 import dimuon_optimizer_b200 as dm
 from gpu_harness import TOL_FP32, Group, rel_fro, storage_ulp, to_dev, to_host
 
-SHAPES = [(256, 384), (300, 200), (8, 512), (40, 100)]
+SHAPES = [(256, 384), (300, 200), (8, 512), (40, 100), (32, 256)]
 FOREIGN = [(520, 136), (2, 2056), (64, 96), (4096, 32)]
 
 
